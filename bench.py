@@ -1,0 +1,399 @@
+#!/usr/bin/env python
+"""Benchmark of the SSD layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one ssd_fwd call (every step of the block-decomposition algorithm)
+on the Mamba-2 2.7B layer shape: batch 8, T 2048, 80 heads, head dim 64,
+state 128, 1 group, chunk 256, bf16 x/B/C/y, fp32 dt/A/D, final states
+returned. Inputs are seeded synthetic data resident in HBM; their working set
+(x and y alone are 168 MB each) exceeds the 126 MB L2, so no flush is needed
+between steps. Under torchrun every rank runs its own copy of the workload
+(weak scaling, no collective on the data path) and rank 0 prints one JSON
+line with the whole-job throughput, timed on the device as the max over ranks.
+
+--impl reference times the fp64 CPU oracle on the host cores instead (a
+bounded sample of the same workload per step); it is a deliberately slow
+program, reported for context.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import shutil
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import ssd_inputs as W  # noqa: E402
+
+WORKLOAD = W.MAMBA2_27B_LAYER
+METRIC = "SSD fwd Mtokens/s & TFLOP/s at 2.7B layer shape; % of bf16/HBM roofline"
+UNIT = "Mtokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ counts
+def alg_counts(w: W.Workload, with_final=True, with_init=False):
+    """Algorithmic FLOPs and bytes of one forward (tensor-core flops, causal half).
+
+    F = b T [ G (Q+1) N + H ((Q+1) P + 4 N P + 2 P N / Q) ]
+    Bytes = b T H P (s_x + s_y) + 4 b T H + 2 b T G N s_bc + 8 H + 4 b H P N per state tensor
+    """
+    b, T, H, P, G, N, Q = w.batch, w.seqlen, w.nheads, w.headdim, w.ngroups, w.dstate, w.chunk_size
+    s = 2 if w.dtype == "bf16" else 4
+    F = b * T * (G * (Q + 1) * N + H * ((Q + 1) * P + 4 * N * P + 2 * P * N / Q))
+    by = b * T * H * P * 2 * s + 4 * b * T * H + 2 * b * T * G * N * s + 8 * H
+    by += 4 * b * H * P * N * (int(with_final) + int(with_init))
+    return float(F), float(by)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = None
+        smi = shutil.which("nvidia-smi")
+        if smi is None:
+            return
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            ident = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+        except Exception:
+            ident = str(device_index)
+        self.path = f"/tmp/ssd_bench_clocks_{os.getpid()}.csv"
+        self.fh = open(self.path, "w")
+        self.proc = subprocess.Popen([smi, "-i", ident, f"--query-gpu={self.FIELDS}",
+                                      "--format=csv,noheader,nounits", "-lms", "100"],
+                                     stdout=self.fh, stderr=subprocess.DEVNULL)
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as fh:
+            for line in fh:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 8:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ helpers
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(v: float, world: int, device) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def oracle_sample(w: W.Workload, budget_s: float, inputs64=None):
+    """Prepare a bounded sample of the workload for the fp64 oracle: the first
+    n heads of batch row 0 (one group, so heads slice freely), n chosen so one
+    run takes about budget_s on the host cores. Returns (run, tokens_equiv, desc)."""
+    import oracle
+    inp = inputs64 if inputs64 is not None else W.workload_inputs(w)
+    x = inp["x"][:1].double().numpy()
+    dt = inp["dt"][:1].double().numpy()
+    A = inp["A"].double().numpy()
+    B = inp["B"][:1].double().numpy()
+    C = inp["C"][:1].double().numpy()
+    D = inp["D"].double().numpy() if inp["D"] is not None else None
+    assert w.ngroups == 1
+
+    def make(nh):
+        xs = np.ascontiguousarray(x[:, :, :nh])
+        dts = np.ascontiguousarray(dt[:, :, :nh])
+        As = np.ascontiguousarray(A[:nh])
+        Ds = np.ascontiguousarray(D[:nh]) if D is not None else None
+        return lambda: oracle.recurrence(xs, dts, As, B, C, Ds)
+
+    threads = oracle.max_threads()
+    nh = min(w.nheads, max(1, threads))
+    t0 = time.perf_counter()
+    make(nh)()
+    t1 = time.perf_counter() - t0
+    scale = budget_s / max(t1, 1e-6)
+    nh2 = int(min(w.nheads, max(1, nh * scale)))
+    run = make(nh2)
+    tokens_equiv = w.seqlen * nh2 / w.nheads   # token-heads of one batch row / heads per token
+    desc = (f"batch row 0, heads 0..{nh2 - 1} of {w.nheads} (T={w.seqlen}); "
+            f"{nh2 * w.seqlen} token-heads = {tokens_equiv:.0f} token-equivalents per run")
+    return run, tokens_equiv, desc, threads
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args):
+    world, rank, local = dist_env()
+    if rank != 0:
+        return 0
+    w = WORKLOAD
+    per_step_budget = max(0.05, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    run, tok, desc, threads = oracle_sample(w, per_step_budget)
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    el = time.perf_counter() - t0
+    value = tok * args.steps / el / 1e6
+    cpu = {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+           "sample": f"fp64 sequential recurrence (C, OpenMP over heads) per step: {desc}"}
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, **w.shape_dict(), "input_dtype": w.dtype},
+            "cpu_baseline": cpu,
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+def kernel_plan(ssd, w, d, bufs, stream):
+    """The kernels of the unfused path as individually timed launches, with the
+    algorithmic bytes each must move per launch."""
+    b, T, H, P, G, N, Q = w.batch, w.seqlen, w.nheads, w.headdim, w.ngroups, w.dstate, w.chunk_size
+    nc = -(-T // Q)
+    s = 2 if w.dtype == "bf16" else 4
+    shp = ssd.make_shape(d["x"], d["B"], Q)
+    cs, S, entry, y, fin = bufs["cs"], bufs["S"], bufs["entry"], bufs["y"], bufs["final"]
+    st_bytes = 4.0 * b * nc * H * P * N
+    plan = [
+        ("chunk_cumsum", lambda: ssd.ssd_chunk_cumsum(d["dt"], d["A"], Q, shp, cs=cs, stream=stream),
+         4.0 * b * T * H + 4.0 * b * H * nc * Q),
+        ("chunk_state", lambda: ssd.ssd_chunk_state(d["x"], d["dt"], d["B"], cs, shp, states=S,
+                                                    stream=stream),
+         s * b * T * H * P + s * b * T * G * N + 4.0 * b * T * H + 4.0 * b * H * nc * Q + st_bytes),
+        ("state_passing", lambda: ssd.ssd_state_passing(S, cs, shp, entry_states=entry,
+                                                        final_states=fin, stream=stream),
+         2 * st_bytes + 4.0 * b * H * P * N + 4.0 * b * H * nc),
+        ("chunk_scan", lambda: ssd.ssd_chunk_scan(d["x"], d["dt"], d["B"], d["C"], d["D"], cs, entry,
+                                                  shp, y=y, stream=stream),
+         2.0 * s * b * T * H * P + 2.0 * s * b * T * G * N + 4.0 * b * T * H + 4.0 * b * H * nc * Q
+         + st_bytes),
+    ]
+    return plan
+
+
+def run_ours(args):
+    world, rank, local = dist_env()
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from structured_state_space_fwd_b200 import build as _b
+    _b.build()
+    import structured_state_space_fwd_b200 as ssd
+
+    w = WORKLOAD
+    inp = W.workload_inputs(w, seed=0)
+    d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+    b, T, H, P, G, N, Q = w.batch, w.seqlen, w.nheads, w.headdim, w.ngroups, w.dstate, w.chunk_size
+    nc = -(-T // Q)
+    stream = torch.cuda.current_stream(dev)
+    shp = ssd.make_shape(d["x"], d["B"], Q)
+    bufs = dict(y=torch.empty_like(d["x"]),
+                final=torch.empty((b, H, P, N), dtype=torch.float32, device=dev),
+                cs=torch.empty((b, H, nc, Q), dtype=torch.float32, device=dev),
+                S=torch.empty((b, nc, H, P, N), dtype=torch.float32, device=dev),
+                entry=torch.empty((b, nc, H, P, N), dtype=torch.float32, device=dev))
+    ws_bytes = ssd.ssd_fwd_workspace_size(shp)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+
+    def step():
+        ssd.ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], chunk_size=Q,
+                    y=bufs["y"], final_states=bufs["final"], return_final_states=True,
+                    workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms_total = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    ms_step = ms_total / args.steps
+    tokens_total = w.tokens * world
+    value = tokens_total * args.steps / (ms_total / 1e3) / 1e6
+
+    F, by = alg_counts(w, with_final=True, with_init=w.initial_states)
+    pk, pk_kind = peaks()
+    t_roof = max(F / (pk["bf16_tflops"] * 1e12), by / (pk["hbm_gbs"] * 1e9))
+    step_s = ms_step / 1e3
+
+    # per-kernel launch durations (each kernel timed alone, same inputs, CUDA events)
+    plan = kernel_plan(ssd, w, d, bufs, stream)
+    ktimes = {}
+    reps = max(3, min(50, args.steps))
+    for name, fn, _ in plan:
+        for _ in range(2):
+            fn()
+        k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        k0.record(stream)
+        for _ in range(reps):
+            fn()
+        k1.record(stream)
+        torch.cuda.synchronize()
+        ktimes[name] = k0.elapsed_time(k1) / reps
+    dom = max(plan, key=lambda p: ktimes[p[0]])
+    dom_s = ktimes[dom[0]] / 1e3
+    achieved = dom[2] / dom_s / 1e9
+    roofline = {"kernel": dom[0], "bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
+                "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                "peak_source": pk_kind + " (burst copy)",
+                "kernel_ms": {k: round(v, 5) for k, v in ktimes.items()}}
+
+    # end to end through the host-buffer entry point (pinned host memory)
+    e2e = None
+    if not args.no_e2e:
+        hp = {k: (v.pin_memory() if v is not None else None) for k, v in inp.items()}
+        hy = torch.empty_like(hp["x"]).pin_memory()
+        hf = torch.empty((b, H, P, N), dtype=torch.float32).pin_memory()
+        n = 0
+        import ctypes
+        nb = ctypes.c_size_t(0)
+        ssd.lib().ssd_fwd_host_workspace_size(ctypes.byref(shp), ctypes.byref(nb))
+        dws = torch.empty(int(nb.value), dtype=torch.uint8, device=dev)
+
+        def e2e_step():
+            ssd.ssd_fwd_host(hp["x"], hp["dt"], hp["A"], hp["B"], hp["C"], hp["D"], chunk_size=Q,
+                             y=hy, final_states=hf, device_workspace=dws, stream=stream)
+        for _ in range(2):
+            e2e_step()
+        ke = max(3, min(20, args.steps))
+        barrier(world)
+        torch.cuda.synchronize()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(ke):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        ms_e2e = max_over_ranks(a0.elapsed_time(a1), world, dev) / ke
+        h2d = sum(v.numel() * v.element_size() for v in hp.values() if v is not None)
+        d2h = hy.numel() * hy.element_size() + hf.numel() * hf.element_size()
+        e2e = {"value": w.tokens * world / (ms_e2e / 1e3) / 1e6, "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": ms_e2e, "api": "ssd_fwd_host (pinned host buffers)"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        run, tok, desc, threads = oracle_sample(w, 15.0, inputs64=inp)
+        t0 = time.perf_counter()
+        run()
+        el = time.perf_counter() - t0
+        cpu = {"value": tok / el / 1e6, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"fp64 sequential recurrence, {desc}; one run of {el:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, **w.shape_dict(), "input_dtype": w.dtype,
+                       "final_states": True, "per_rank_batch": b,
+                       "l2": "inputs larger than L2 (x and y 168 MB each), no flush"},
+            "tflops": F * world / step_s / 1e12,
+            "step_roofline": {"t_roof_us": t_roof * 1e6, "t_step_us": step_s * 1e6,
+                              "frac": t_roof / step_s, "alg_gflop": F / 1e9, "alg_mb": by / 1e6,
+                              "peaks": pk_kind},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": 4 * args.steps,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,170 @@
+/*
+ * ssd.h - C ABI of libssd, the forward pass of the state space dual (SSD) layer
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The layer ("Transformers are SSMs: Generalized Models and Efficient
+ * Algorithms Through Structured State Space Duality", Knowl 1) is the
+ * scalar-identity selective SSM, per batch row b and head h:
+ *
+ *     h_t = exp(dt_t * A_h) * h_{t-1} + dt_t * x_t (outer) B_t      h_{-1} = h_init or 0
+ *     y_t = C_t . h_t + D_h * x_t
+ *
+ * evaluated through its dual form Y = (L o C B^T) X with the 1-semiseparable
+ * decay mask L_ji = prod_{s=i+1}^{j} a_s, by the block-decomposition algorithm
+ * of Knowl 2: chunks of Q tokens, a quadratic (masked attention) product inside
+ * each chunk and a linear recurrence over chunk states between chunks.
+ *
+ * Shapes (row-major, contiguous, innermost last):
+ *     x, y            [batch, seqlen, nheads, headdim]      dtype (fp32 or bf16)
+ *     dt              [batch, seqlen, nheads]               fp32
+ *     A, D            [nheads]                              fp32
+ *     B, C            [batch, seqlen, ngroups, dstate]      dtype
+ *     states          [batch, nheads, headdim, dstate]      fp32
+ * Head h reads B and C of group g = h / (nheads / ngroups) (Knowl 7: grouped
+ * heads share B and C; ngroups = 1 is the multi-input pattern).
+ *
+ * Conventions for every entry point:
+ *   - Device pointers are CUDA device (or managed) memory owned by the caller.
+ *     The library allocates no device memory and keeps no state between calls,
+ *     so calls on different streams or host threads are independent.
+ *   - All argument checks run on the host before anything is enqueued; a
+ *     rejected call enqueues nothing and returns SSD_ERR_INVALID_ARG or
+ *     SSD_ERR_UNSUPPORTED synchronously.
+ *   - Device entry points are asynchronous on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream) and never synchronize. A launch failure
+ *     returns SSD_ERR_CUDA; ssd_last_error_detail() then names the CUDA error.
+ *   - Inputs may alias one another; an output must not overlap any input, any
+ *     other output or the workspace (SSD_ERR_INVALID_ARG).
+ *   - x, B, C, y, the state tensors and the workspace must be 16-byte aligned;
+ *     dt, A and D 4-byte aligned.
+ */
+#ifndef SSD_H_
+#define SSD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SSD_API __attribute__((visibility("default")))
+#else
+#define SSD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SSD_OK = 0,
+    SSD_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, overlap, small workspace */
+    SSD_ERR_UNSUPPORTED = 2,   /* valid shape outside what the kernels implement */
+    SSD_ERR_CUDA = 3,          /* a CUDA call failed; see ssd_last_error_detail() */
+    SSD_ERR_TIMEOUT = 4        /* a bounded device-side wait gave up */
+} ssd_status_t;
+
+typedef enum { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype_t;
+
+typedef struct {
+    int64_t batch;       /* b >= 0                                          */
+    int64_t seqlen;      /* T >= 0; T need not be a multiple of chunk_size  */
+    int64_t nheads;      /* H >= 1                                          */
+    int64_t headdim;     /* P in [1, 256]                                   */
+    int64_t ngroups;     /* G >= 1, divides H                               */
+    int64_t dstate;      /* N in [1, 256]                                   */
+    int64_t chunk_size;  /* Q in {16, 32, 64, 128, 256}                     */
+    int32_t dtype;       /* ssd_dtype_t of x, B, C and y                    */
+    int32_t reserved;    /* must be 0                                       */
+} ssd_shape_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+SSD_API const char* ssd_status_string(ssd_status_t status);
+
+/* Detail of the last SSD_ERR_CUDA / SSD_ERR_TIMEOUT on the calling host thread
+ * ("" if none). The pointer stays valid until the next call on that thread. */
+SSD_API const char* ssd_last_error_detail(void);
+
+/* Library version as major*10000 + minor*100 + patch. */
+SSD_API int ssd_version(void);
+
+/* Bytes of device workspace ssd_fwd needs for `shape`, written to *bytes.
+ * Returns SSD_ERR_INVALID_ARG / SSD_ERR_UNSUPPORTED for a shape ssd_fwd rejects. */
+SSD_API ssd_status_t ssd_fwd_workspace_size(const ssd_shape_t* shape, size_t* bytes);
+
+/*
+ * Full SSD layer forward (Knowl 2, whole algorithm; Knowl 1 for the result).
+ *   x, dt, A, B, C     inputs as above (device).
+ *   D                  [H] fp32 skip weights, or NULL for D = 0.
+ *   initial_states     [b,H,P,N] fp32 state entering the sequence, or NULL for 0.
+ *   y                  [b,T,H,P] output in `dtype` (device), rounded to nearest even.
+ *   final_states       [b,H,P,N] fp32 state after the last token, or NULL to skip.
+ *                      Must not be the same memory as initial_states.
+ *   workspace          device scratch of at least ssd_fwd_workspace_size() bytes
+ *                      (may be NULL when that size is 0). Its contents on entry
+ *                      are ignored; concurrent calls need separate workspaces.
+ * Result (y, final_states) equals the recurrence above up to rounding: the
+ * decay math and accumulation are fp32 for both dtypes.
+ */
+SSD_API ssd_status_t ssd_fwd(const ssd_shape_t* shape,
+                     const void* x, const float* dt, const float* A,
+                     const void* B, const void* C, const float* D,
+                     const float* initial_states,
+                     void* y, float* final_states,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of device workspace ssd_fwd_host needs (inputs, outputs and ssd_fwd's
+ * own workspace are staged there). */
+SSD_API ssd_status_t ssd_fwd_host_workspace_size(const ssd_shape_t* shape, size_t* bytes);
+
+/*
+ * Same computation as ssd_fwd on HOST buffers: copies the inputs to the device
+ * workspace on `stream`, runs ssd_fwd there, copies y (and final_states when
+ * non-NULL) back, and synchronizes `stream` before returning, so the host
+ * outputs are ready on return. Host buffers should be page-locked for full
+ * copy bandwidth; pageable memory works but is slower. The device workspace
+ * must hold ssd_fwd_host_workspace_size() bytes.
+ */
+SSD_API ssd_status_t ssd_fwd_host(const ssd_shape_t* shape,
+                          const void* x, const float* dt, const float* A,
+                          const void* B, const void* C, const float* D,
+                          const float* initial_states,
+                          void* y, float* final_states,
+                          void* device_workspace, size_t workspace_bytes, void* stream);
+
+/* ---- The four steps of the block-decomposition algorithm, one call each. ----
+ * ssd_fwd runs the same steps (or a fused equivalent); these entry points
+ * expose each one with its intermediate tensors for callers that need them:
+ *     cs       [b, H, nc, Q]      fp32, nc = ceil(T / Q)
+ *     states   [b, nc, H, P, N]   fp32
+ */
+
+/* Step 1 (Knowl 2, "intra-chunk cumulative products of A", kept as log sums):
+ * cs[b,h,c,k] = sum_{k'<=k} dt[b, cQ+k', h] * A[h], inclusive, within chunk c.
+ * Entries past the end of a partial last chunk repeat its last value. */
+SSD_API ssd_status_t ssd_chunk_cumsum(const ssd_shape_t* shape, const float* dt, const float* A,
+                              float* cs, void* stream);
+
+/* Step 2 (Knowl 2, "right factor chunk state" B^T (decayed X)):
+ * states[b,c,h,p,n] = sum_{k in chunk c} exp(cs[..,last] - cs[..,k]) * dt_k * x_k[p] * B_k[n],
+ * the state chunk c alone produces from a zero state. */
+SSD_API ssd_status_t ssd_chunk_state(const ssd_shape_t* shape, const void* x, const float* dt,
+                             const void* B, const float* cs, float* states, void* stream);
+
+/* Step 3 (Knowl 2, inter-chunk recurrence h_{c+1} = (prod_t a_t) h_c + S_c):
+ * entry_states[b,c] receives h_c, the state entering chunk c (h_0 = initial_states
+ * or 0); final_states (nullable) receives h_nc. */
+SSD_API ssd_status_t ssd_state_passing(const ssd_shape_t* shape, const float* states, const float* cs,
+                               const float* initial_states, float* entry_states,
+                               float* final_states, void* stream);
+
+/* Step 4 (Knowl 2, Y_diag + Y_off per chunk, plus the D skip term):
+ * y[j] = sum_{i<=j in chunk} (C_j . B_i) exp(cs_j - cs_i) dt_i x_i
+ *        + exp(cs_j) C_j . h_c + D_h x_j. */
+SSD_API ssd_status_t ssd_chunk_scan(const ssd_shape_t* shape, const void* x, const float* dt,
+                            const void* B, const void* C, const float* D, const float* cs,
+                            const float* entry_states, void* y, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSD_H_ */

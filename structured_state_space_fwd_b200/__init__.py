@@ -1,0 +1,153 @@
+"""Thin Python binding of libssd, the B200 SSD layer forward.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of libssd.so. PyTorch supplies device memory and the current stream.
+If the shared library is missing or fails to load, every call raises; there
+is no fallback implementation.
+
+    y, final = ssd_fwd(x, dt, A, B, C, D, chunk_size=256,
+                       initial_states=None, return_final_states=True)
+
+Shapes: x[b,T,H,P], dt[b,T,H], A[H], B/C[b,T,G,N], D[H], states[b,H,P,N]
+("Transformers are SSMs: Generalized Models and Efficient Algorithms Through
+Structured State Space Duality", Knowl 1, 2 and 7).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from ._lib import (SSD_BF16, SSD_F32, SSDError, ShapeT, check, lib, lib_path,  # noqa: F401
+                   status_string)
+
+__all__ = ["ssd_fwd", "ssd_fwd_host", "ssd_fwd_workspace_size", "ssd_chunk_cumsum",
+           "ssd_chunk_state", "ssd_state_passing", "ssd_chunk_scan", "SSDError", "make_shape",
+           "lib_path"]
+
+_DT = {torch.float32: SSD_F32, torch.bfloat16: SSD_BF16}
+
+
+def make_shape(x: torch.Tensor, B: torch.Tensor, chunk_size: int) -> ShapeT:
+    b, T, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    if x.dtype not in _DT:
+        raise TypeError(f"x must be float32 or bfloat16, got {x.dtype}")
+    return ShapeT(b, T, H, P, G, N, int(chunk_size), _DT[x.dtype], 0)
+
+
+def _p(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t, name, dtype=None, device=True):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if device and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t
+
+
+def ssd_fwd_workspace_size(shape: ShapeT) -> int:
+    n = ctypes.c_size_t(0)
+    check(lib().ssd_fwd_workspace_size(ctypes.byref(shape), ctypes.byref(n)), "ssd_fwd_workspace_size")
+    return int(n.value)
+
+
+def ssd_fwd(x, dt, A, B, C, D=None, chunk_size: int = 256, initial_states=None,
+            return_final_states: bool = False, y=None, final_states=None, workspace=None,
+            stream=None):
+    """SSD layer forward on the GPU; returns y, or (y, final_states)."""
+    _need(x, "x")
+    _need(dt, "dt", torch.float32)
+    _need(A, "A", torch.float32)
+    _need(B, "B", x.dtype)
+    _need(C, "C", x.dtype)
+    if D is not None:
+        _need(D, "D", torch.float32)
+    if initial_states is not None:
+        _need(initial_states, "initial_states", torch.float32)
+    shape = make_shape(x, B, chunk_size)
+    if y is None:
+        y = torch.empty_like(x)
+    if return_final_states and final_states is None:
+        final_states = torch.empty((x.shape[0], x.shape[2], x.shape[3], B.shape[3]),
+                                   dtype=torch.float32, device=x.device)
+    nbytes = ssd_fwd_workspace_size(shape)
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=x.device)
+    check(lib().ssd_fwd(ctypes.byref(shape), _p(x), _p(dt), _p(A), _p(B), _p(C), _p(D),
+                        _p(initial_states), _p(y), _p(final_states), _p(workspace),
+                        ctypes.c_size_t(nbytes), _stream(stream)), "ssd_fwd")
+    return (y, final_states) if return_final_states else y
+
+
+def ssd_fwd_host(x, dt, A, B, C, D=None, chunk_size: int = 256, initial_states=None,
+                 y=None, final_states=None, device_workspace=None, stream=None):
+    """ssd_fwd on host (CPU, ideally pinned) tensors; synchronous. Returns (y, final_states)."""
+    for t, n in ((x, "x"), (dt, "dt"), (A, "A"), (B, "B"), (C, "C")):
+        _need(t, n, device=False)
+    shape = make_shape(x, B, chunk_size)
+    if y is None:
+        y = torch.empty_like(x)
+    n = ctypes.c_size_t(0)
+    check(lib().ssd_fwd_host_workspace_size(ctypes.byref(shape), ctypes.byref(n)),
+          "ssd_fwd_host_workspace_size")
+    if device_workspace is None or device_workspace.numel() < n.value:
+        device_workspace = torch.empty(max(int(n.value), 1), dtype=torch.uint8, device="cuda")
+    check(lib().ssd_fwd_host(ctypes.byref(shape), _p(x), _p(dt), _p(A), _p(B), _p(C), _p(D),
+                             _p(initial_states), _p(y), _p(final_states), _p(device_workspace),
+                             ctypes.c_size_t(n.value), _stream(stream)), "ssd_fwd_host")
+    return y, final_states
+
+
+def ssd_chunk_cumsum(dt, A, chunk_size, shape: ShapeT, cs=None, stream=None):
+    nc = -(-shape.seqlen // chunk_size)
+    if cs is None:
+        cs = torch.empty((shape.batch, shape.nheads, nc, chunk_size), dtype=torch.float32,
+                         device=dt.device)
+    check(lib().ssd_chunk_cumsum(ctypes.byref(shape), _p(dt), _p(A), _p(cs), _stream(stream)),
+          "ssd_chunk_cumsum")
+    return cs
+
+
+def ssd_chunk_state(x, dt, B, cs, shape: ShapeT, states=None, stream=None):
+    nc = cs.shape[2]
+    if states is None:
+        states = torch.empty((shape.batch, nc, shape.nheads, shape.headdim, shape.dstate),
+                             dtype=torch.float32, device=x.device)
+    check(lib().ssd_chunk_state(ctypes.byref(shape), _p(x), _p(dt), _p(B), _p(cs), _p(states),
+                                _stream(stream)), "ssd_chunk_state")
+    return states
+
+
+def ssd_state_passing(states, cs, shape: ShapeT, initial_states=None, entry_states=None,
+                      final_states=None, stream=None):
+    if entry_states is None:
+        entry_states = torch.empty_like(states)
+    if final_states is None:
+        final_states = torch.empty((shape.batch, shape.nheads, shape.headdim, shape.dstate),
+                                   dtype=torch.float32, device=states.device)
+    check(lib().ssd_state_passing(ctypes.byref(shape), _p(states), _p(cs), _p(initial_states),
+                                  _p(entry_states), _p(final_states), _stream(stream)),
+          "ssd_state_passing")
+    return entry_states, final_states
+
+
+def ssd_chunk_scan(x, dt, B, C, D, cs, entry_states, shape: ShapeT, y=None, stream=None):
+    if y is None:
+        y = torch.empty_like(x)
+    check(lib().ssd_chunk_scan(ctypes.byref(shape), _p(x), _p(dt), _p(B), _p(C), _p(D), _p(cs),
+                               _p(entry_states), _p(y), _stream(stream)), "ssd_chunk_scan")
+    return y

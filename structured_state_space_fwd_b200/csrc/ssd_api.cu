@@ -1,0 +1,342 @@
+// C ABI of libssd: host-side argument checks, workspace layout and dispatch of
+// the block-decomposition steps ("Transformers are SSMs", Knowl 2) onto the
+// caller's stream. Nothing here allocates device memory or synchronizes,
+// except ssd_fwd_host, whose contract is to return finished host outputs.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <initializer_list>
+
+#include "ssd.h"
+#include "ssd_internal.h"
+
+namespace {
+
+thread_local char g_detail[256] = "";
+
+void set_detail(const char* what, cudaError_t e) {
+    snprintf(g_detail, sizeof(g_detail), "%s: %s (%d)", what, cudaGetErrorString(e), (int)e);
+}
+
+constexpr int64_t kMaxDim = 256;
+
+bool is_pow2_chunk(int64_t q) {
+    return q == 16 || q == 32 || q == 64 || q == 128 || q == 256;
+}
+
+// Shape rules shared by every entry point.
+ssd_status_t check_shape(const ssd_shape_t* s) {
+    if (!s) return SSD_ERR_INVALID_ARG;
+    if (s->reserved != 0) return SSD_ERR_INVALID_ARG;
+    if (s->batch < 0 || s->seqlen < 0) return SSD_ERR_INVALID_ARG;
+    if (s->nheads < 1 || s->headdim < 1 || s->ngroups < 1 || s->dstate < 1)
+        return SSD_ERR_INVALID_ARG;
+    if (s->nheads % s->ngroups != 0) return SSD_ERR_INVALID_ARG;
+    if (s->dtype != SSD_F32 && s->dtype != SSD_BF16) return SSD_ERR_INVALID_ARG;
+    if (s->chunk_size < 1) return SSD_ERR_INVALID_ARG;
+    if (!is_pow2_chunk(s->chunk_size)) return SSD_ERR_UNSUPPORTED;
+    if (s->headdim > kMaxDim || s->dstate > kMaxDim) return SSD_ERR_UNSUPPORTED;
+    // keep every element index well inside int64 and grid sizes inside CUDA limits
+    const double tok = (double)s->batch * (double)s->seqlen;
+    if (tok * (double)s->nheads * (double)s->headdim > 4.0e15) return SSD_ERR_UNSUPPORTED;
+    if (tok * (double)s->ngroups * (double)s->dstate > 4.0e15) return SSD_ERR_UNSUPPORTED;
+    if ((double)s->batch * s->nheads * s->headdim * s->dstate > 4.0e15) return SSD_ERR_UNSUPPORTED;
+    if (s->batch > 65535) return SSD_ERR_UNSUPPORTED;                 // grid.z
+    const int64_t nc = s->seqlen > 0 ? (s->seqlen + s->chunk_size - 1) / s->chunk_size : 0;
+    if (nc * s->nheads > 2147483647LL) return SSD_ERR_UNSUPPORTED;    // grid.y
+    if (s->nheads > 65535) return SSD_ERR_UNSUPPORTED;
+    return SSD_OK;
+}
+
+size_t elem_size(int dtype) { return dtype == SSD_BF16 ? 2 : 4; }
+
+struct Range {
+    const void* p;
+    size_t bytes;
+};
+
+bool overlaps(Range a, Range b) {
+    if (!a.p || !b.p || a.bytes == 0 || b.bytes == 0) return false;
+    const uintptr_t a0 = (uintptr_t)a.p, b0 = (uintptr_t)b.p;
+    return a0 < b0 + b.bytes && b0 < a0 + a.bytes;
+}
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+struct Sizes {
+    size_t x, dt, hv, bc, st, cs, chunk_states;
+};
+
+Sizes sizes_of(const ssd::Dims& d) {
+    Sizes z;
+    const size_t es = elem_size(d.dtype);
+    z.x = (size_t)(d.b * d.T * d.H * d.P) * es;
+    z.dt = (size_t)(d.b * d.T * d.H) * 4;
+    z.hv = (size_t)d.H * 4;
+    z.bc = (size_t)(d.b * d.T * d.G * d.N) * es;
+    z.st = (size_t)(d.b * d.H * d.P * d.N) * 4;
+    z.cs = (size_t)(d.b * d.H * d.nc * d.Q) * 4;
+    z.chunk_states = (size_t)(d.b * d.nc * d.H * d.P * d.N) * 4;
+    return z;
+}
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Workspace of ssd_fwd: [cs | chunk states S | entry states h_c], each 256-byte aligned.
+struct FwdWorkspace {
+    size_t off_cs, off_S, off_entry, total;
+};
+
+FwdWorkspace fwd_workspace(const ssd::Dims& d) {
+    const Sizes z = sizes_of(d);
+    FwdWorkspace w;
+    w.off_cs = 0;
+    w.off_S = align_up(z.cs, 256);
+    w.off_entry = w.off_S + align_up(z.chunk_states, 256);
+    w.total = w.off_entry + align_up(z.chunk_states, 256);
+    if (d.b == 0 || d.T == 0) w.total = 0;
+    return w;
+}
+
+ssd_status_t cuda_status(const char* what, cudaError_t e) {
+    if (e == cudaSuccess) return SSD_OK;
+    set_detail(what, e);
+    return SSD_ERR_CUDA;
+}
+
+ssd_status_t check_fwd_args(const ssd_shape_t* shape, const void* x, const float* dt,
+                            const float* A, const void* B, const void* C, const float* D,
+                            const float* init, void* y, float* final_states,
+                            const void* workspace, size_t workspace_bytes) {
+    ssd_status_t st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    const ssd::Dims d = ssd::make_dims(*shape);
+    const Sizes z = sizes_of(d);
+    // a pointer may be NULL only when its tensor has no elements
+    if ((!x && z.x) || (!dt && z.dt) || !A || (!B && z.bc) || (!C && z.bc) || (!y && z.x))
+        return SSD_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(y, 16))
+        return SSD_ERR_INVALID_ARG;
+    if (!aligned(dt, 4) || !aligned(A, 4) || (D && !aligned(D, 4))) return SSD_ERR_INVALID_ARG;
+    if ((init && !aligned(init, 16)) || (final_states && !aligned(final_states, 16)))
+        return SSD_ERR_INVALID_ARG;
+    if (workspace && !aligned(workspace, 16)) return SSD_ERR_INVALID_ARG;
+    const FwdWorkspace w = fwd_workspace(d);
+    if (workspace_bytes < w.total || (w.total > 0 && !workspace)) return SSD_ERR_INVALID_ARG;
+    const Range ins[] = {{x, z.x}, {dt, z.dt}, {A, z.hv}, {B, z.bc}, {C, z.bc},
+                         {D, D ? z.hv : 0}, {init, init ? z.st : 0}};
+    const Range outs[] = {{y, z.x}, {final_states, final_states ? z.st : 0},
+                          {workspace, w.total}};
+    for (const Range& o : outs) {
+        for (const Range& i : ins)
+            if (overlaps(o, i)) return SSD_ERR_INVALID_ARG;
+    }
+    for (int i = 0; i < 3; ++i)
+        for (int j = i + 1; j < 3; ++j)
+            if (overlaps(outs[i], outs[j])) return SSD_ERR_INVALID_ARG;
+    if (final_states && init && final_states == init) return SSD_ERR_INVALID_ARG;
+    return SSD_OK;
+}
+
+ssd_status_t run_fwd(const ssd::Dims& d, const void* x, const float* dt, const float* A,
+                     const void* B, const void* C, const float* D, const float* init, void* y,
+                     float* final_states, void* workspace, cudaStream_t stream) {
+    if (d.b == 0) return SSD_OK;
+    if (d.T == 0) return cuda_status("final states", ssd::launch_copy_or_zero_states(d, init, final_states, stream));
+    const FwdWorkspace w = fwd_workspace(d);
+    char* ws = (char*)workspace;
+    float* cs = (float*)(ws + w.off_cs);
+    float* S = (float*)(ws + w.off_S);
+    float* entry = (float*)(ws + w.off_entry);
+    ssd_status_t st;
+    if ((st = cuda_status("chunk cumsum", ssd::launch_chunk_cumsum(d, dt, A, cs, stream))) != SSD_OK)
+        return st;
+    if ((st = cuda_status("chunk state",
+                          ssd::launch_chunk_state_simt(d, x, dt, B, cs, S, stream))) != SSD_OK)
+        return st;
+    if ((st = cuda_status("state passing", ssd::launch_state_passing(d, S, cs, init, entry,
+                                                                      final_states, stream))) != SSD_OK)
+        return st;
+    return cuda_status("chunk scan",
+                       ssd::launch_chunk_scan_simt(d, x, dt, B, C, D, cs, entry, y, stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ssd_status_string(ssd_status_t s) {
+    switch (s) {
+        case SSD_OK: return "SSD_OK";
+        case SSD_ERR_INVALID_ARG: return "SSD_ERR_INVALID_ARG";
+        case SSD_ERR_UNSUPPORTED: return "SSD_ERR_UNSUPPORTED";
+        case SSD_ERR_CUDA: return "SSD_ERR_CUDA";
+        case SSD_ERR_TIMEOUT: return "SSD_ERR_TIMEOUT";
+    }
+    return "SSD_ERR_UNKNOWN";
+}
+
+const char* ssd_last_error_detail(void) { return g_detail; }
+
+int ssd_version(void) { return 100; }
+
+ssd_status_t ssd_fwd_workspace_size(const ssd_shape_t* shape, size_t* bytes) {
+    if (!bytes) return SSD_ERR_INVALID_ARG;
+    ssd_status_t st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    *bytes = fwd_workspace(ssd::make_dims(*shape)).total;
+    return SSD_OK;
+}
+
+ssd_status_t ssd_fwd(const ssd_shape_t* shape, const void* x, const float* dt, const float* A,
+                     const void* B, const void* C, const float* D, const float* initial_states,
+                     void* y, float* final_states, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+    ssd_status_t st = check_fwd_args(shape, x, dt, A, B, C, D, initial_states, y, final_states,
+                                     workspace, workspace_bytes);
+    if (st != SSD_OK) return st;
+    return run_fwd(ssd::make_dims(*shape), x, dt, A, B, C, D, initial_states, y, final_states,
+                   workspace, (cudaStream_t)stream);
+}
+
+// Host-buffer variant: [fwd workspace | x | dt | A | B | C | D | init | y | final]
+ssd_status_t ssd_fwd_host_workspace_size(const ssd_shape_t* shape, size_t* bytes) {
+    if (!bytes) return SSD_ERR_INVALID_ARG;
+    ssd_status_t st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    const ssd::Dims d = ssd::make_dims(*shape);
+    const Sizes z = sizes_of(d);
+    size_t tot = align_up(fwd_workspace(d).total, 256);
+    for (size_t s : {z.x, z.dt, z.hv, z.bc, z.bc, z.hv, z.st, z.x, z.st}) tot += align_up(s, 256);
+    *bytes = tot;
+    return SSD_OK;
+}
+
+ssd_status_t ssd_fwd_host(const ssd_shape_t* shape, const void* x, const float* dt,
+                          const float* A, const void* B, const void* C, const float* D,
+                          const float* initial_states, void* y, float* final_states,
+                          void* device_workspace, size_t workspace_bytes, void* stream) {
+    ssd_status_t st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    {
+        const Sizes z0 = sizes_of(ssd::make_dims(*shape));
+        if ((!x && z0.x) || (!dt && z0.dt) || !A || (!B && z0.bc) || (!C && z0.bc) || (!y && z0.x))
+            return SSD_ERR_INVALID_ARG;
+    }
+    if (!device_workspace || !aligned(device_workspace, 256)) return SSD_ERR_INVALID_ARG;
+    size_t need = 0;
+    ssd_fwd_host_workspace_size(shape, &need);
+    if (workspace_bytes < need) return SSD_ERR_INVALID_ARG;
+    const ssd::Dims d = ssd::make_dims(*shape);
+    const Sizes z = sizes_of(d);
+    cudaStream_t s = (cudaStream_t)stream;
+    char* base = (char*)device_workspace;
+    size_t off = align_up(fwd_workspace(d).total, 256);
+    auto take = [&](size_t bytes) {
+        char* p = base + off;
+        off += align_up(bytes, 256);
+        return p;
+    };
+    void* dx = take(z.x);
+    float* ddt = (float*)take(z.dt);
+    float* dA = (float*)take(z.hv);
+    void* dB = take(z.bc);
+    void* dC = take(z.bc);
+    float* dD = (float*)take(z.hv);
+    float* dinit = (float*)take(z.st);
+    void* dy = take(z.x);
+    float* dfinal = (float*)take(z.st);
+    struct Cp { void* dst; const void* src; size_t n; };
+    const Cp h2d[] = {{dx, x, z.x}, {ddt, dt, z.dt}, {dA, A, z.hv}, {dB, B, z.bc}, {dC, C, z.bc},
+                      {dD, D, D ? z.hv : 0}, {dinit, initial_states, initial_states ? z.st : 0}};
+    for (const Cp& c : h2d) {
+        if (c.n == 0) continue;
+        if ((st = cuda_status("host to device copy",
+                              cudaMemcpyAsync(c.dst, c.src, c.n, cudaMemcpyHostToDevice, s))) != SSD_OK)
+            return st;
+    }
+    st = run_fwd(d, dx, ddt, dA, dB, dC, D ? dD : nullptr, initial_states ? dinit : nullptr, dy,
+                 final_states ? dfinal : nullptr, base, s);
+    if (st != SSD_OK) return st;
+    if (z.x && (st = cuda_status("device to host copy",
+                                 cudaMemcpyAsync(y, dy, z.x, cudaMemcpyDeviceToHost, s))) != SSD_OK)
+        return st;
+    if (final_states && z.st &&
+        (st = cuda_status("device to host copy",
+                          cudaMemcpyAsync(final_states, dfinal, z.st, cudaMemcpyDeviceToHost, s))) != SSD_OK)
+        return st;
+    return cuda_status("stream synchronize", cudaStreamSynchronize(s));
+}
+
+ssd_status_t ssd_chunk_cumsum(const ssd_shape_t* shape, const float* dt, const float* A,
+                              float* cs, void* stream) {
+    ssd_status_t st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    if (!dt || !A || !cs) return SSD_ERR_INVALID_ARG;
+    const ssd::Dims d = ssd::make_dims(*shape);
+    const Sizes z = sizes_of(d);
+    if (overlaps({cs, z.cs}, {dt, z.dt}) || overlaps({cs, z.cs}, {A, z.hv}))
+        return SSD_ERR_INVALID_ARG;
+    return cuda_status("chunk cumsum", ssd::launch_chunk_cumsum(d, dt, A, cs, (cudaStream_t)stream));
+}
+
+ssd_status_t ssd_chunk_state(const ssd_shape_t* shape, const void* x, const float* dt,
+                             const void* B, const float* cs, float* states, void* stream) {
+    ssd_status_t st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    if (!x || !dt || !B || !cs || !states) return SSD_ERR_INVALID_ARG;
+    const ssd::Dims d = ssd::make_dims(*shape);
+    const Sizes z = sizes_of(d);
+    const Range o{states, z.chunk_states};
+    if (overlaps(o, {x, z.x}) || overlaps(o, {dt, z.dt}) || overlaps(o, {B, z.bc}) ||
+        overlaps(o, {cs, z.cs}))
+        return SSD_ERR_INVALID_ARG;
+    return cuda_status("chunk state", ssd::launch_chunk_state_simt(d, x, dt, B, cs, states,
+                                                                     (cudaStream_t)stream));
+}
+
+ssd_status_t ssd_state_passing(const ssd_shape_t* shape, const float* states, const float* cs,
+                               const float* initial_states, float* entry_states,
+                               float* final_states, void* stream) {
+    ssd_status_t st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    if (!states || !cs || !entry_states) return SSD_ERR_INVALID_ARG;
+    const ssd::Dims d = ssd::make_dims(*shape);
+    const Sizes z = sizes_of(d);
+    const Range ins[] = {{states, z.chunk_states}, {cs, z.cs},
+                         {initial_states, initial_states ? z.st : 0}};
+    const Range outs[] = {{entry_states, z.chunk_states}, {final_states, final_states ? z.st : 0}};
+    for (const Range& o : outs)
+        for (const Range& i : ins)
+            if (overlaps(o, i)) return SSD_ERR_INVALID_ARG;
+    if (overlaps(outs[0], outs[1])) return SSD_ERR_INVALID_ARG;
+    if (d.T == 0)
+        return cuda_status("final states", ssd::launch_copy_or_zero_states(d, initial_states,
+                                                                           final_states,
+                                                                           (cudaStream_t)stream));
+    return cuda_status("state passing",
+                       ssd::launch_state_passing(d, states, cs, initial_states, entry_states,
+                                                 final_states, (cudaStream_t)stream));
+}
+
+ssd_status_t ssd_chunk_scan(const ssd_shape_t* shape, const void* x, const float* dt,
+                            const void* B, const void* C, const float* D, const float* cs,
+                            const float* entry_states, void* y, void* stream) {
+    ssd_status_t st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    if (!x || !dt || !B || !C || !cs || !entry_states || !y) return SSD_ERR_INVALID_ARG;
+    const ssd::Dims d = ssd::make_dims(*shape);
+    const Sizes z = sizes_of(d);
+    const Range o{y, z.x};
+    const Range ins[] = {{x, z.x}, {dt, z.dt}, {B, z.bc}, {C, z.bc}, {D, D ? z.hv : 0},
+                         {cs, z.cs}, {entry_states, z.chunk_states}};
+    for (const Range& i : ins)
+        if (overlaps(o, i)) return SSD_ERR_INVALID_ARG;
+    return cuda_status("chunk scan", ssd::launch_chunk_scan_simt(d, x, dt, B, C, D, cs,
+                                                                   entry_states, y,
+                                                                   (cudaStream_t)stream));
+}
+
+}  // extern "C"

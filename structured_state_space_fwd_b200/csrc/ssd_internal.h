@@ -1,0 +1,38 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ssd.h"
+
+namespace ssd {
+
+struct Dims {
+    int64_t b, T, H, P, G, N, Q, nc;
+    int dtype;  // ssd_dtype_t
+};
+
+inline Dims make_dims(const ssd_shape_t& s) {
+    Dims d;
+    d.b = s.batch; d.T = s.seqlen; d.H = s.nheads; d.P = s.headdim; d.G = s.ngroups;
+    d.N = s.dstate; d.Q = s.chunk_size; d.dtype = s.dtype;
+    d.nc = d.T > 0 ? (d.T + d.Q - 1) / d.Q : 0;
+    return d;
+}
+
+// CUDA-core kernels (any supported shape, fp32 or bf16 storage, fp32 math).
+cudaError_t launch_chunk_cumsum(const Dims& d, const float* dt, const float* A, float* cs,
+                                cudaStream_t st);
+cudaError_t launch_chunk_state_simt(const Dims& d, const void* x, const float* dt, const void* B,
+                                    const float* cs, float* states, cudaStream_t st);
+cudaError_t launch_state_passing(const Dims& d, const float* states, const float* cs,
+                                 const float* init, float* entry, float* final_states,
+                                 cudaStream_t st);
+cudaError_t launch_chunk_scan_simt(const Dims& d, const void* x, const float* dt, const void* B,
+                                   const void* C, const float* D, const float* cs,
+                                   const float* entry, void* y, cudaStream_t st);
+cudaError_t launch_copy_or_zero_states(const Dims& d, const float* init, float* final_states,
+                                       cudaStream_t st);
+
+}  // namespace ssd

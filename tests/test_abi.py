@@ -1,0 +1,182 @@
+"""Host-only checks of the C ABI: the library loads, exports every declared
+symbol, and rejects bad arguments before launching anything.
+
+No test here computes on a GPU. On a machine without CUDA the calls use
+placeholder addresses that the library never dereferences (every call is
+expected to fail validation); on a machine with CUDA they use real device
+buffers, so even a validation bug could not touch foreign memory.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from structured_state_space_fwd_b200 import build
+    build.build()
+    from structured_state_space_fwd_b200 import _lib
+    return _lib
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "ssd.h")).read()
+    return sorted(set(re.findall(r"SSD_API\s+[\w\s\*]+?\b(ssd_\w+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert len(names) >= 11
+    lib = L.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(L):
+    for code, name in enumerate(["SSD_OK", "SSD_ERR_INVALID_ARG", "SSD_ERR_UNSUPPORTED",
+                                 "SSD_ERR_CUDA", "SSD_ERR_TIMEOUT"]):
+        assert L.status_string(code) == name
+    assert L.lib().ssd_version() >= 100
+
+
+def shape(**kw):
+    from structured_state_space_fwd_b200._lib import ShapeT
+    d = dict(batch=2, seqlen=300, nheads=4, headdim=64, ngroups=2, dstate=64, chunk_size=128,
+             dtype=1, reserved=0)
+    d.update(kw)
+    return ShapeT(**d)
+
+
+def ws_size(L, s):
+    n = ctypes.c_size_t(0)
+    st = L.lib().ssd_fwd_workspace_size(ctypes.byref(s), ctypes.byref(n))
+    return st, n.value
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(nheads=6, ngroups=4), 1),        # G does not divide H
+    (dict(headdim=0), 1),
+    (dict(dstate=-1), 1),
+    (dict(batch=-1), 1),
+    (dict(dtype=7), 1),
+    (dict(reserved=3), 1),
+    (dict(chunk_size=0), 1),
+    (dict(chunk_size=96), 2),              # not a supported chunk size
+    (dict(chunk_size=512), 2),
+    (dict(headdim=512), 2),
+    (dict(dstate=300), 2),
+])
+def test_shape_rejections(L, kw, code):
+    st, _ = ws_size(L, shape(**kw))
+    assert st == code
+
+
+def test_workspace_size_monotone(L):
+    st, a = ws_size(L, shape(seqlen=256))
+    assert st == 0 and a > 0
+    st, b = ws_size(L, shape(seqlen=512))
+    assert st == 0 and b > a
+    st, z = ws_size(L, shape(seqlen=0))
+    assert st == 0 and z == 0
+
+
+class Bufs:
+    """Real device buffers on a CUDA machine, otherwise placeholder addresses."""
+
+    def __init__(self, s):
+        self.real = torch.cuda.is_available()
+        b, T, H, P, G, N = s.batch, s.seqlen, s.nheads, s.headdim, s.ngroups, s.dstate
+        es = 2 if s.dtype == 1 else 4
+        sizes = dict(x=b * T * H * P * es, dt=b * T * H * 4, A=H * 4, B=b * T * G * N * es,
+                     C=b * T * G * N * es, D=H * 4, init=b * H * P * N * 4, y=b * T * H * P * es,
+                     final=b * H * P * N * 4)
+        _, ws = ws_size(lib_mod(), s)
+        sizes["ws"] = ws
+        self.t = {}
+        self.addr = {}
+        base = 1 << 40
+        for k, n in sizes.items():
+            if self.real:
+                self.t[k] = torch.empty(max(n, 16), dtype=torch.uint8, device="cuda")
+                self.addr[k] = self.t[k].data_ptr()
+            else:
+                self.addr[k] = base
+                base += ((n + 4095) // 4096 + 1) * 4096
+        self.ws_bytes = ws
+
+    def p(self, k):
+        return ctypes.c_void_p(self.addr[k]) if k else None
+
+
+def lib_mod():
+    from structured_state_space_fwd_b200 import _lib
+    return _lib
+
+
+def call_fwd(L, s, bufs, **over):
+    names = ["x", "dt", "A", "B", "C", "D", "init", "y", "final", "ws"]
+    args = {k: bufs.p(k) for k in names}
+    ws_bytes = over.pop("ws_bytes", bufs.ws_bytes)
+    for k, v in over.items():
+        args[k] = v
+    return L.lib().ssd_fwd(ctypes.byref(s), args["x"], args["dt"], args["A"], args["B"],
+                           args["C"], args["D"], args["init"], args["y"], args["final"],
+                           args["ws"], ctypes.c_size_t(ws_bytes), None)
+
+
+def off(bufs, k, delta):
+    return ctypes.c_void_p(bufs.addr[k] + delta)
+
+
+@pytest.mark.parametrize("case", ["null_x", "null_y", "null_dt", "misaligned_x", "misaligned_y",
+                                  "y_is_x", "y_overlaps_B", "final_is_init", "final_overlaps_y",
+                                  "small_ws", "null_ws", "ws_overlaps_x", "bad_shape"])
+def test_fwd_argument_rejections(L, case):
+    s = shape()
+    bufs = Bufs(s)
+    over = {
+        "null_x": dict(x=None), "null_y": dict(y=None), "null_dt": dict(dt=None),
+        "misaligned_x": dict(x=off(bufs, "x", 2)), "misaligned_y": dict(y=off(bufs, "y", 8)),
+        "y_is_x": dict(y=bufs.p("x")), "y_overlaps_B": dict(y=off(bufs, "B", 16)),
+        "final_is_init": dict(final=bufs.p("init")),
+        "final_overlaps_y": dict(final=bufs.p("y")),
+        "small_ws": dict(ws_bytes=bufs.ws_bytes - 1), "null_ws": dict(ws=None),
+        "ws_overlaps_x": dict(ws=bufs.p("x")),
+        "bad_shape": None,
+    }[case]
+    if over is None:
+        st = call_fwd(L, shape(nheads=5, ngroups=2), bufs)
+    else:
+        st = call_fwd(L, s, bufs, **over)
+    assert st == 1
+
+
+def test_step_entry_rejections(L):
+    s = shape()
+    bufs = Bufs(s)
+    lib = L.lib()
+    assert lib.ssd_chunk_cumsum(ctypes.byref(s), None, bufs.p("A"), bufs.p("ws"), None) == 1
+    assert lib.ssd_chunk_cumsum(ctypes.byref(s), bufs.p("dt"), bufs.p("A"), bufs.p("dt"), None) == 1
+    assert lib.ssd_chunk_state(ctypes.byref(s), bufs.p("x"), bufs.p("dt"), bufs.p("B"),
+                               bufs.p("ws"), bufs.p("x"), None) == 1
+    assert lib.ssd_state_passing(ctypes.byref(s), bufs.p("ws"), bufs.p("ws"), None, None,
+                                 None, None) == 1
+    assert lib.ssd_chunk_scan(ctypes.byref(s), bufs.p("x"), bufs.p("dt"), bufs.p("B"),
+                              bufs.p("C"), None, bufs.p("ws"), bufs.p("ws"), bufs.p("x"),
+                              None) == 1
+    bad = shape(chunk_size=100)
+    assert lib.ssd_chunk_cumsum(ctypes.byref(bad), bufs.p("dt"), bufs.p("A"), bufs.p("ws"),
+                                None) == 2
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    from structured_state_space_fwd_b200 import _lib
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "lib_path", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        _lib.lib()

@@ -1,0 +1,225 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Metric: max|y - y_ref| / max|y_ref| over the compared elements, the same for
+final states. Bars: 5e-3 for bf16 storage (fp32 accumulation), 1e-5 for the
+fp32 path. Small cases compare every element; full-size workloads compare
+whole (batch, head) sequences the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import ssd_inputs as W
+from ssd_inputs import make_inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-5, "bf16": 5e-3}
+
+
+@pytest.fixture(scope="module")
+def ssd(cuda_device):
+    from structured_state_space_fwd_b200 import build
+    build.build()
+    import structured_state_space_fwd_b200 as m
+    return m
+
+
+def to_dev(inp):
+    return {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+
+
+def run(ssd, inp, Q, final=True):
+    d = to_dev(inp)
+    out = ssd.ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], chunk_size=Q,
+                      initial_states=d["initial_states"], return_final_states=final)
+    torch.cuda.synchronize()
+    return out
+
+
+def check_full(ssd, inp, Q, dtype, tol=None):
+    tol = tol or TOL[dtype]
+    y, fin = run(ssd, inp, Q)
+    y_ref, f_ref, _ = oracle.recurrence(**inp)
+    ey = oracle.rel_err(y.float().cpu(), y_ref)
+    ef = oracle.rel_err(fin.cpu(), f_ref)
+    assert ey <= tol, f"y rel err {ey:.3e} > {tol}"
+    assert ef <= tol, f"final rel err {ef:.3e} > {tol}"
+    return ey, ef
+
+
+def test_tiny_fp32_workload(ssd):
+    w = W.TINY_FP32
+    inp = W.workload_inputs(w)
+    check_full(ssd, inp, w.chunk_size, "f32")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("Q", [16, 32, 64, 128, 256])
+def test_small_ragged(ssd, dtype, Q):
+    # T = 300 is not a multiple of any chunk size; several chunks and a partial tail.
+    inp = make_inputs(batch=2, seqlen=300, nheads=4, headdim=64, ngroups=2, dstate=64,
+                      dtype=dtype, initial_states=True, seed=Q)
+    check_full(ssd, inp, Q, dtype)
+
+
+@pytest.mark.parametrize("P,N,G,H", [(16, 16, 1, 2), (32, 128, 1, 3), (64, 256, 4, 8),
+                                     (128, 32, 2, 2), (48, 24, 1, 2), (256, 256, 1, 1),
+                                     (7, 5, 1, 3)])
+def test_shapes(ssd, P, N, G, H):
+    for dtype in ("f32", "bf16"):
+        inp = make_inputs(batch=1, seqlen=200, nheads=H, headdim=P, ngroups=G, dstate=N,
+                          dtype=dtype, initial_states=(N % 2 == 0), seed=P + N)
+        check_full(ssd, inp, 64, dtype)
+
+
+def test_no_D_no_init(ssd):
+    inp = make_inputs(batch=2, seqlen=130, nheads=2, headdim=64, ngroups=1, dstate=32,
+                      dtype="bf16", with_D=False, seed=3)
+    check_full(ssd, inp, 64, "bf16")
+
+
+def test_seqlen_one_and_shorter_than_chunk(ssd):
+    for T in (1, 5, 63):
+        inp = make_inputs(batch=3, seqlen=T, nheads=2, headdim=32, ngroups=1, dstate=16,
+                          dtype="f32", initial_states=True, seed=T)
+        check_full(ssd, inp, 64, "f32")
+
+
+def test_empty_sequence_returns_initial_state(ssd):
+    inp = make_inputs(batch=2, seqlen=0, nheads=2, headdim=16, ngroups=1, dstate=16,
+                      dtype="bf16", initial_states=True, seed=0)
+    y, fin = run(ssd, inp, 64)
+    assert y.numel() == 0
+    assert torch.equal(fin.cpu(), inp["initial_states"])
+    inp["initial_states"] = None
+    y, fin = run(ssd, inp, 64)
+    assert torch.count_nonzero(fin).item() == 0
+
+
+def test_empty_batch(ssd):
+    inp = make_inputs(batch=0, seqlen=64, nheads=2, headdim=16, ngroups=1, dstate=16,
+                      dtype="bf16", seed=0)
+    y, fin = run(ssd, inp, 64)
+    assert y.numel() == 0 and fin.numel() == 0
+
+
+def test_steps_against_oracle(ssd):
+    # Each of the four steps, through its own entry point, against the oracle's
+    # definition of the step's output.
+    Q = 64
+    inp = make_inputs(batch=2, seqlen=200, nheads=4, headdim=32, ngroups=2, dstate=48,
+                      dtype="bf16", initial_states=True, seed=11)
+    d = to_dev(inp)
+    shp = ssd.make_shape(d["x"], d["B"], Q)
+    cs = ssd.ssd_chunk_cumsum(d["dt"], d["A"], Q, shp)
+    cs_ref = oracle.chunk_cumsum(inp["dt"], inp["A"], Q)
+    torch.cuda.synchronize()
+    assert np.max(np.abs(cs.cpu().double().numpy() - cs_ref)) <= 1e-5 * max(1.0, np.max(np.abs(cs_ref)))
+
+    S = ssd.ssd_chunk_state(d["x"], d["dt"], d["B"], cs, shp)
+    S_ref = oracle.chunk_states(inp["x"], inp["dt"], inp["A"], inp["B"], Q)
+    torch.cuda.synchronize()
+    assert oracle.rel_err(S.cpu(), S_ref) <= 1e-5
+
+    entry, fin = ssd.ssd_state_passing(S, cs, shp, initial_states=d["initial_states"])
+    y_ref, f_ref, e_ref = oracle.recurrence(**inp, chunk_size=Q)
+    torch.cuda.synchronize()
+    assert oracle.rel_err(entry.cpu(), e_ref) <= 1e-5
+    assert oracle.rel_err(fin.cpu(), f_ref) <= 1e-5
+
+    # step 4 from the oracle's own entry states, so its error is its own
+    e_dev = torch.from_numpy(e_ref).float().cuda()
+    y = ssd.ssd_chunk_scan(d["x"], d["dt"], d["B"], d["C"], d["D"], cs, e_dev, shp)
+    torch.cuda.synchronize()
+    assert oracle.rel_err(y.float().cpu(), y_ref) <= 5e-3
+
+
+def test_chunk_size_invariance(ssd):
+    inp = make_inputs(batch=1, seqlen=1000, nheads=4, headdim=64, ngroups=1, dstate=128,
+                      dtype="bf16", initial_states=True, seed=5)
+    outs = [run(ssd, inp, Q) for Q in (64, 128, 256)]
+    y_ref, f_ref, _ = oracle.recurrence(**inp)
+    for y, f in outs:
+        assert oracle.rel_err(y.float().cpu(), y_ref) <= 5e-3
+        assert oracle.rel_err(f.cpu(), f_ref) <= 5e-3
+
+
+def test_continuation_on_gpu(ssd):
+    # Knowl 8: split the sequence, pass the final state of the first part as the
+    # initial state of the second; equals one call on the whole sequence.
+    inp = make_inputs(batch=2, seqlen=700, nheads=2, headdim=64, ngroups=1, dstate=64,
+                      dtype="f32", initial_states=True, seed=9)
+    y, f = run(ssd, inp, 128)
+    T1 = 333
+    a = {k: (v[:, :T1].contiguous() if k in ("x", "dt", "B", "C") else v) for k, v in inp.items()}
+    y1, f1 = run(ssd, a, 128)
+    b = {k: (v[:, T1:].contiguous() if k in ("x", "dt", "B", "C") else v) for k, v in inp.items()}
+    b["initial_states"] = f1.cpu()
+    y2, f2 = run(ssd, b, 128)
+    assert oracle.rel_err(torch.cat([y1, y2], 1).cpu(), y.cpu()) <= 1e-5
+    assert oracle.rel_err(f2.cpu(), f.cpu()) <= 1e-5
+
+
+def test_deterministic(ssd):
+    inp = make_inputs(batch=2, seqlen=512, nheads=4, headdim=64, ngroups=1, dstate=128,
+                      dtype="bf16", initial_states=True, seed=1)
+    y1, f1 = run(ssd, inp, 256)
+    y2, f2 = run(ssd, inp, 256)
+    assert torch.equal(y1, y2) and torch.equal(f1, f2)
+
+
+def test_host_buffer_entry_point(ssd):
+    inp = make_inputs(batch=2, seqlen=300, nheads=4, headdim=64, ngroups=2, dstate=64,
+                      dtype="bf16", initial_states=True, seed=2)
+    pinned = {k: (v.pin_memory() if v is not None else None) for k, v in inp.items()}
+    y = torch.empty_like(pinned["x"]).pin_memory()
+    fin = torch.empty(tuple(inp["initial_states"].shape), dtype=torch.float32).pin_memory()
+    ssd.ssd_fwd_host(pinned["x"], pinned["dt"], pinned["A"], pinned["B"], pinned["C"],
+                     pinned["D"], chunk_size=128, initial_states=pinned["initial_states"],
+                     y=y, final_states=fin)
+    yd, fd = run(ssd, inp, 128)
+    assert torch.equal(y, yd.cpu()) and torch.equal(fin, fd.cpu())
+
+
+# ---------------------------------------------------------------- full size
+def sampled_check(ssd, w, pairs, seed=0):
+    inp = W.workload_inputs(w, seed=seed)
+    y, fin = run(ssd, inp, w.chunk_size)
+    y_ref, f_ref, _ = oracle.recurrence(**inp, bh_list=pairs)
+    yc = y.float().cpu().numpy()
+    fc = fin.cpu().numpy()
+    ys = np.stack([yc[b, :, h] for b, h in pairs])
+    yr = np.stack([y_ref[b, :, h] for b, h in pairs])
+    fs = np.stack([fc[b, h] for b, h in pairs])
+    fr = np.stack([f_ref[b, h] for b, h in pairs])
+    ey, ef = oracle.rel_err(ys, yr), oracle.rel_err(fs, fr)
+    assert np.isfinite(yc).all() and np.isfinite(fc).all()
+    assert ey <= TOL[w.dtype], f"{w.name}: y rel err {ey:.3e}"
+    assert ef <= TOL[w.dtype], f"{w.name}: final rel err {ef:.3e}"
+    return ey, ef
+
+
+def corners(b, H):
+    return sorted({(0, 0), (b - 1, H - 1), (b // 2, H // 2), (0, H - 1), (b - 1, 0)})
+
+
+def test_full_mamba2_layer(ssd):
+    w = W.MAMBA2_27B_LAYER
+    sampled_check(ssd, w, corners(w.batch, w.nheads) + [(3, 41)])
+
+
+@pytest.mark.parametrize("w", W.seqlen_sweep(), ids=lambda w: w.name)
+def test_full_seqlen_sweep(ssd, w):
+    sampled_check(ssd, w, corners(w.batch, w.nheads)[:3])
+
+
+@pytest.mark.parametrize("w", W.dstate_sweep(), ids=lambda w: w.name)
+def test_full_dstate_sweep(ssd, w):
+    sampled_check(ssd, w, corners(w.batch, w.nheads)[:3])
+
+
+def test_full_long_context(ssd):
+    w = W.LONG_CONTEXT
+    sampled_check(ssd, w, [(0, 0), (0, 5), (0, 18), (0, 31)])
