@@ -111,6 +111,31 @@ SSD_API ssd_status_t ssd_fwd(const ssd_shape_t* shape,
                      void* y, float* final_states,
                      void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * ssd_fwd without a caller-provided workspace, for callers that cannot
+ * allocate device memory: hosts that own every device allocation and give a
+ * library only its input and output buffers, or call paths that cannot afford
+ * cudaMalloc's possible device-wide synchronization. The pages describe no
+ * such entry point; it is a deployment convenience of this library.
+ *   Arguments are those of ssd_fwd minus the workspace. Scratch space comes
+ *   from one static device array of 64 MiB that every GPU loading libssd
+ *   reserves until the process exits. A shape whose ssd_fwd workspace
+ *   (ssd_fwd_workspace_size) exceeds 64 MiB is rejected with
+ *   SSD_ERR_UNSUPPORTED before anything is enqueued; ssd_last_error_detail()
+ *   then says so. The library allocates nothing on this path.
+ *   The first call on a device looks up that device's scratch address
+ *   (cudaGetSymbolAddress, with the device current); make that first call
+ *   before any stream capture. All calls on a device share the one array and
+ *   it keeps the last call's contents, which no call relies on; calls that can
+ *   overlap on the GPU (different streams, or different host threads without
+ *   ordering) race on it and must be serialized by the caller.
+ */
+SSD_API ssd_status_t ssd_fwd_no_alloc(const ssd_shape_t* shape,
+                                      const void* x, const float* dt, const float* A,
+                                      const void* B, const void* C, const float* D,
+                                      const float* initial_states,
+                                      void* y, float* final_states, void* stream);
+
 /* Bytes of device workspace ssd_fwd_host needs (inputs, outputs and ssd_fwd's
  * own workspace are staged there). */
 SSD_API ssd_status_t ssd_fwd_host_workspace_size(const ssd_shape_t* shape, size_t* bytes);

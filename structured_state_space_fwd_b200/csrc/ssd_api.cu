@@ -165,6 +165,8 @@ ssd_status_t run_fwd(const ssd::Dims& d, const void* x, const float* dt, const f
 
 }  // namespace
 
+void ssd::set_error_detail(const char* msg) { snprintf(g_detail, sizeof(g_detail), "%s", msg); }
+
 extern "C" {
 
 const char* ssd_status_string(ssd_status_t s) {

@@ -32,6 +32,9 @@ cudaError_t launch_state_passing(const Dims& d, const float* states, const float
 cudaError_t launch_chunk_scan_simt(const Dims& d, const void* x, const float* dt, const void* B,
                                    const void* C, const float* D, const float* cs,
                                    const float* entry, void* y, cudaStream_t st);
+// Sets the message ssd_last_error_detail() returns on the calling host thread.
+void set_error_detail(const char* msg);
+
 cudaError_t launch_copy_or_zero_states(const Dims& d, const float* init, float* final_states,
                                        cudaStream_t st);
 
