@@ -6,6 +6,7 @@
 
 #include <algorithm>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <initializer_list>
 
@@ -84,18 +85,48 @@ Sizes sizes_of(const ssd::Dims& d) {
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Workspace of ssd_fwd: [cs | chunk states S | entry states h_c], each 256-byte aligned.
+// Which kernels ssd_fwd runs. SSD_PATH=steps forces the four separate steps,
+// SSD_PATH=simt the CUDA-core kernels only (for testing the paths against
+// each other); by default the fused tensor-core kernel runs where supported.
+enum class Path { Fused, Steps, Simt };
+
+Path pick_path(const ssd::Dims& d) {
+    const char* e = getenv("SSD_PATH");
+    const bool tc = ssd::tc_supported(d);
+    if (e && strcmp(e, "simt") == 0) return Path::Simt;
+    if (e && strcmp(e, "steps") == 0) return tc ? Path::Steps : Path::Simt;
+    return tc ? Path::Fused : Path::Simt;
+}
+
+bool steps_use_tc(const ssd::Dims& d) {
+    const char* e = getenv("SSD_PATH");
+    return !(e && strcmp(e, "simt") == 0) && ssd::tc_supported(d);
+}
+
+// Workspace of ssd_fwd, regions 256-byte aligned:
+//   fused path:  [sync ints: ticket, error, flags[b*H] | chain state [b,H,P,N]]
+//   step paths:  [cs | chunk states S | entry states h_c]
 struct FwdWorkspace {
-    size_t off_cs, off_S, off_entry, total;
+    Path path;
+    size_t off_cs, off_S, off_entry;   // step paths
+    size_t off_sync, off_chain;        // fused path
+    size_t total;
 };
 
 FwdWorkspace fwd_workspace(const ssd::Dims& d) {
     const Sizes z = sizes_of(d);
-    FwdWorkspace w;
-    w.off_cs = 0;
-    w.off_S = align_up(z.cs, 256);
-    w.off_entry = w.off_S + align_up(z.chunk_states, 256);
-    w.total = w.off_entry + align_up(z.chunk_states, 256);
+    FwdWorkspace w = {};
+    w.path = pick_path(d);
+    if (w.path == Path::Fused) {
+        w.off_sync = 0;
+        w.off_chain = align_up(sizeof(int) * (size_t)(2 + d.b * d.H), 256);
+        w.total = w.off_chain + align_up(z.st, 256);
+    } else {
+        w.off_cs = 0;
+        w.off_S = align_up(z.cs, 256);
+        w.off_entry = w.off_S + align_up(z.chunk_states, 256);
+        w.total = w.off_entry + align_up(z.chunk_states, 256);
+    }
     if (d.b == 0 || d.T == 0) w.total = 0;
     return w;
 }
@@ -147,20 +178,29 @@ ssd_status_t run_fwd(const ssd::Dims& d, const void* x, const float* dt, const f
     if (d.T == 0) return cuda_status("final states", ssd::launch_copy_or_zero_states(d, init, final_states, stream));
     const FwdWorkspace w = fwd_workspace(d);
     char* ws = (char*)workspace;
+    if (w.path == Path::Fused) {
+        float* chain = final_states ? final_states : (float*)(ws + w.off_chain);
+        return cuda_status("fused forward",
+                           ssd::launch_fused_tc(d, x, dt, A, B, C, D, init, y, chain,
+                                                (int*)(ws + w.off_sync), stream));
+    }
     float* cs = (float*)(ws + w.off_cs);
     float* S = (float*)(ws + w.off_S);
     float* entry = (float*)(ws + w.off_entry);
+    const bool tc = w.path == Path::Steps;
     ssd_status_t st;
     if ((st = cuda_status("chunk cumsum", ssd::launch_chunk_cumsum(d, dt, A, cs, stream))) != SSD_OK)
         return st;
     if ((st = cuda_status("chunk state",
-                          ssd::launch_chunk_state_simt(d, x, dt, B, cs, S, stream))) != SSD_OK)
+                          tc ? ssd::launch_chunk_state_tc(d, x, dt, B, cs, S, stream)
+                             : ssd::launch_chunk_state_simt(d, x, dt, B, cs, S, stream))) != SSD_OK)
         return st;
     if ((st = cuda_status("state passing", ssd::launch_state_passing(d, S, cs, init, entry,
                                                                       final_states, stream))) != SSD_OK)
         return st;
     return cuda_status("chunk scan",
-                       ssd::launch_chunk_scan_simt(d, x, dt, B, C, D, cs, entry, y, stream));
+                       tc ? ssd::launch_chunk_scan_tc(d, x, dt, B, C, D, cs, entry, y, stream)
+                          : ssd::launch_chunk_scan_simt(d, x, dt, B, C, D, cs, entry, y, stream));
 }
 
 }  // namespace
@@ -295,6 +335,9 @@ ssd_status_t ssd_chunk_state(const ssd_shape_t* shape, const void* x, const floa
     if (overlaps(o, {x, z.x}) || overlaps(o, {dt, z.dt}) || overlaps(o, {B, z.bc}) ||
         overlaps(o, {cs, z.cs}))
         return SSD_ERR_INVALID_ARG;
+    if (steps_use_tc(d))
+        return cuda_status("chunk state", ssd::launch_chunk_state_tc(d, x, dt, B, cs, states,
+                                                                       (cudaStream_t)stream));
     return cuda_status("chunk state", ssd::launch_chunk_state_simt(d, x, dt, B, cs, states,
                                                                      (cudaStream_t)stream));
 }
@@ -336,6 +379,10 @@ ssd_status_t ssd_chunk_scan(const ssd_shape_t* shape, const void* x, const float
                          {cs, z.cs}, {entry_states, z.chunk_states}};
     for (const Range& i : ins)
         if (overlaps(o, i)) return SSD_ERR_INVALID_ARG;
+    if (steps_use_tc(d))
+        return cuda_status("chunk scan", ssd::launch_chunk_scan_tc(d, x, dt, B, C, D, cs,
+                                                                     entry_states, y,
+                                                                     (cudaStream_t)stream));
     return cuda_status("chunk scan", ssd::launch_chunk_scan_simt(d, x, dt, B, C, D, cs,
                                                                    entry_states, y,
                                                                    (cudaStream_t)stream));

@@ -32,6 +32,18 @@ cudaError_t launch_state_passing(const Dims& d, const float* states, const float
 cudaError_t launch_chunk_scan_simt(const Dims& d, const void* x, const float* dt, const void* B,
                                    const void* C, const float* D, const float* cs,
                                    const float* entry, void* y, cudaStream_t st);
+// Tensor-core path (sm_100a tcgen05): bf16, head dim 64, state dim 128, chunk 128/256.
+bool tc_supported(const Dims& d);
+cudaError_t launch_chunk_state_tc(const Dims& d, const void* x, const float* dt, const void* B,
+                                  const float* cs, float* states, cudaStream_t st);
+cudaError_t launch_chunk_scan_tc(const Dims& d, const void* x, const float* dt, const void* B,
+                                 const void* C, const float* D, const float* cs,
+                                 const float* entry, void* y, cudaStream_t st);
+// Whole forward in one kernel; sync_ints holds 2 + b*H ints, chain b*H*P*N floats.
+cudaError_t launch_fused_tc(const Dims& d, const void* x, const float* dt, const float* A,
+                            const void* B, const void* C, const float* D, const float* init,
+                            void* y, float* chain, int* sync_ints, cudaStream_t st);
+
 // Sets the message ssd_last_error_detail() returns on the calling host thread.
 void set_error_detail(const char* msg);
 

@@ -223,3 +223,67 @@ def test_full_dstate_sweep(ssd, w):
 def test_full_long_context(ssd):
     w = W.LONG_CONTEXT
     sampled_check(ssd, w, [(0, 0), (0, 5), (0, 18), (0, 31)])
+
+
+# ---------------------------------------------------------------- tensor-core path
+# bf16, head dim 64, state dim 128, chunk 128 or 256 run on the tcgen05 kernels:
+# the fused kernel by default, the separate tensor-core steps with SSD_PATH=steps.
+@pytest.fixture
+def path_env(monkeypatch):
+    def set_path(p):
+        if p == "fused":
+            monkeypatch.delenv("SSD_PATH", raising=False)
+        else:
+            monkeypatch.setenv("SSD_PATH", p)
+    return set_path
+
+
+@pytest.mark.parametrize("path", ["fused", "steps"])
+@pytest.mark.parametrize("Q", [128, 256])
+@pytest.mark.parametrize("T", [1, 100, 256, 700, 1300])
+def test_tensor_path_ragged(ssd, path_env, path, Q, T):
+    path_env(path)
+    inp = make_inputs(batch=2, seqlen=T, nheads=8, headdim=64, ngroups=2, dstate=128,
+                      dtype="bf16", initial_states=True, seed=T + Q)
+    check_full(ssd, inp, Q, "bf16")
+
+
+@pytest.mark.parametrize("path", ["fused", "steps"])
+@pytest.mark.parametrize("H,G", [(1, 1), (3, 1), (6, 3), (5, 5), (12, 1)])
+def test_tensor_path_head_blocks(ssd, path_env, path, H, G):
+    path_env(path)
+    inp = make_inputs(batch=3, seqlen=520, nheads=H, headdim=64, ngroups=G, dstate=128,
+                      dtype="bf16", initial_states=(H % 2 == 0), seed=H * 10 + G)
+    check_full(ssd, inp, 256, "bf16")
+
+
+def test_tensor_steps_against_oracle(ssd, path_env):
+    path_env("steps")
+    Q = 256
+    inp = make_inputs(batch=2, seqlen=600, nheads=4, headdim=64, ngroups=1, dstate=128,
+                      dtype="bf16", initial_states=True, seed=21)
+    d = to_dev(inp)
+    shp = ssd.make_shape(d["x"], d["B"], Q)
+    cs = ssd.ssd_chunk_cumsum(d["dt"], d["A"], Q, shp)
+    S = ssd.ssd_chunk_state(d["x"], d["dt"], d["B"], cs, shp)
+    S_ref = oracle.chunk_states(inp["x"], inp["dt"], inp["A"], inp["B"], Q)
+    torch.cuda.synchronize()
+    assert oracle.rel_err(S.cpu(), S_ref) <= 5e-3
+    y_ref, f_ref, e_ref = oracle.recurrence(**inp, chunk_size=Q)
+    e_dev = torch.from_numpy(e_ref).float().cuda()
+    y = ssd.ssd_chunk_scan(d["x"], d["dt"], d["B"], d["C"], d["D"], cs, e_dev, shp)
+    torch.cuda.synchronize()
+    assert oracle.rel_err(y.float().cpu(), y_ref) <= 5e-3
+
+
+def test_paths_agree(ssd, path_env):
+    inp = make_inputs(batch=2, seqlen=900, nheads=4, headdim=64, ngroups=1, dstate=128,
+                      dtype="bf16", initial_states=True, seed=33)
+    outs = {}
+    for p in ("fused", "steps", "simt"):
+        path_env(p)
+        outs[p] = run(ssd, inp, 256)
+    y_ref, f_ref, _ = oracle.recurrence(**inp)
+    for p, (y, f) in outs.items():
+        assert oracle.rel_err(y.float().cpu(), y_ref) <= 5e-3, p
+        assert oracle.rel_err(f.cpu(), f_ref) <= 5e-3, p
