@@ -39,6 +39,9 @@ WORKLOAD = W.MAMBA2_27B_LAYER
 METRIC = "SSD fwd Mtokens/s & TFLOP/s at 2.7B layer shape; % of bf16/HBM roofline"
 UNIT = "Mtokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant kernel, from
+# one ncu capture of this workload (profiles/); None until captured for the current kernel
+TRAFFIC = {}
 
 
 # ------------------------------------------------------------------ counts
@@ -264,11 +267,19 @@ def run_ours(args):
                     y=bufs["y"], final_states=bufs["final"], return_final_states=True,
                     workspace=ws, stream=stream)
 
+    path_name, kernels_per_step = ssd.ssd_fwd_plan(shp)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
 
     clocks = ClockSampler(local)
+    # keep the GPU busy for ~0.5 s before the timed region so that the clock
+    # samples taken around it reflect clocks under this load (untimed)
+    t_soak = time.perf_counter()
+    while time.perf_counter() - t_soak < args.soak_s:
+        for _ in range(20):
+            step()
+        torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -289,31 +300,38 @@ def run_ours(args):
     t_roof = max(F / (pk["bf16_tflops"] * 1e12), by / (pk["hbm_gbs"] * 1e9))
     step_s = ms_step / 1e3
 
-    # per-kernel launch durations (each kernel timed alone, same inputs, CUDA events)
-    plan = kernel_plan(ssd, w, d, bufs, stream)
-    ktimes = {}
-    reps = max(3, min(50, args.steps))
-    for name, fn, _ in plan:
-        for _ in range(2):
-            fn()
-        k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        k0.record(stream)
-        for _ in range(reps):
-            fn()
-        k1.record(stream)
-        torch.cuda.synchronize()
-        ktimes[name] = k0.elapsed_time(k1) / reps
-    dom = max(plan, key=lambda p: ktimes[p[0]])
+    # dominant kernel and its average launch duration (CUDA events on its stream)
+    if path_name == "fused":
+        # one kernel per step: the fused forward; its launch duration is the
+        # timed step (which also holds the small counter memset before it)
+        ktimes = {"ssd_tc_kernel<fused>": ms_step}
+        dom = ("ssd_tc_kernel<fused>", None, by)
+    else:
+        plan = kernel_plan(ssd, w, d, bufs, stream)
+        ktimes = {}
+        reps = max(3, min(50, args.steps))
+        for name, fn, _ in plan:
+            for _ in range(2):
+                fn()
+            k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            k0.record(stream)
+            for _ in range(reps):
+                fn()
+            k1.record(stream)
+            torch.cuda.synchronize()
+            ktimes[name] = k0.elapsed_time(k1) / reps
+        dom = max(plan, key=lambda p: ktimes[p[0]])
     dom_s = ktimes[dom[0]] / 1e3
     achieved = dom[2] / dom_s / 1e9
     roofline = {"kernel": dom[0], "bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
-                "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": None,
-                "peak_source": pk_kind + " (burst copy)",
+                "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": TRAFFIC.get(path_name),
+                "peak_source": pk_kind + " (burst copy, MEASURED_PEAKS hbm_gbs)",
+                "alg_bytes_per_launch": dom[2], "path": path_name,
                 "kernel_ms": {k: round(v, 5) for k, v in ktimes.items()}}
 
     # end to end through the host-buffer entry point (pinned host memory)
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not args.profile:
         hp = {k: (v.pin_memory() if v is not None else None) for k, v in inp.items()}
         hy = torch.empty_like(hp["x"]).pin_memory()
         hf = torch.empty((b, H, P, N), dtype=torch.float32).pin_memory()
@@ -346,7 +364,7 @@ def run_ours(args):
                "ms_per_step": ms_e2e, "api": "ssd_fwd_host (pinned host buffers)"}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.profile:
         run, tok, desc, threads = oracle_sample(w, 15.0, inputs64=inp)
         t0 = time.perf_counter()
         run()
@@ -369,7 +387,7 @@ def run_ours(args):
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": 4 * args.steps,
+            "gpu_launches": kernels_per_step * args.steps,
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)
@@ -382,11 +400,15 @@ def run_ours(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--soak-s", type=float, default=0.5,
+                    help="untimed load before the timed region, for the clock samples")
+    ap.add_argument("--profile", action="store_true",
+                    help="warmup and timed steps only (for ncu): no e2e, no CPU baseline")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -86,6 +86,13 @@ SSD_API const char* ssd_last_error_detail(void);
 /* Library version as major*10000 + minor*100 + patch. */
 SSD_API int ssd_version(void);
 
+/* Which kernels ssd_fwd launches for `shape` (host-only query, nothing runs):
+ * *path receives a static name ("fused": one tensor-core kernel per call;
+ * "steps": the four step kernels on tensor cores; "simt": the four step kernels
+ * on CUDA cores) and *kernels the number of kernel launches per call (the
+ * fused path also enqueues one small memset of its workspace counters). */
+SSD_API ssd_status_t ssd_fwd_plan(const ssd_shape_t* shape, const char** path, int* kernels);
+
 /* Bytes of device workspace ssd_fwd needs for `shape`, written to *bytes.
  * Returns SSD_ERR_INVALID_ARG / SSD_ERR_UNSUPPORTED for a shape ssd_fwd rejects. */
 SSD_API ssd_status_t ssd_fwd_workspace_size(const ssd_shape_t* shape, size_t* bytes);

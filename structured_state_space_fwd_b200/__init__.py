@@ -22,7 +22,7 @@ import torch
 from ._lib import (SSD_BF16, SSD_F32, SSDError, ShapeT, check, lib, lib_path,  # noqa: F401
                    status_string)
 
-__all__ = ["ssd_fwd", "ssd_fwd_host", "ssd_fwd_workspace_size", "ssd_chunk_cumsum",
+__all__ = ["ssd_fwd", "ssd_fwd_host", "ssd_fwd_workspace_size", "ssd_fwd_plan", "ssd_chunk_cumsum",
            "ssd_chunk_state", "ssd_state_passing", "ssd_chunk_scan", "SSDError", "make_shape",
            "lib_path"]
 
@@ -57,6 +57,14 @@ def _need(t, name, dtype=None, device=True):
     if dtype is not None and t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     return t
+
+
+def ssd_fwd_plan(shape: ShapeT) -> tuple[str, int]:
+    """(path name, kernel launches per ssd_fwd call) for this shape."""
+    name = ctypes.c_char_p()
+    n = ctypes.c_int(0)
+    check(lib().ssd_fwd_plan(ctypes.byref(shape), ctypes.byref(name), ctypes.byref(n)), "ssd_fwd_plan")
+    return name.value.decode(), int(n.value)
 
 
 def ssd_fwd_workspace_size(shape: ShapeT) -> int:

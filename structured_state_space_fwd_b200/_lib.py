@@ -37,6 +37,8 @@ _SIGS = {
     "ssd_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "ssd_last_error_detail": ([], ctypes.c_char_p),
     "ssd_version": ([], ctypes.c_int),
+    "ssd_fwd_plan": ([ctypes.POINTER(ShapeT), ctypes.POINTER(ctypes.c_char_p),
+                      ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
     "ssd_fwd_workspace_size": ([ctypes.POINTER(ShapeT), ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
     "ssd_fwd": ([ctypes.POINTER(ShapeT)] + [_VP] * 10 + [ctypes.c_size_t, _VP], ctypes.c_int),
     "ssd_fwd_host_workspace_size": ([ctypes.POINTER(ShapeT), ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),

@@ -224,6 +224,17 @@ const char* ssd_last_error_detail(void) { return g_detail; }
 
 int ssd_version(void) { return 100; }
 
+ssd_status_t ssd_fwd_plan(const ssd_shape_t* shape, const char** path, int* kernels) {
+    if (!path || !kernels) return SSD_ERR_INVALID_ARG;
+    ssd_status_t st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    const ssd::Dims d = ssd::make_dims(*shape);
+    const Path p = pick_path(d);
+    *path = p == Path::Fused ? "fused" : (p == Path::Steps ? "steps" : "simt");
+    *kernels = (d.b == 0) ? 0 : (d.T == 0 ? 1 : (p == Path::Fused ? 1 : 4));
+    return SSD_OK;
+}
+
 ssd_status_t ssd_fwd_workspace_size(const ssd_shape_t* shape, size_t* bytes) {
     if (!bytes) return SSD_ERR_INVALID_ARG;
     ssd_status_t st = check_shape(shape);

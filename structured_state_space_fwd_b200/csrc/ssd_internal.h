@@ -1,6 +1,7 @@
 // Internal declarations shared by the library's translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -43,6 +44,13 @@ cudaError_t launch_chunk_scan_tc(const Dims& d, const void* x, const float* dt, 
 cudaError_t launch_fused_tc(const Dims& d, const void* x, const float* dt, const float* A,
                             const void* B, const void* C, const float* D, const float* init,
                             void* y, float* chain, int* sync_ints, cudaStream_t st);
+
+int pick_kheads(int64_t heads_per_group);
+// TMA maps of x, B, C (bf16, 4-D, 64 x 1 x 128 x 1 boxes, 128-byte swizzle).
+bool make_tc_maps(const Dims& d, const void* x, const void* B, const void* C, CUtensorMap* maps);
+cudaError_t launch_fused_ws(const Dims& d, const CUtensorMap* maps, const void* x, const float* dt,
+                            const float* A, const float* D, const float* init, void* y,
+                            float* chain, int* sync_ints, int kheads, cudaStream_t st);
 
 // Sets the message ssd_last_error_detail() returns on the calling host thread.
 void set_error_detail(const char* msg);

@@ -36,6 +36,8 @@
 #include <cuda_runtime.h>
 
 #include <cstdio>
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "sm100.cuh"
@@ -247,7 +249,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < nsub; ++s) {
             const int64_t t0 = tc0 + (int64_t)s * kTile;
             const int len = (int)min((int64_t)kTile, T - t0);
-            // previous users of sX / sP / sWX / sH and of the TMEM accumulators are done
+            // previous users of sX / sP / sWX / sH and of the TMEM accumulators are done;
+            // the generic-proxy reads of sX are ordered before the next TMA write into it
+            fence_proxy_async_smem();
             tc_fence_before();
             __syncthreads();
             if (tid == 0) {
@@ -481,11 +485,20 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+}  // namespace
+
 int pick_kheads(int64_t heads_per_group) {
     for (int k = 4; k > 1; --k)
         if (heads_per_group % k == 0) return k;
     return 1;
 }
+
+bool make_tc_maps(const Dims& d, const void* x, const void* B, const void* C, CUtensorMap* maps) {
+    return make_map(&maps[0], x, d.P, d.H, d.T, d.b) && make_map(&maps[1], B, d.N, d.G, d.T, d.b) &&
+           make_map(&maps[2], C ? C : B, d.N, d.G, d.T, d.b);
+}
+
+namespace {
 
 template <int kMode>
 cudaError_t launch_tc(const Dims& d, TcParams prm, const void* x, const void* B, const void* C,
@@ -547,6 +560,14 @@ cudaError_t launch_fused_tc(const Dims& d, const void* x, const float* dt, const
     // sync_ints: [0] ticket, [1] error, [2 ..] flags[b*H]; zeroed here.
     cudaError_t e = cudaMemsetAsync(sync_ints, 0, sizeof(int) * (size_t)(2 + d.b * d.H), st);
     if (e != cudaSuccess) return e;
+    const char* v = getenv("SSD_FUSED");
+    if (!(v && strcmp(v, "v0") == 0)) {
+        // default: the warp-specialized persistent kernel (ssd_fused.cu)
+        CUtensorMap maps[3];
+        if (!make_tc_maps(d, x, B, C, maps)) return cudaErrorInvalidValue;
+        return launch_fused_ws(d, maps, x, dt, A, D, init, y, chain, sync_ints,
+                               pick_kheads(d.H / d.G), st);
+    }
     TcParams prm = {};
     prm.x = (const __nv_bfloat16*)x;
     prm.dt = dt;

@@ -287,3 +287,29 @@ def test_paths_agree(ssd, path_env):
     for p, (y, f) in outs.items():
         assert oracle.rel_err(y.float().cpu(), y_ref) <= 5e-3, p
         assert oracle.rel_err(f.cpu(), f_ref) <= 5e-3, p
+
+
+# ---------------------------------------------------------------- fused kernel, whole tensors
+# The fused kernel against the four-step tensor-core path (itself checked against the
+# oracle above) on EVERY element of full-size workloads, and bitwise repeatability
+# across runs: a race between the kernel's warp roles shows up in either check.
+def _paths_full(ssd, path_env, w, seed=0, reps=3):
+    inp = W.workload_inputs(w, seed=seed)
+    path_env("steps")
+    y_ref, f_ref = run(ssd, inp, w.chunk_size)
+    path_env("fused")
+    outs = [run(ssd, inp, w.chunk_size) for _ in range(reps)]
+    ref_max = y_ref.float().abs().max().item()
+    for y, f in outs:
+        ey = (y.float() - y_ref.float()).abs().max().item() / ref_max
+        ef = ((f - f_ref).abs().max() / f_ref.abs().max()).item()
+        assert ey <= 5e-3, f"{w.name}: fused vs steps y rel err {ey:.3e}"
+        assert ef <= 5e-3, f"{w.name}: fused vs steps final rel err {ef:.3e}"
+    for y, f in outs[1:]:
+        assert torch.equal(y, outs[0][0]) and torch.equal(f, outs[0][1]), f"{w.name}: not repeatable"
+
+
+@pytest.mark.parametrize("w", [W.MAMBA2_27B_LAYER, W.seqlen_sweep()[4], W.LONG_CONTEXT],
+                         ids=lambda w: w.name)
+def test_fused_matches_steps_on_every_element(ssd, path_env, w):
+    _paths_full(ssd, path_env, w)
