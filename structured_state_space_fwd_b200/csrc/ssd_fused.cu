@@ -7,13 +7,16 @@
 // so that HBM traffic, tensor-core MMAs and CUDA-core work overlap:
 //
 //   warp 0      TMA producer: B/C tiles of a unit (one ring slot per 128-token
-//               tile), x tile of each item (3-deep ring)
+//               tile), x tile of each item (2-deep ring)
 //   warp 1      TMEM owner and MMA issuer (one thread)
 //   warp 2      per item: dt loads, cumulative sum of dt*A (log2 units) and the
 //               per-token factors exp(cs_last - cs_i) dt_i and exp(cs_j)
+//   warp 3      lane 0 releases chain flags
 //   warps 4-7   mask group: P = (C B^T) o mask from TMEM G into TMEM P (bf16,
 //               the A operand of the Y product), and w o x into shared memory
-//   warps 8-11  state/epilogue group: h as bf16 operand, h <- e h + S,
+//   warps 8-15  state/epilogue group, two warps per TMEM lane quarter, each
+//               owning half of the head dim: drains S, Y, R from TMEM, then
+//               h <- e h + S, the bf16 state operand, w o x of the next item,
 //               y = Y + exp(cs) R + D x to global memory, state hand-off
 //
 // Work: persistent CTAs take units (chunk c, batch row b, block of k heads of
@@ -41,18 +44,20 @@ using namespace sm100;
 constexpr int kTile = 128;
 constexpr int kP = 64;
 constexpr int kN = 128;
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
 constexpr int kXStages = 3;
+constexpr int kWXStages = 1;
 constexpr int kCsStages = 4;
+constexpr int kPubStages = 4;
 
 constexpr uint32_t kAtom = kTile * 128;          // 16 KB: 128 rows of 128 bytes
 constexpr uint32_t kBCSlot = 2 * (kN / 64) * kAtom;  // B and C of one tile: 64 KB
 constexpr uint32_t kOffBC = 0;                   // 2 slots
 constexpr uint32_t kOffX = kOffBC + 2 * kBCSlot;    // kXStages x 16 KB
 constexpr uint32_t kOffWX = kOffX + kXStages * kAtom;
-constexpr uint32_t kOffH = kOffWX + kAtom;
+constexpr uint32_t kOffH = kOffWX + kWXStages * kAtom;
 constexpr uint32_t kOffCs = kOffH + kN * 128;    // kCsStages x 4 arrays x 128 floats
-constexpr uint32_t kCsSlot = 5 * kTile * 4;   // cs, dt, w, u, v (per item)
+constexpr uint32_t kCsSlot = 6 * kTile * 4;   // cs, dt, w, u, v (per item), then D_h
 constexpr uint32_t kOffBar = kOffCs + kCsStages * kCsSlot;
 constexpr uint32_t kSmemBytes = kOffBar + 512;
 
@@ -82,8 +87,12 @@ struct Bars {
     uint64_t bc_full[2], bc_empty[2], g_full[2], g_empty[2];
     uint64_t x_full[kXStages], x_empty[kXStages];
     uint64_t cs_full[kCsStages], cs_empty[kCsStages];
-    uint64_t p_full, p_empty, wx_full, wx_empty, h_full, h_empty, acc_full, acc_empty, fin;
-    uint64_t chain_ok, pub;   // state hand-off inside the state/epilogue group
+    uint64_t wx_full[kWXStages], wx_empty[kWXStages];
+    uint64_t p_full, p_empty, h_full, h_empty, fin;
+    uint64_t sr_full, sr_empty;   // S and R accumulators (state product, C h^T)
+    uint64_t y_full, y_empty;     // Y accumulator (P x)
+    uint64_t chain_ok;                          // chain flag observed (state group)
+    uint64_t pub_full[kPubStages], pub_empty[kPubStages];  // state stored / flag released
     uint32_t tmem;
     int abort;
 };
@@ -137,6 +146,16 @@ __device__ __forceinline__ bool wait_bar_all(uint64_t* bar, uint32_t parity, Bar
     return __all_sync(0xffffffffu, ok);
 }
 
+// Half of a row of the bf16 state operand: thread (n, half) writes h[32 half + i][n],
+// i < 32, into chunks 4 half .. 4 half + 3 of row n.
+__device__ __forceinline__ void write_h_half(uint8_t* sh, int n, int half, const float (&hh)[32]) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+        *reinterpret_cast<uint4*>(sh + sw128_off(n, 4 * half + c)) =
+            make_uint4(pack_bf16(hh[8 * c], hh[8 * c + 1]), pack_bf16(hh[8 * c + 2], hh[8 * c + 3]),
+                       pack_bf16(hh[8 * c + 4], hh[8 * c + 5]), pack_bf16(hh[8 * c + 6], hh[8 * c + 7]));
+}
+
 // bf16 copy of the state as the B operand of C h^T: row n (one thread) holds
 // h[0..63][n], 128-byte swizzled rows.
 __device__ __forceinline__ void write_h_operand(uint8_t* sh, int n, const float (&hreg)[kP]) {
@@ -168,7 +187,8 @@ __device__ __forceinline__ Unit decode(const Params& p, int u) {
 __global__ void __launch_bounds__(kThreads, 1)
     ssd_fused_ws_kernel(const __grid_constant__ CUtensorMap tm_x,
                         const __grid_constant__ CUtensorMap tm_B,
-                        const __grid_constant__ CUtensorMap tm_C, const Params prm) {
+                        const __grid_constant__ CUtensorMap tm_C,
+                        const __grid_constant__ CUtensorMap tm_y, const Params prm) {
     extern __shared__ __align__(1024) uint8_t smem[];
     Bars* bs = reinterpret_cast<Bars*>(smem + kOffBar);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -184,28 +204,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int i = 0; i < kXStages; ++i) {
             mbar_init(&bs->x_full[i], 1);
-            mbar_init(&bs->x_empty[i], 1 + 128 + 128);
+            // Y product (commit) + state group twice (w o x, then the skip term x)
+            mbar_init(&bs->x_empty[i], 1 + 256 + 256);
         }
         for (int i = 0; i < kCsStages; ++i) {
             mbar_init(&bs->cs_full[i], 32);
-            mbar_init(&bs->cs_empty[i], 128 + 128);
+            mbar_init(&bs->cs_empty[i], 128 + 256);
         }
         mbar_init(&bs->p_full, 128);
         mbar_init(&bs->p_empty, 1);
-        mbar_init(&bs->wx_full, 128);
-        mbar_init(&bs->wx_empty, 1);
-        mbar_init(&bs->h_full, 128);
+        for (int i = 0; i < kWXStages; ++i) {
+            mbar_init(&bs->wx_full[i], 256);
+            mbar_init(&bs->wx_empty[i], 1);   // S product (commit)
+        }
+        mbar_init(&bs->h_full, 256);
         mbar_init(&bs->h_empty, 1);
-        mbar_init(&bs->acc_full, 1);
-        mbar_init(&bs->acc_empty, 128);
+        mbar_init(&bs->sr_full, 1);
+        mbar_init(&bs->sr_empty, 256);
+        mbar_init(&bs->y_full, 1);
+        mbar_init(&bs->y_empty, 256);
         mbar_init(&bs->fin, 1);
         mbar_init(&bs->chain_ok, 1);
-        mbar_init(&bs->pub, 128);
+        for (int i = 0; i < kPubStages; ++i) {
+            mbar_init(&bs->pub_full[i], 256);
+            mbar_init(&bs->pub_empty[i], 1);
+        }
         bs->abort = 0;
         fence_barrier_init();
         prefetch_tmap(&tm_x);
         prefetch_tmap(&tm_B);
         prefetch_tmap(&tm_C);
+        prefetch_tmap(&tm_y);
     }
     if (warp == 1) tmem_alloc(&bs->tmem, 512);
     tc_fence_before();
@@ -285,35 +314,40 @@ __global__ void __launch_bounds__(kThreads, 1)
                             mma_commit(&bs->g_full[sl]);
                         }
                         const uint32_t pn = n & 1;
-                        if (!wait_bar(&bs->p_full, pn, bs, err)) goto drain;
-                        if (!wait_bar(&bs->x_full[xs], (n / kXStages) & 1, bs, err)) goto drain;
-                        if (!wait_bar(&bs->wx_full, pn, bs, err)) goto drain;
+                        const int ws = n % kWXStages;
+                        // S = B^T (w o x) and R = C h^T do not need P: issue them first
+                        if (!wait_bar(&bs->wx_full[ws], (n / kWXStages) & 1, bs, err)) goto drain;
                         if (!wait_bar(&bs->h_full, pn, bs, err)) goto drain;
-                        if (!wait_bar(&bs->acc_empty, pn ^ 1, bs, err)) goto drain;
+                        if (!wait_bar(&bs->sr_empty, pn ^ 1, bs, err)) goto drain;
                         tc_fence_after();
                         const uint32_t aB = smem_u32(smem + kOffBC + sl * kBCSlot);
                         const uint32_t aC = aB + kBCSlot / 2;
                         const uint32_t aX = smem_u32(smem + kOffX + xs * kAtom);
-                        const uint32_t aWX = smem_u32(smem + kOffWX);
+                        const uint32_t aWX = smem_u32(smem + kOffWX + ws * kAtom);
                         const uint32_t aH = smem_u32(smem + kOffH);
+#pragma unroll
+                        for (int kk = 0; kk < kTile / 16; ++kk) {
+                            mma_bf16(tmem + kColS, sw128_desc(aB + kk * 2048, kAtom, 1024),
+                                     sw128_desc(aWX + kk * 2048, kAtom, 1024), idS, kk > 0);
+                            mma_bf16(tmem + kColR,
+                                     sw128_desc(aC + (kk >> 2) * kAtom + (kk & 3) * 32, 16, 1024),
+                                     sw128_desc(aH + kk * 2048, kAtom, 1024), idY, kk > 0);
+                        }
+                        mma_commit(&bs->wx_empty[ws]);
+                        mma_commit(&bs->h_empty);
+                        mma_commit(&bs->sr_full);
+                        // Y = P x once the mask group has written P
+                        if (!wait_bar(&bs->p_full, pn, bs, err)) goto drain;
+                        if (!wait_bar(&bs->x_full[xs], (n / kXStages) & 1, bs, err)) goto drain;
+                        if (!wait_bar(&bs->y_empty, pn ^ 1, bs, err)) goto drain;
+                        tc_fence_after();
 #pragma unroll
                         for (int kk = 0; kk < kTile / 16; ++kk)
                             mma_bf16_tmem_a(tmem + kColY, tmem + kColP + 8 * kk,
                                             sw128_desc(aX + kk * 2048, kAtom, 1024), idY, kk > 0);
-#pragma unroll
-                        for (int kk = 0; kk < kTile / 16; ++kk)
-                            mma_bf16(tmem + kColS, sw128_desc(aB + kk * 2048, kAtom, 1024),
-                                     sw128_desc(aWX + kk * 2048, kAtom, 1024), idS, kk > 0);
-#pragma unroll
-                        for (int kk = 0; kk < kN / 16; ++kk)
-                            mma_bf16(tmem + kColR,
-                                     sw128_desc(aC + (kk >> 2) * kAtom + (kk & 3) * 32, 16, 1024),
-                                     sw128_desc(aH + kk * 2048, kAtom, 1024), idY, kk > 0);
                         mma_commit(&bs->p_empty);
-                        mma_commit(&bs->wx_empty);
-                        mma_commit(&bs->h_empty);
                         mma_commit(&bs->x_empty[xs]);
-                        mma_commit(&bs->acc_full);
+                        mma_commit(&bs->y_full);
                         if (kh == kh_n - 1) mma_commit(&bs->bc_empty[sl]);
                     }
                 }
@@ -332,6 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kh = 0; kh < kh_n; ++kh) {
                 const int h = U.hb * kh_n + kh;
                 const float a2 = prm.A[h] * kLog2e;
+                const float d_h = prm.D ? prm.D[h] : 0.f;
                 for (int s = 0; s < U.nsub; ++s, ++n) {
                     const int cb = n % kCsStages;
                     if (!wait_bar_all(&bs->cs_empty[cb], ((n / kCsStages) & 1) ^ 1, bs, err)) goto done;
@@ -384,7 +419,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                     reinterpret_cast<float4*>(w)[lane] = w4;
                     reinterpret_cast<float4*>(uu)[lane] = u4;
                     reinterpret_cast<float4*>(vv)[lane] = v4;
+                    if (lane == 0) vv[kTile] = d_h;
+                    __syncwarp();
                     mbar_arrive(&bs->cs_full[cb]);
+                }
+            }
+        }
+    } else if (warp == 3) {
+        if (lane == 0) {
+            // ---------------------------------------------------------- chain publisher
+            // The state group stores a head's state and arrives on pub_full; this lane
+            // then makes those stores visible GPU-wide (one fence, cumulative over the
+            // stores ordered before the barrier) and releases the head's chain flag.
+            int np = 0;
+            for (int u = blockIdx.x; u < prm.nunits; u += gridDim.x) {
+                const Unit U = decode(prm, u);
+                for (int kh = 0; kh < kh_n; ++kh, ++np) {
+                    const int h = U.hb * kh_n + kh;
+                    const int ps = np % kPubStages;
+                    if (!wait_bar(&bs->pub_full[ps], (np / kPubStages) & 1, bs, err)) goto done;
+                    __threadfence();
+                    st_release(prm.flags + (int64_t)U.b * H + h, U.c + 1);
+                    mbar_arrive(&bs->pub_empty[ps]);
                 }
             }
         }
@@ -401,15 +457,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int mm = m + s, sl = mm & 1;
                     const uint32_t pn = n & 1;
                     const int cb = n % kCsStages, xs = n % kXStages;
-                    if (kh == 0 && !wait_bar_all(&bs->g_full[sl], (mm >> 1) & 1, bs, err)) goto done;
                     if (!wait_bar_all(&bs->cs_full[cb], (n / kCsStages) & 1, bs, err)) goto done;
+                    const float* cs = reinterpret_cast<const float*>(smem + kOffCs + cb * kCsSlot);
+                    const float* dts = cs + kTile;
+                    const float* vv = dts + 3 * kTile;
+                    // masked diagonal block P = G o mask into TMEM
+                    if (kh == 0 && !wait_bar_all(&bs->g_full[sl], (mm >> 1) & 1, bs, err)) goto done;
                     if (!wait_bar_all(&bs->p_empty, pn ^ 1, bs, err)) goto done;
                     tc_fence_after();
                     __syncwarp();
-                    const float* cs = reinterpret_cast<const float*>(smem + kOffCs + cb * kCsSlot);
-                    const float* dts = cs + kTile;
-                    const float* wv = dts + kTile;
-                    const float* vv = wv + 2 * kTile;
                     const float csj = cs[j];
 #pragma unroll 1
                     for (int blk = 0; blk < 4; ++blk) {
@@ -459,26 +515,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_before();
                     mbar_arrive(&bs->p_full);
                     if (kh == kh_n - 1) mbar_arrive(&bs->g_empty[sl]);
-                    // w o x, rows scaled by exp(cs_last - cs_i) dt_i
-                    if (!wait_bar_all(&bs->x_full[xs], (n / kXStages) & 1, bs, err)) goto done;
-                    if (!wait_bar_all(&bs->wx_empty, pn ^ 1, bs, err)) goto done;
-                    {
-                        const uint8_t* sx = smem + kOffX + xs * kAtom;
-                        uint8_t* swx = smem + kOffWX;
-                        const float w = wv[j];
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            const uint4 xv = *reinterpret_cast<const uint4*>(sx + sw128_off(j, q));
-                            const float2 a = unpack_bf16(xv.x), b = unpack_bf16(xv.y);
-                            const float2 c2 = unpack_bf16(xv.z), d2 = unpack_bf16(xv.w);
-                            *reinterpret_cast<uint4*>(swx + sw128_off(j, q)) = make_uint4(
-                                pack_bf16(w * a.x, w * a.y), pack_bf16(w * b.x, w * b.y),
-                                pack_bf16(w * c2.x, w * c2.y), pack_bf16(w * d2.x, w * d2.y));
-                        }
-                    }
-                    fence_proxy_async_smem();
-                    mbar_arrive(&bs->wx_full);
-                    mbar_arrive(&bs->x_empty[xs]);
                     mbar_arrive(&bs->cs_empty[cb]);
                 }
             }
@@ -486,138 +522,187 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp >= 8) {
         // ------------------------------------------------------------ state / epilogue group
-        const int wq = warp - 8;
-        const int r = tid - 256;  // row j of the tile for outputs, n of the state
-        const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+        // Per item n: drain S and R as soon as they are done (so the next item's S and R
+        // can follow Y on the tensor pipe), update the state, stage the next operand
+        // (next tile's state, or publish this head and enter the next one), build w o x
+        // for item n+1, then drain Y and finish y_n.
+        const int q = warp & 3;                 // TMEM lane quarter
+        const int ph = (warp - 8) >> 2;         // half of the head dim this warp owns
+        const int r = q * 32 + lane;            // tile row for outputs, state index n
+        const bool leader = (warp == 8 && lane == 0);
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         const int64_t PN = (int64_t)kP * kN;
-        int n = 0, nchain = 0, npub = 0;
+        int nchain = 0, npub = 0;
+        float hreg[32];  // h[32 ph + i][r] of the head being processed
+        // State entering chunk U.c of head h into hreg, and its bf16 copy as the B operand
+        // of the first tile's C h^T (item `item`). Returns false on abort.
+        auto enter_head = [&](const Unit& U, int h, int item) -> bool {
+            if (U.c == 0) {
+                const float* src =
+                    prm.init ? prm.init + ((int64_t)U.b * H + h) * PN + (int64_t)(32 * ph) * kN + r : nullptr;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) hreg[i] = src ? __ldg(src + (int64_t)i * kN) : 0.f;
+            } else {
+                if (leader) {
+                    const int* f = prm.flags + (int64_t)U.b * H + h;
+                    bool ok = false;
+                    const uint64_t t0 = global_ns();
+                    for (uint32_t it = 0;; ++it) {
+                        if (ld_acquire(f) >= U.c) { ok = true; break; }
+                        if ((it & 15) == 15 &&
+                            (*(volatile int*)&bs->abort || global_ns() - t0 > 2000000000ull))
+                            break;
+                    }
+                    if (!ok) {
+                        *(volatile int*)&bs->abort = 1;
+                        atomicExch(err, 1);
+                    }
+                    mbar_arrive(&bs->chain_ok);
+                }
+                if (!wait_bar_all(&bs->chain_ok, nchain & 1, bs, err)) return false;
+                ++nchain;
+                if (*(volatile int*)&bs->abort) return false;
+                __threadfence();
+                const float* src = prm.chain + ((int64_t)U.b * H + h) * PN + (int64_t)(32 * ph) * kN + r;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) hreg[i] = __ldcg(src + (int64_t)i * kN);
+            }
+            if (!wait_bar_all(&bs->h_empty, (item & 1) ^ 1, bs, err)) return false;
+            write_h_half(smem + kOffH, r, ph, hreg);
+            fence_proxy_async_smem();
+            mbar_arrive(&bs->h_full);
+            return true;
+        };
+        // w o x of item `item`: row r of the x tile scaled by w_r = exp(cs_last - cs_r) dt_r,
+        // this warp's half of the head dim. Returns false on abort.
+        auto make_wx = [&](int item) -> bool {
+            const int xs = item % kXStages, ws = item % kWXStages, cb = item % kCsStages;
+            if (!wait_bar_all(&bs->cs_full[cb], (item / kCsStages) & 1, bs, err)) return false;
+            if (!wait_bar_all(&bs->x_full[xs], (item / kXStages) & 1, bs, err)) return false;
+            if (!wait_bar_all(&bs->wx_empty[ws], ((item / kWXStages) & 1) ^ 1, bs, err)) return false;
+            const float w = reinterpret_cast<const float*>(smem + kOffCs + cb * kCsSlot)[2 * kTile + r];
+            const uint8_t* sx = smem + kOffX + xs * kAtom;
+            uint8_t* swx = smem + kOffWX + ws * kAtom;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const uint32_t off = sw128_off(r, 4 * ph + c);
+                const uint4 xv = *reinterpret_cast<const uint4*>(sx + off);
+                const float2 a = unpack_bf16(xv.x), b = unpack_bf16(xv.y);
+                const float2 c2 = unpack_bf16(xv.z), d2 = unpack_bf16(xv.w);
+                *reinterpret_cast<uint4*>(swx + off) =
+                    make_uint4(pack_bf16(w * a.x, w * a.y), pack_bf16(w * b.x, w * b.y),
+                               pack_bf16(w * c2.x, w * c2.y), pack_bf16(w * d2.x, w * d2.y));
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&bs->wx_full[ws]);
+            mbar_arrive(&bs->x_empty[xs]);
+            return true;
+        };
+        if (blockIdx.x < prm.nunits) {
+            const Unit U0 = decode(prm, blockIdx.x);
+            if (!enter_head(U0, U0.hb * kh_n, 0)) goto done;
+            if (!make_wx(0)) goto done;
+        }
+        int n = 0;
         for (int u = blockIdx.x; u < prm.nunits; u += gridDim.x) {
             const Unit U = decode(prm, u);
             for (int kh = 0; kh < kh_n; ++kh) {
                 const int h = U.hb * kh_n + kh;
-                const float D_h = prm.D ? prm.D[h] : 0.f;
-                float hreg[kP];
-                // state entering the chunk
-                if (U.c == 0) {
-                    const float* src = prm.init ? prm.init + ((int64_t)U.b * H + h) * PN + r : nullptr;
-#pragma unroll
-                    for (int p = 0; p < kP; ++p) hreg[p] = src ? __ldg(src + (int64_t)p * kN) : 0.f;
-                } else {
-                    if (r == 0) {
-                        const int* f = prm.flags + (int64_t)U.b * H + h;
-                        bool ok = false;
-                        const uint64_t t0 = global_ns();
-                        for (uint32_t it = 0;; ++it) {
-                            if (ld_acquire(f) >= U.c) { ok = true; break; }
-                            if ((it & 15) == 15 &&
-                                (*(volatile int*)&bs->abort || global_ns() - t0 > 2000000000ull))
-                                break;
-                        }
-                        if (!ok) {
-                            *(volatile int*)&bs->abort = 1;
-                            atomicExch(err, 1);
-                        }
-                        mbar_arrive(&bs->chain_ok);
-                    }
-                    if (!wait_bar_all(&bs->chain_ok, nchain & 1, bs, err)) goto done;
-                    ++nchain;
-                    if (*(volatile int*)&bs->abort) goto done;
-                    __threadfence();
-                    const float* src = prm.chain + ((int64_t)U.b * H + h) * PN + r;
-#pragma unroll
-                    for (int p = 0; p < kP; ++p) hreg[p] = __ldcg(src + (int64_t)p * kN);
-                }
                 for (int s = 0; s < U.nsub; ++s, ++n) {
                     const uint32_t pn = n & 1;
-                    const int cb = n % kCsStages, xs = n % kXStages;
-                    const int64_t t0 = U.tc0 + (int64_t)s * kTile;
-                    const int len = (int)min((int64_t)kTile, T - t0);
-                    // h as the B operand of C h^T (row n holds h[0..63][n]); for the first
-                    // tile of the head here, for later tiles right after the state update
-                    if (s == 0) {
-                        if (!wait_bar_all(&bs->h_empty, pn ^ 1, bs, err)) goto done;
-                        write_h_operand(smem + kOffH, r, hreg);
-                        fence_proxy_async_smem();
-                        mbar_arrive(&bs->h_full);
-                    }
+                    const int cb = n % kCsStages, xs = n % kXStages, ws = n % kWXStages;
+                    const bool has_next = (s + 1 < U.nsub) || (kh + 1 < kh_n) ||
+                                          (u + (int)gridDim.x < prm.nunits);
                     if (!wait_bar_all(&bs->cs_full[cb], (n / kCsStages) & 1, bs, err)) goto done;
-                    if (!wait_bar_all(&bs->x_full[xs], (n / kXStages) & 1, bs, err)) goto done;
-                    if (!wait_bar_all(&bs->acc_full, pn, bs, err)) goto done;
+                    if (!wait_bar_all(&bs->sr_full, pn, bs, err)) goto done;
                     tc_fence_after();
                     __syncwarp();
                     const float* cs = reinterpret_cast<const float*>(smem + kOffCs + cb * kCsSlot);
                     const float* uu = cs + 3 * kTile;
                     const float e = uu[kTile - 1];   // exp(cs_last): decay over the whole tile
-                    // h <- e h + S  (lane n holds S[n][0..63])
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
+                    const float D_h = uu[2 * kTile];
+                    const float uj = uu[r];
+                    // drain S and R (this warp's 32 columns), release them, update the state
+                    float rv[32];
+                    {
                         float sv[32];
-                        tmem_ld32(tmem + lane_base + kColS + 32 * half, sv);
+                        tmem_ld32(tmem + lane_base + kColS + 32 * ph, sv);
+                        tmem_ld32(tmem + lane_base + kColR + 32 * ph, rv);
                         tmem_ld_wait();
+                        tc_fence_before();
+                        mbar_arrive(&bs->sr_empty);
 #pragma unroll
-                        for (int p = 0; p < 32; ++p)
-                            hreg[32 * half + p] = fmaf(e, hreg[32 * half + p], sv[p]);
+                        for (int i = 0; i < 32; ++i) hreg[i] = fmaf(e, hreg[i], sv[i]);
                     }
                     if (s + 1 < U.nsub) {
-                        // the R product of this item has completed (acc_full), so the
-                        // operand buffer is free: stage the state entering the next tile
-                        write_h_operand(smem + kOffH, r, hreg);
+                        // R of this item is complete, so the operand buffer is free:
+                        // stage the state entering the next tile
+                        write_h_half(smem + kOffH, r, ph, hreg);
                         fence_proxy_async_smem();
                         mbar_arrive(&bs->h_full);
                     } else {
-                        // hand the state of head h on to the next chunk before the epilogue
-                        float* dst = prm.chain + ((int64_t)U.b * H + h) * PN + r;
+                        // hand the state of head h on (flag released by warp 3) ...
+                        const int ps = npub % kPubStages;
+                        if (!wait_bar_all(&bs->pub_empty[ps], ((npub / kPubStages) & 1) ^ 1, bs, err))
+                            goto done;
+                        float* dst = prm.chain + ((int64_t)U.b * H + h) * PN + (int64_t)(32 * ph) * kN + r;
 #pragma unroll
-                        for (int p = 0; p < kP; ++p) __stcg(dst + (int64_t)p * kN, hreg[p]);
-                        __threadfence();
-                        mbar_arrive(&bs->pub);
-                        if (r == 0) {
-                            if (wait_bar(&bs->pub, npub & 1, bs, err))
-                                st_release(prm.flags + (int64_t)U.b * H + h, U.c + 1);
-                        }
+                        for (int i = 0; i < 32; ++i) __stcg(dst + (int64_t)i * kN, hreg[i]);
+                        mbar_arrive(&bs->pub_full[ps]);
                         ++npub;
-                        // lane 0 may have waited above: reconverge before warp-collective tcgen05.ld
-                        __syncwarp();
+                        // ... and enter the next head, so the next item's products can start
+                        if (kh + 1 < kh_n) {
+                            if (!enter_head(U, h + 1, n + 1)) goto done;
+                        } else if (u + (int)gridDim.x < prm.nunits) {
+                            const Unit U2 = decode(prm, u + gridDim.x);
+                            if (!enter_head(U2, U2.hb * kh_n, n + 1)) goto done;
+                        }
                     }
-                    // y_j = Y_j + exp(cs_j) R_j + D x_j
-                    const float uj = uu[r];
-                    const uint8_t* sx = smem + kOffX + xs * kAtom;
-                    __nv_bfloat16* yrow = prm.y + (((int64_t)U.b * T + t0 + r) * H + h) * kP;
-                    uint32_t pk[32];
+                    if (has_next && !make_wx(n + 1)) goto done;
+                    // skip-term x of this item, then Y
+                    uint4 xq[4];
+                    {
+                        const uint8_t* sx = smem + kOffX + xs * kAtom;
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        float yv[32], rv[32];
-                        tmem_ld32(tmem + lane_base + kColY + 32 * half, yv);
-                        tmem_ld32(tmem + lane_base + kColR + 32 * half, rv);
-                        tmem_ld_wait();
+                        for (int c = 0; c < 4; ++c)
+                            xq[c] = *reinterpret_cast<const uint4*>(sx + sw128_off(r, 4 * ph + c));
+                    }
+                    if (!wait_bar_all(&bs->y_full, pn, bs, err)) goto done;
+                    tc_fence_after();
+                    __syncwarp();
+                    float yv[32];
+                    tmem_ld32(tmem + lane_base + kColY + 32 * ph, yv);
+                    tmem_ld_wait();
+                    tc_fence_before();
+                    mbar_arrive(&bs->y_empty);
+                    // generic-proxy reads of the x slot are done before the next TMA load into it
+                    fence_proxy_async_smem();
+                    mbar_arrive(&bs->x_empty[xs]);
+                    // y_j = Y_j + exp(cs_j) R_j + D x_j: this thread's 64 contiguous bytes of row r
+                    {
+                        const int64_t t0 = U.tc0 + (int64_t)s * kTile;
+                        uint4 out[4];
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const uint4 xv =
-                                *reinterpret_cast<const uint4*>(sx + sw128_off(r, 4 * half + q));
-                            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                        for (int c = 0; c < 4; ++c) {
+                            const uint32_t xw[4] = {xq[c].x, xq[c].y, xq[c].z, xq[c].w};
+                            uint32_t o[4];
 #pragma unroll
                             for (int e2 = 0; e2 < 4; ++e2) {
                                 const float2 xf = unpack_bf16(xw[e2]);
-                                const int c0 = 8 * q + 2 * e2;
-                                pk[16 * half + 4 * q + e2] =
-                                    pack_bf16(fmaf(uj, rv[c0], yv[c0]) + D_h * xf.x,
-                                              fmaf(uj, rv[c0 + 1], yv[c0 + 1]) + D_h * xf.y);
+                                const int i0 = 8 * c + 2 * e2;
+                                o[e2] = pack_bf16(fmaf(uj, rv[i0], yv[i0]) + D_h * xf.x,
+                                                  fmaf(uj, rv[i0 + 1], yv[i0 + 1]) + D_h * xf.y);
                             }
+                            out[c] = make_uint4(o[0], o[1], o[2], o[3]);
+                        }
+                        if (t0 + r < T) {
+                            uint4* dst = reinterpret_cast<uint4*>(
+                                prm.y + (((int64_t)U.b * T + t0 + r) * H + h) * kP + 32 * ph);
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) dst[c] = out[c];
                         }
                     }
-                    tc_fence_before();
-                    mbar_arrive(&bs->acc_empty);
-                    // the x tile was read through the generic proxy; the next TMA load into
-                    // this slot is an async-proxy write, so order the reads before it
-                    fence_proxy_async_smem();
-                    mbar_arrive(&bs->x_empty[xs]);
                     mbar_arrive(&bs->cs_empty[cb]);
-                    if (r < len) {
-                        uint4* dst = reinterpret_cast<uint4*>(yrow);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-                    }
                 }
             }
         }
@@ -665,7 +750,7 @@ cudaError_t launch_fused_ws(const Dims& d, const CUtensorMap* maps, const void* 
                              (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     const int grid = prm.nunits < g_num_sms ? prm.nunits : g_num_sms;
-    ssd_fused_ws_kernel<<<grid, kThreads, kSmemBytes, st>>>(maps[0], maps[1], maps[2], prm);
+    ssd_fused_ws_kernel<<<grid, kThreads, kSmemBytes, st>>>(maps[0], maps[1], maps[2], maps[3], prm);
     return cudaGetLastError();
 }
 

@@ -493,9 +493,11 @@ int pick_kheads(int64_t heads_per_group) {
     return 1;
 }
 
-bool make_tc_maps(const Dims& d, const void* x, const void* B, const void* C, CUtensorMap* maps) {
+bool make_tc_maps(const Dims& d, const void* x, const void* B, const void* C, const void* y,
+                  CUtensorMap* maps) {
     return make_map(&maps[0], x, d.P, d.H, d.T, d.b) && make_map(&maps[1], B, d.N, d.G, d.T, d.b) &&
-           make_map(&maps[2], C ? C : B, d.N, d.G, d.T, d.b);
+           make_map(&maps[2], C ? C : B, d.N, d.G, d.T, d.b) &&
+           make_map(&maps[3], y ? y : x, d.P, d.H, d.T, d.b);
 }
 
 namespace {
@@ -563,8 +565,8 @@ cudaError_t launch_fused_tc(const Dims& d, const void* x, const float* dt, const
     const char* v = getenv("SSD_FUSED");
     if (!(v && strcmp(v, "v0") == 0)) {
         // default: the warp-specialized persistent kernel (ssd_fused.cu)
-        CUtensorMap maps[3];
-        if (!make_tc_maps(d, x, B, C, maps)) return cudaErrorInvalidValue;
+        CUtensorMap maps[4];
+        if (!make_tc_maps(d, x, B, C, y, maps)) return cudaErrorInvalidValue;
         return launch_fused_ws(d, maps, x, dt, A, D, init, y, chain, sync_ints,
                                pick_kheads(d.H / d.G), st);
     }
