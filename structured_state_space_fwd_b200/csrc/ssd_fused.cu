@@ -89,8 +89,8 @@ struct Bars {
     uint64_t cs_full[kCsStages], cs_empty[kCsStages];
     uint64_t wx_full[kWXStages], wx_empty[kWXStages];
     uint64_t p_full, p_empty, h_full, h_empty, fin;
-    uint64_t sr_full, sr_empty;   // S and R accumulators (state product, C h^T)
-    uint64_t y_full, y_empty;     // Y accumulator (P x)
+    uint64_t sr_full, s_empty;    // S and R done; S drained by the state group
+    uint64_t y_full, ry_empty;    // Y done; R and Y drained by the state group
     uint64_t chain_ok;                          // chain flag observed (state group)
     uint64_t pub_full[kPubStages], pub_empty[kPubStages];  // state stored / flag released
     uint32_t tmem;
@@ -220,9 +220,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&bs->h_full, 256);
         mbar_init(&bs->h_empty, 1);
         mbar_init(&bs->sr_full, 1);
-        mbar_init(&bs->sr_empty, 256);
+        mbar_init(&bs->s_empty, 256);
         mbar_init(&bs->y_full, 1);
-        mbar_init(&bs->y_empty, 256);
+        mbar_init(&bs->ry_empty, 256);
         mbar_init(&bs->fin, 1);
         mbar_init(&bs->chain_ok, 1);
         for (int i = 0; i < kPubStages; ++i) {
@@ -304,47 +304,48 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if (!wait_bar(&bs->g_empty[sl], ph ^ 1, bs, err)) goto drain;
                             tc_fence_after();
                             const uint32_t gB = smem_u32(smem + kOffBC + sl * kBCSlot);
-                            const uint32_t gC = gB + kBCSlot / 2;
+                            const uint64_t dGA = sw128_desc(gB + kBCSlot / 2, 16, 1024);
+                            const uint64_t dGB = sw128_desc(gB, 16, 1024);
 #pragma unroll
                             for (int kk = 0; kk < kN / 16; ++kk) {
-                                const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
-                                mma_bf16(tmem + kColG + 128 * sl, sw128_desc(gC + off, 16, 1024),
-                                         sw128_desc(gB + off, 16, 1024), idG, kk > 0);
+                                // start address advances by (kk/4) atoms + (kk%4) x 32 bytes
+                                const uint64_t off = (uint64_t)(((kk >> 2) * kAtom + (kk & 3) * 32) >> 4);
+                                mma_bf16(tmem + kColG + 128 * sl, dGA + off, dGB + off, idG, kk > 0);
                             }
                             mma_commit(&bs->g_full[sl]);
                         }
                         const uint32_t pn = n & 1;
                         const int ws = n % kWXStages;
-                        // S = B^T (w o x) and R = C h^T do not need P: issue them first
+                        // S = B^T (w o x) and R = C h^T first: the state update waits on them
                         if (!wait_bar(&bs->wx_full[ws], (n / kWXStages) & 1, bs, err)) goto drain;
                         if (!wait_bar(&bs->h_full, pn, bs, err)) goto drain;
-                        if (!wait_bar(&bs->sr_empty, pn ^ 1, bs, err)) goto drain;
+                        if (!wait_bar(&bs->s_empty, pn ^ 1, bs, err)) goto drain;
+                        if (!wait_bar(&bs->ry_empty, pn ^ 1, bs, err)) goto drain;
                         tc_fence_after();
                         const uint32_t aB = smem_u32(smem + kOffBC + sl * kBCSlot);
-                        const uint32_t aC = aB + kBCSlot / 2;
-                        const uint32_t aX = smem_u32(smem + kOffX + xs * kAtom);
-                        const uint32_t aWX = smem_u32(smem + kOffWX + ws * kAtom);
-                        const uint32_t aH = smem_u32(smem + kOffH);
+                        const uint64_t dSA = sw128_desc(aB, kAtom, 1024);
+                        const uint64_t dSB = sw128_desc(smem_u32(smem + kOffWX + ws * kAtom), kAtom, 1024);
+                        const uint64_t dRA = sw128_desc(aB + kBCSlot / 2, 16, 1024);
+                        const uint64_t dRB = sw128_desc(smem_u32(smem + kOffH), kAtom, 1024);
 #pragma unroll
                         for (int kk = 0; kk < kTile / 16; ++kk) {
-                            mma_bf16(tmem + kColS, sw128_desc(aB + kk * 2048, kAtom, 1024),
-                                     sw128_desc(aWX + kk * 2048, kAtom, 1024), idS, kk > 0);
-                            mma_bf16(tmem + kColR,
-                                     sw128_desc(aC + (kk >> 2) * kAtom + (kk & 3) * 32, 16, 1024),
-                                     sw128_desc(aH + kk * 2048, kAtom, 1024), idY, kk > 0);
+                            const uint64_t rows = (uint64_t)(kk * (2048 >> 4));   // 16 rows of 128 B
+                            const uint64_t kofs = (uint64_t)(((kk >> 2) * kAtom + (kk & 3) * 32) >> 4);
+                            mma_bf16(tmem + kColS, dSA + rows, dSB + rows, idS, kk > 0);
+                            mma_bf16(tmem + kColR, dRA + kofs, dRB + rows, idY, kk > 0);
                         }
                         mma_commit(&bs->wx_empty[ws]);
                         mma_commit(&bs->h_empty);
                         mma_commit(&bs->sr_full);
-                        // Y = P x once the mask group has written P
+                        // Y = P x (P straight from TMEM)
                         if (!wait_bar(&bs->p_full, pn, bs, err)) goto drain;
                         if (!wait_bar(&bs->x_full[xs], (n / kXStages) & 1, bs, err)) goto drain;
-                        if (!wait_bar(&bs->y_empty, pn ^ 1, bs, err)) goto drain;
                         tc_fence_after();
+                        const uint64_t dXB = sw128_desc(smem_u32(smem + kOffX + xs * kAtom), kAtom, 1024);
 #pragma unroll
                         for (int kk = 0; kk < kTile / 16; ++kk)
                             mma_bf16_tmem_a(tmem + kColY, tmem + kColP + 8 * kk,
-                                            sw128_desc(aX + kk * 2048, kAtom, 1024), idY, kk > 0);
+                                            dXB + (uint64_t)(kk * (2048 >> 4)), idY, kk > 0);
                         mma_commit(&bs->p_empty);
                         mma_commit(&bs->x_empty[xs]);
                         mma_commit(&bs->y_full);
@@ -622,15 +623,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float e = uu[kTile - 1];   // exp(cs_last): decay over the whole tile
                     const float D_h = uu[2 * kTile];
                     const float uj = uu[r];
-                    // drain S and R (this warp's 32 columns), release them, update the state
-                    float rv[32];
+                    // drain S (this warp's 32 columns), release it, update the state
                     {
                         float sv[32];
                         tmem_ld32(tmem + lane_base + kColS + 32 * ph, sv);
-                        tmem_ld32(tmem + lane_base + kColR + 32 * ph, rv);
                         tmem_ld_wait();
                         tc_fence_before();
-                        mbar_arrive(&bs->sr_empty);
+                        mbar_arrive(&bs->s_empty);
 #pragma unroll
                         for (int i = 0; i < 32; ++i) hreg[i] = fmaf(e, hreg[i], sv[i]);
                     }
@@ -659,47 +658,53 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                     if (has_next && !make_wx(n + 1)) goto done;
-                    // skip-term x of this item, then Y
-                    uint4 xq[4];
-                    {
-                        const uint8_t* sx = smem + kOffX + xs * kAtom;
-#pragma unroll
-                        for (int c = 0; c < 4; ++c)
-                            xq[c] = *reinterpret_cast<const uint4*>(sx + sw128_off(r, 4 * ph + c));
-                    }
+                    // R and Y (this warp's 32 columns) in two halves of 16:
+                    // y_j = Y_j + exp(cs_j) R_j + D x_j, this thread's bytes of row r
                     if (!wait_bar_all(&bs->y_full, pn, bs, err)) goto done;
                     tc_fence_after();
                     __syncwarp();
-                    float yv[32];
-                    tmem_ld32(tmem + lane_base + kColY + 32 * ph, yv);
-                    tmem_ld_wait();
-                    tc_fence_before();
-                    mbar_arrive(&bs->y_empty);
-                    // generic-proxy reads of the x slot are done before the next TMA load into it
-                    fence_proxy_async_smem();
-                    mbar_arrive(&bs->x_empty[xs]);
-                    // y_j = Y_j + exp(cs_j) R_j + D x_j: this thread's 64 contiguous bytes of row r
                     {
                         const int64_t t0 = U.tc0 + (int64_t)s * kTile;
-                        uint4 out[4];
+                        const uint8_t* sx = smem + kOffX + xs * kAtom;
+                        uint4* dst = reinterpret_cast<uint4*>(
+                            prm.y + (((int64_t)U.b * T + t0 + r) * H + h) * kP + 32 * ph);
+                        const bool valid = t0 + r < T;
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            const uint32_t xw[4] = {xq[c].x, xq[c].y, xq[c].z, xq[c].w};
-                            uint32_t o[4];
+                        for (int hf = 0; hf < 2; ++hf) {
+                            float yv[16], rv[16];
+                            tmem_ld16(tmem + lane_base + kColY + 32 * ph + 16 * hf, yv);
+                            tmem_ld16(tmem + lane_base + kColR + 32 * ph + 16 * hf, rv);
+                            uint4 xq[2];
 #pragma unroll
-                            for (int e2 = 0; e2 < 4; ++e2) {
-                                const float2 xf = unpack_bf16(xw[e2]);
-                                const int i0 = 8 * c + 2 * e2;
-                                o[e2] = pack_bf16(fmaf(uj, rv[i0], yv[i0]) + D_h * xf.x,
-                                                  fmaf(uj, rv[i0 + 1], yv[i0 + 1]) + D_h * xf.y);
+                            for (int c = 0; c < 2; ++c)
+                                xq[c] = *reinterpret_cast<const uint4*>(sx + sw128_off(r, 4 * ph + 2 * hf + c));
+                            tmem_ld_wait();
+                            if (hf == 1) {
+                                tc_fence_before();
+                                mbar_arrive(&bs->ry_empty);
+                                // generic-proxy reads of the x slot are done before the next
+                                // TMA load into it
+                                fence_proxy_async_smem();
+                                mbar_arrive(&bs->x_empty[xs]);
                             }
-                            out[c] = make_uint4(o[0], o[1], o[2], o[3]);
-                        }
-                        if (t0 + r < T) {
-                            uint4* dst = reinterpret_cast<uint4*>(
-                                prm.y + (((int64_t)U.b * T + t0 + r) * H + h) * kP + 32 * ph);
+                            uint4 out[2];
 #pragma unroll
-                            for (int c = 0; c < 4; ++c) dst[c] = out[c];
+                            for (int c = 0; c < 2; ++c) {
+                                const uint32_t xw[4] = {xq[c].x, xq[c].y, xq[c].z, xq[c].w};
+                                uint32_t o[4];
+#pragma unroll
+                                for (int e2 = 0; e2 < 4; ++e2) {
+                                    const float2 xf = unpack_bf16(xw[e2]);
+                                    const int i0 = 8 * c + 2 * e2;
+                                    o[e2] = pack_bf16(fmaf(uj, rv[i0], yv[i0]) + D_h * xf.x,
+                                                      fmaf(uj, rv[i0 + 1], yv[i0 + 1]) + D_h * xf.y);
+                                }
+                                out[c] = make_uint4(o[0], o[1], o[2], o[3]);
+                            }
+                            if (valid) {
+                                dst[2 * hf] = out[0];
+                                dst[2 * hf + 1] = out[1];
+                            }
                         }
                     }
                     mbar_arrive(&bs->cs_empty[cb]);
