@@ -68,6 +68,10 @@ constexpr uint32_t kColR = 384;
 constexpr uint32_t kColS = 448;
 
 constexpr float kLog2e = 1.4426950408889634f;
+// Widest cs range (log2 units) of a 32-row diagonal block for which the masked
+// product is formed as exp2(cs_j - cs_e) * exp2(cs_e - cs_i): both factors then
+// stay within 2^+-64, far from fp32 overflow for any finite G.
+constexpr float kFactorRangeLog2 = 64.f;
 
 struct Params {
     const __nv_bfloat16* x;
@@ -113,6 +117,10 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
     __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&u);
     return __bfloat1622float2(h);
 }
+__device__ __forceinline__ uint32_t pack_bf16(float2 v) { return pack_bf16(v.x, v.y); }
+// packed fp32 pairs (one instruction for two lanes of arithmetic)
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
 __device__ __forceinline__ uint64_t global_ns() {
     uint64_t t;
@@ -120,14 +128,27 @@ __device__ __forceinline__ uint64_t global_ns() {
     return t;
 }
 
-// Bounded mbarrier wait (about 2 s) that also gives up as soon as another role
-// aborted. try_wait itself suspends the thread for a while, so no sleep is added.
+// A suspend-time hint on try_wait measured slower here (the woken thread
+// resumes later than a spinning one notices), so waits spin by default.
+#ifndef SSD_WAIT_HINT_NS
+#define SSD_WAIT_HINT_NS 0u
+#endif
+__device__ __forceinline__ bool try_wait(uint64_t* bar, uint32_t parity) {
+#if SSD_WAIT_HINT_NS > 0
+    return mbar_try_wait_hint(bar, parity, SSD_WAIT_HINT_NS);
+#else
+    return mbar_try_wait(bar, parity);
+#endif
+}
+
+// Bounded mbarrier wait (about 2 s) that also gives up once another role
+// aborted (checked every 16 polls).
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Bars* bs, int* err) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63) == 0) {
+        if (try_wait(bar, parity)) return true;
+        if ((i & 15) == 0) {
             if (*(volatile int*)&bs->abort) return false;
             if (global_ns() - t0 > 2000000000ull) {
                 *(volatile int*)&bs->abort = 1;
@@ -154,18 +175,6 @@ __device__ __forceinline__ void write_h_half(uint8_t* sh, int n, int half, const
         *reinterpret_cast<uint4*>(sh + sw128_off(n, 4 * half + c)) =
             make_uint4(pack_bf16(hh[8 * c], hh[8 * c + 1]), pack_bf16(hh[8 * c + 2], hh[8 * c + 3]),
                        pack_bf16(hh[8 * c + 4], hh[8 * c + 5]), pack_bf16(hh[8 * c + 6], hh[8 * c + 7]));
-}
-
-// bf16 copy of the state as the B operand of C h^T: row n (one thread) holds
-// h[0..63][n], 128-byte swizzled rows.
-__device__ __forceinline__ void write_h_operand(uint8_t* sh, int n, const float (&hreg)[kP]) {
-#pragma unroll
-    for (int q = 0; q < 8; ++q)
-        *reinterpret_cast<uint4*>(sh + sw128_off(n, q)) =
-            make_uint4(pack_bf16(hreg[8 * q], hreg[8 * q + 1]),
-                       pack_bf16(hreg[8 * q + 2], hreg[8 * q + 3]),
-                       pack_bf16(hreg[8 * q + 4], hreg[8 * q + 5]),
-                       pack_bf16(hreg[8 * q + 6], hreg[8 * q + 7]));
 }
 
 struct Unit {
@@ -457,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int s = 0; s < U.nsub; ++s, ++n) {
                     const int mm = m + s, sl = mm & 1;
                     const uint32_t pn = n & 1;
-                    const int cb = n % kCsStages, xs = n % kXStages;
+                    const int cb = n % kCsStages;
                     if (!wait_bar_all(&bs->cs_full[cb], (n / kCsStages) & 1, bs, err)) goto done;
                     const float* cs = reinterpret_cast<const float*>(smem + kOffCs + cb * kCsSlot);
                     const float* dts = cs + kTile;
@@ -468,46 +477,68 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
                     __syncwarp();
                     const float csj = cs[j];
+                    const int jj = j & 31;   // row within this warp's diagonal block
 #pragma unroll 1
                     for (int blk = 0; blk < 4; ++blk) {
                         uint32_t pk[16];
                         if (blk > wq) {
 #pragma unroll
                             for (int q = 0; q < 16; ++q) pk[q] = 0u;
-                        } else if (blk < wq) {
-                            // strictly below the diagonal block: every i < every j, and
-                            // exp(cs_j - cs_i) = exp(cs_j - cs_ref) exp(cs_ref - cs_i) with
-                            // ref the last row of column block blk; both factors are <= 1
-                            float gv[32];
-                            tmem_ld32(tmem + lane_base + kColG + 128 * sl + 32 * blk, gv);
-                            const float uj = exp2f(csj - cs[32 * blk + 31]);
-                            tmem_ld_wait();
-#pragma unroll
-                            for (int e4 = 0; e4 < 8; ++e4) {
-                                const float4 v4 = reinterpret_cast<const float4*>(vv)[blk * 8 + e4];
-                                pk[e4 * 2] = pack_bf16(gv[e4 * 4] * uj * v4.x, gv[e4 * 4 + 1] * uj * v4.y);
-                                pk[e4 * 2 + 1] =
-                                    pack_bf16(gv[e4 * 4 + 2] * uj * v4.z, gv[e4 * 4 + 3] * uj * v4.w);
-                            }
                         } else {
                             float gv[32];
                             tmem_ld32(tmem + lane_base + kColG + 128 * sl + 32 * blk, gv);
+                            // exp(cs_j - cs_i) dt_i = exp(cs_j - cs_e) * v_i with e the last row of
+                            // column block blk and v_i = exp(cs_e - cs_i) dt_i (<= dt_i). Below the
+                            // diagonal block the first factor is <= 1 too; on it, it is >= 1 and
+                            // bounded by the block's own cs range, which decides whether the
+                            // factored form is safe in fp32 or the exponent is taken per element.
+                            const float ce = cs[32 * blk + 31];
+                            const float a = exp2f(csj - ce);
+                            const bool exact = blk == wq && cs[32 * blk] - ce > kFactorRangeLog2;
+                            const float2 a2 = make_float2(a, a);
                             tmem_ld_wait();
+                            if (blk < wq) {
 #pragma unroll
-                            for (int e4 = 0; e4 < 8; ++e4) {
-                                const float4 c4 = reinterpret_cast<const float4*>(cs)[blk * 8 + e4];
-                                const float4 d4 = reinterpret_cast<const float4*>(dts)[blk * 8 + e4];
-                                const int i0 = blk * 32 + e4 * 4;
-                                const float m0 = exp2f(csj - c4.x) * d4.x;
-                                const float m1 = exp2f(csj - c4.y) * d4.y;
-                                const float m2 = exp2f(csj - c4.z) * d4.z;
-                                const float m3 = exp2f(csj - c4.w) * d4.w;
-                                const float p0 = (i0 <= j) ? gv[e4 * 4] * m0 : 0.f;
-                                const float p1 = (i0 + 1 <= j) ? gv[e4 * 4 + 1] * m1 : 0.f;
-                                const float p2 = (i0 + 2 <= j) ? gv[e4 * 4 + 2] * m2 : 0.f;
-                                const float p3 = (i0 + 3 <= j) ? gv[e4 * 4 + 3] * m3 : 0.f;
-                                pk[e4 * 2] = pack_bf16(p0, p1);
-                                pk[e4 * 2 + 1] = pack_bf16(p2, p3);
+                                for (int e4 = 0; e4 < 8; ++e4) {
+                                    const float4 v4 = reinterpret_cast<const float4*>(vv)[blk * 8 + e4];
+                                    pk[e4 * 2] = pack_bf16(mul2(make_float2(gv[e4 * 4], gv[e4 * 4 + 1]),
+                                                                mul2(make_float2(v4.x, v4.y), a2)));
+                                    pk[e4 * 2 + 1] = pack_bf16(mul2(make_float2(gv[e4 * 4 + 2], gv[e4 * 4 + 3]),
+                                                                    mul2(make_float2(v4.z, v4.w), a2)));
+                                }
+                            } else if (!exact) {
+#pragma unroll
+                                for (int e4 = 0; e4 < 8; ++e4) {
+                                    const float4 v4 = reinterpret_cast<const float4*>(vv)[blk * 8 + e4];
+                                    float2 p01 = mul2(make_float2(gv[e4 * 4], gv[e4 * 4 + 1]),
+                                                      mul2(make_float2(v4.x, v4.y), a2));
+                                    float2 p23 = mul2(make_float2(gv[e4 * 4 + 2], gv[e4 * 4 + 3]),
+                                                      mul2(make_float2(v4.z, v4.w), a2));
+                                    const int i0 = e4 * 4;   // causal mask: column i kept while i <= row
+                                    p01.x = i0 <= jj ? p01.x : 0.f;
+                                    p01.y = i0 + 1 <= jj ? p01.y : 0.f;
+                                    p23.x = i0 + 2 <= jj ? p23.x : 0.f;
+                                    p23.y = i0 + 3 <= jj ? p23.y : 0.f;
+                                    pk[e4 * 2] = pack_bf16(p01);
+                                    pk[e4 * 2 + 1] = pack_bf16(p23);
+                                }
+                            } else {
+#pragma unroll
+                                for (int e4 = 0; e4 < 8; ++e4) {
+                                    const float4 c4 = reinterpret_cast<const float4*>(cs)[blk * 8 + e4];
+                                    const float4 d4 = reinterpret_cast<const float4*>(dts)[blk * 8 + e4];
+                                    const int i0 = blk * 32 + e4 * 4;
+                                    const float m0 = exp2f(csj - c4.x) * d4.x;
+                                    const float m1 = exp2f(csj - c4.y) * d4.y;
+                                    const float m2 = exp2f(csj - c4.z) * d4.z;
+                                    const float m3 = exp2f(csj - c4.w) * d4.w;
+                                    const float p0 = (i0 <= j) ? gv[e4 * 4] * m0 : 0.f;
+                                    const float p1 = (i0 + 1 <= j) ? gv[e4 * 4 + 1] * m1 : 0.f;
+                                    const float p2 = (i0 + 2 <= j) ? gv[e4 * 4 + 2] * m2 : 0.f;
+                                    const float p3 = (i0 + 3 <= j) ? gv[e4 * 4 + 3] * m3 : 0.f;
+                                    pk[e4 * 2] = pack_bf16(p0, p1);
+                                    pk[e4 * 2 + 1] = pack_bf16(p2, p3);
+                                }
                             }
                         }
                         tmem_st16(tmem + lane_base + kColP + 16 * blk, pk);
@@ -523,10 +554,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp >= 8) {
         // ------------------------------------------------------------ state / epilogue group
-        // Per item n: drain S and R as soon as they are done (so the next item's S and R
-        // can follow Y on the tensor pipe), update the state, stage the next operand
-        // (next tile's state, or publish this head and enter the next one), build w o x
-        // for item n+1, then drain Y and finish y_n.
+        // Iteration n finishes item n and prepares item n+1: drain S_n as soon as it is
+        // done (so the next S and R can follow Y on the tensor pipe), update the state,
+        // stage the next state operand (next tile of this head, or publish this head and
+        // enter the next one), build w o x of item n+1, then drain Y_n and R_n into y_n.
         const int q = warp & 3;                 // TMEM lane quarter
         const int ph = (warp - 8) >> 2;         // half of the head dim this warp owns
         const int r = q * 32 + lane;            // tile row for outputs, state index n
@@ -550,6 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t t0 = global_ns();
                     for (uint32_t it = 0;; ++it) {
                         if (ld_acquire(f) >= U.c) { ok = true; break; }
+                        if (it >= 8) __nanosleep(32);
                         if ((it & 15) == 15 &&
                             (*(volatile int*)&bs->abort || global_ns() - t0 > 2000000000ull))
                             break;
@@ -574,140 +606,155 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&bs->h_full);
             return true;
         };
-        // w o x of item `item`: row r of the x tile scaled by w_r = exp(cs_last - cs_r) dt_r,
-        // this warp's half of the head dim. Returns false on abort.
-        auto make_wx = [&](int item) -> bool {
-            const int xs = item % kXStages, ws = item % kWXStages, cb = item % kCsStages;
-            if (!wait_bar_all(&bs->cs_full[cb], (item / kCsStages) & 1, bs, err)) return false;
-            if (!wait_bar_all(&bs->x_full[xs], (item / kXStages) & 1, bs, err)) return false;
-            if (!wait_bar_all(&bs->wx_empty[ws], ((item / kWXStages) & 1) ^ 1, bs, err)) return false;
-            const float w = reinterpret_cast<const float*>(smem + kOffCs + cb * kCsSlot)[2 * kTile + r];
-            const uint8_t* sx = smem + kOffX + xs * kAtom;
-            uint8_t* swx = smem + kOffWX + ws * kAtom;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const uint32_t off = sw128_off(r, 4 * ph + c);
-                const uint4 xv = *reinterpret_cast<const uint4*>(sx + off);
-                const float2 a = unpack_bf16(xv.x), b = unpack_bf16(xv.y);
-                const float2 c2 = unpack_bf16(xv.z), d2 = unpack_bf16(xv.w);
-                *reinterpret_cast<uint4*>(swx + off) =
-                    make_uint4(pack_bf16(w * a.x, w * a.y), pack_bf16(w * b.x, w * b.y),
-                               pack_bf16(w * c2.x, w * c2.y), pack_bf16(w * d2.x, w * d2.y));
-            }
-            fence_proxy_async_smem();
-            mbar_arrive(&bs->wx_full[ws]);
-            mbar_arrive(&bs->x_empty[xs]);
-            return true;
-        };
-        if (blockIdx.x < prm.nunits) {
-            const Unit U0 = decode(prm, blockIdx.x);
-            if (!enter_head(U0, U0.hb * kh_n, 0)) goto done;
-            if (!make_wx(0)) goto done;
-        }
-        int n = 0;
-        for (int u = blockIdx.x; u < prm.nunits; u += gridDim.x) {
-            const Unit U = decode(prm, u);
-            for (int kh = 0; kh < kh_n; ++kh) {
-                const int h = U.hb * kh_n + kh;
-                for (int s = 0; s < U.nsub; ++s, ++n) {
-                    const uint32_t pn = n & 1;
-                    const int cb = n % kCsStages, xs = n % kXStages, ws = n % kWXStages;
-                    const bool has_next = (s + 1 < U.nsub) || (kh + 1 < kh_n) ||
-                                          (u + (int)gridDim.x < prm.nunits);
-                    if (!wait_bar_all(&bs->cs_full[cb], (n / kCsStages) & 1, bs, err)) goto done;
-                    if (!wait_bar_all(&bs->sr_full, pn, bs, err)) goto done;
-                    tc_fence_after();
-                    __syncwarp();
-                    const float* cs = reinterpret_cast<const float*>(smem + kOffCs + cb * kCsSlot);
-                    const float* uu = cs + 3 * kTile;
+        // items in the order every role walks them: nx is the next one (unit, head,
+        // tile), cur the one being finished (batch row, head, first token, last tile
+        // of its chunk or not)
+        int nx_u = blockIdx.x, nx_kh = 0, nx_s = 0;
+        bool nx_ok = nx_u < prm.nunits;
+        Unit nxU{};
+        if (nx_ok) nxU = decode(prm, nx_u);
+        bool cur_ok = false, cur_last = false;
+        int cur_b = 0, cur_h = 0;
+        int64_t cur_t0 = 0;
+        for (int n = -1; cur_ok || nx_ok; ++n) {
+            const int nn = n < 0 ? 0 : n;
+            const uint32_t pn = nn & 1;
+            const int cb = nn % kCsStages, xs = nn % kXStages;
+            const float* cs = reinterpret_cast<const float*>(smem + kOffCs + cb * kCsSlot);
+            const float* uu = cs + 3 * kTile;
+            if (cur_ok) {
+                if (!wait_bar_all(&bs->cs_full[cb], (nn / kCsStages) & 1, bs, err)) goto done;
+                if (!wait_bar_all(&bs->sr_full, pn, bs, err)) goto done;
+                tc_fence_after();
+                __syncwarp();
+                // drain S (this warp's 32 columns), release it, update the state
+                {
                     const float e = uu[kTile - 1];   // exp(cs_last): decay over the whole tile
-                    const float D_h = uu[2 * kTile];
-                    const float uj = uu[r];
-                    // drain S (this warp's 32 columns), release it, update the state
-                    {
-                        float sv[32];
-                        tmem_ld32(tmem + lane_base + kColS + 32 * ph, sv);
-                        tmem_ld_wait();
+                    const float2 e2 = make_float2(e, e);
+                    float sv[32];
+                    tmem_ld32(tmem + lane_base + kColS + 32 * ph, sv);
+                    tmem_ld_wait();
+                    tc_fence_before();
+                    mbar_arrive(&bs->s_empty);
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        const float2 t = fma2(e2, make_float2(hreg[i], hreg[i + 1]),
+                                              make_float2(sv[i], sv[i + 1]));
+                        hreg[i] = t.x;
+                        hreg[i + 1] = t.y;
+                    }
+                }
+                if (!cur_last) {
+                    // R of this item is complete, so the operand buffer is free:
+                    // stage the state entering the next tile
+                    write_h_half(smem + kOffH, r, ph, hreg);
+                    fence_proxy_async_smem();
+                    mbar_arrive(&bs->h_full);
+                } else {
+                    // hand the state of head h on (flag released by warp 3)
+                    const int ps = npub % kPubStages;
+                    if (!wait_bar_all(&bs->pub_empty[ps], ((npub / kPubStages) & 1) ^ 1, bs, err))
+                        goto done;
+                    float* dst = prm.chain + ((int64_t)cur_b * H + cur_h) * PN + (int64_t)(32 * ph) * kN + r;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) __stcg(dst + (int64_t)i * kN, hreg[i]);
+                    mbar_arrive(&bs->pub_full[ps]);
+                    ++npub;
+                }
+            }
+            if (nx_ok) {
+                const int item = n + 1;
+                // a new head: its entering state, so the next item's products can start
+                if (nx_s == 0 && !enter_head(nxU, nxU.hb * kh_n + nx_kh, item)) goto done;
+                // w o x of the next item: row r of its x tile scaled by
+                // w_r = exp(cs_last - cs_r) dt_r, this warp's half of the head dim
+                const int xs1 = item % kXStages, ws1 = item % kWXStages, cb1 = item % kCsStages;
+                if (!wait_bar_all(&bs->cs_full[cb1], (item / kCsStages) & 1, bs, err)) goto done;
+                if (!wait_bar_all(&bs->x_full[xs1], (item / kXStages) & 1, bs, err)) goto done;
+                if (!wait_bar_all(&bs->wx_empty[ws1], ((item / kWXStages) & 1) ^ 1, bs, err)) goto done;
+                const float w = reinterpret_cast<const float*>(smem + kOffCs + cb1 * kCsSlot)[2 * kTile + r];
+                const float2 w2 = make_float2(w, w);
+                const uint8_t* sx = smem + kOffX + xs1 * kAtom;
+                uint8_t* swx = smem + kOffWX + ws1 * kAtom;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint32_t off = sw128_off(r, 4 * ph + c);
+                    const uint4 xv = *reinterpret_cast<const uint4*>(sx + off);
+                    *reinterpret_cast<uint4*>(swx + off) =
+                        make_uint4(pack_bf16(mul2(w2, unpack_bf16(xv.x))), pack_bf16(mul2(w2, unpack_bf16(xv.y))),
+                                   pack_bf16(mul2(w2, unpack_bf16(xv.z))), pack_bf16(mul2(w2, unpack_bf16(xv.w))));
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(&bs->wx_full[ws1]);
+                mbar_arrive(&bs->x_empty[xs1]);
+            }
+            if (cur_ok) {
+                // R and Y (this warp's 32 columns) in two halves of 16:
+                // y_j = Y_j + exp(cs_j) R_j + D x_j, this thread's bytes of row r
+                if (!wait_bar_all(&bs->y_full, pn, bs, err)) goto done;
+                tc_fence_after();
+                __syncwarp();
+                const float uj = uu[r];
+                const float D_h = uu[2 * kTile];
+                const float2 u2 = make_float2(uj, uj), d2 = make_float2(D_h, D_h);
+                const uint8_t* sx = smem + kOffX + xs * kAtom;
+                uint4* dst = reinterpret_cast<uint4*>(
+                    prm.y + (((int64_t)cur_b * T + cur_t0 + r) * H + cur_h) * kP + 32 * ph);
+                const bool valid = cur_t0 + r < T;
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    float yv[16], rv[16];
+                    tmem_ld16(tmem + lane_base + kColY + 32 * ph + 16 * hf, yv);
+                    tmem_ld16(tmem + lane_base + kColR + 32 * ph + 16 * hf, rv);
+                    uint4 xq[2];
+#pragma unroll
+                    for (int c = 0; c < 2; ++c)
+                        xq[c] = *reinterpret_cast<const uint4*>(sx + sw128_off(r, 4 * ph + 2 * hf + c));
+                    tmem_ld_wait();
+                    if (hf == 1) {
                         tc_fence_before();
-                        mbar_arrive(&bs->s_empty);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) hreg[i] = fmaf(e, hreg[i], sv[i]);
-                    }
-                    if (s + 1 < U.nsub) {
-                        // R of this item is complete, so the operand buffer is free:
-                        // stage the state entering the next tile
-                        write_h_half(smem + kOffH, r, ph, hreg);
+                        mbar_arrive(&bs->ry_empty);
+                        // generic-proxy reads of the x slot are done before the next
+                        // TMA load into it
                         fence_proxy_async_smem();
-                        mbar_arrive(&bs->h_full);
-                    } else {
-                        // hand the state of head h on (flag released by warp 3) ...
-                        const int ps = npub % kPubStages;
-                        if (!wait_bar_all(&bs->pub_empty[ps], ((npub / kPubStages) & 1) ^ 1, bs, err))
-                            goto done;
-                        float* dst = prm.chain + ((int64_t)U.b * H + h) * PN + (int64_t)(32 * ph) * kN + r;
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) __stcg(dst + (int64_t)i * kN, hreg[i]);
-                        mbar_arrive(&bs->pub_full[ps]);
-                        ++npub;
-                        // ... and enter the next head, so the next item's products can start
-                        if (kh + 1 < kh_n) {
-                            if (!enter_head(U, h + 1, n + 1)) goto done;
-                        } else if (u + (int)gridDim.x < prm.nunits) {
-                            const Unit U2 = decode(prm, u + gridDim.x);
-                            if (!enter_head(U2, U2.hb * kh_n, n + 1)) goto done;
-                        }
+                        mbar_arrive(&bs->x_empty[xs]);
                     }
-                    if (has_next && !make_wx(n + 1)) goto done;
-                    // R and Y (this warp's 32 columns) in two halves of 16:
-                    // y_j = Y_j + exp(cs_j) R_j + D x_j, this thread's bytes of row r
-                    if (!wait_bar_all(&bs->y_full, pn, bs, err)) goto done;
-                    tc_fence_after();
-                    __syncwarp();
-                    {
-                        const int64_t t0 = U.tc0 + (int64_t)s * kTile;
-                        const uint8_t* sx = smem + kOffX + xs * kAtom;
-                        uint4* dst = reinterpret_cast<uint4*>(
-                            prm.y + (((int64_t)U.b * T + t0 + r) * H + h) * kP + 32 * ph);
-                        const bool valid = t0 + r < T;
+                    uint4 out[2];
 #pragma unroll
-                        for (int hf = 0; hf < 2; ++hf) {
-                            float yv[16], rv[16];
-                            tmem_ld16(tmem + lane_base + kColY + 32 * ph + 16 * hf, yv);
-                            tmem_ld16(tmem + lane_base + kColR + 32 * ph + 16 * hf, rv);
-                            uint4 xq[2];
+                    for (int c = 0; c < 2; ++c) {
+                        const uint32_t xw[4] = {xq[c].x, xq[c].y, xq[c].z, xq[c].w};
+                        uint32_t o[4];
 #pragma unroll
-                            for (int c = 0; c < 2; ++c)
-                                xq[c] = *reinterpret_cast<const uint4*>(sx + sw128_off(r, 4 * ph + 2 * hf + c));
-                            tmem_ld_wait();
-                            if (hf == 1) {
-                                tc_fence_before();
-                                mbar_arrive(&bs->ry_empty);
-                                // generic-proxy reads of the x slot are done before the next
-                                // TMA load into it
-                                fence_proxy_async_smem();
-                                mbar_arrive(&bs->x_empty[xs]);
-                            }
-                            uint4 out[2];
-#pragma unroll
-                            for (int c = 0; c < 2; ++c) {
-                                const uint32_t xw[4] = {xq[c].x, xq[c].y, xq[c].z, xq[c].w};
-                                uint32_t o[4];
-#pragma unroll
-                                for (int e2 = 0; e2 < 4; ++e2) {
-                                    const float2 xf = unpack_bf16(xw[e2]);
-                                    const int i0 = 8 * c + 2 * e2;
-                                    o[e2] = pack_bf16(fmaf(uj, rv[i0], yv[i0]) + D_h * xf.x,
-                                                      fmaf(uj, rv[i0 + 1], yv[i0 + 1]) + D_h * xf.y);
-                                }
-                                out[c] = make_uint4(o[0], o[1], o[2], o[3]);
-                            }
-                            if (valid) {
-                                dst[2 * hf] = out[0];
-                                dst[2 * hf + 1] = out[1];
-                            }
+                        for (int e2 = 0; e2 < 4; ++e2) {
+                            const int i0 = 8 * c + 2 * e2;
+                            const float2 t = fma2(u2, make_float2(rv[i0], rv[i0 + 1]),
+                                                  make_float2(yv[i0], yv[i0 + 1]));
+                            o[e2] = pack_bf16(fma2(d2, unpack_bf16(xw[e2]), t));
                         }
+                        out[c] = make_uint4(o[0], o[1], o[2], o[3]);
                     }
-                    mbar_arrive(&bs->cs_empty[cb]);
+                    if (valid) {
+                        dst[2 * hf] = out[0];
+                        dst[2 * hf + 1] = out[1];
+                    }
+                }
+                mbar_arrive(&bs->cs_empty[cb]);
+            }
+            // step the item iterator
+            cur_ok = nx_ok;
+            if (nx_ok) {
+                cur_b = nxU.b;
+                cur_h = nxU.hb * kh_n + nx_kh;
+                cur_t0 = nxU.tc0 + (int64_t)nx_s * kTile;
+                cur_last = nx_s + 1 >= nxU.nsub;
+                if (++nx_s >= nxU.nsub) {
+                    nx_s = 0;
+                    if (++nx_kh >= kh_n) {
+                        nx_kh = 0;
+                        nx_u += gridDim.x;
+                        nx_ok = nx_u < prm.nunits;
+                        if (nx_ok) nxU = decode(prm, nx_u);
+                    }
                 }
             }
         }

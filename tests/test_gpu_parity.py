@@ -257,6 +257,22 @@ def test_tensor_path_head_blocks(ssd, path_env, path, H, G):
     check_full(ssd, inp, 256, "bf16")
 
 
+@pytest.mark.parametrize("path", ["fused", "steps"])
+@pytest.mark.parametrize("scale", [8.0, 64.0])
+def test_tensor_path_strong_decay(ssd, path_env, path, scale):
+    # Every other head decays `scale` times faster, so that one 32-token block spans
+    # far more than 2^64 of decay: the masked diagonal block then takes its
+    # exponents element by element instead of in factored form. The other heads
+    # keep the mild decay of the standard draw.
+    path_env(path)
+    inp = make_inputs(batch=2, seqlen=700, nheads=8, headdim=64, ngroups=2, dstate=128,
+                      dtype="bf16", initial_states=True, seed=int(scale))
+    A = inp["A"].clone()
+    A[::2] *= scale
+    inp["A"] = A
+    check_full(ssd, inp, 256, "bf16")
+
+
 def test_tensor_steps_against_oracle(ssd, path_env):
     path_env("steps")
     Q = 256
