@@ -1,31 +1,30 @@
 // Warp-specialized, persistent single-pass SSD forward for sm_100a.
 //
-// Same arithmetic as the fused mode of ssd_tc.cu ("Transformers are SSMs",
-// Knowl 2, chunks chained through one L2-resident state buffer; the 128x128
-// diagonal blocks of each chunk in the quadratic masked form, the lower
-// off-diagonal 128-block through the state after the first tile), organised
-// so that HBM traffic, tensor-core MMAs and CUDA-core work overlap:
+// "Transformers are SSMs" (Knowl 2, Knowl 7) with the chunk equal to one
+// 128-token tile: per tile the diagonal block in the quadratic masked form,
+// everything before the tile through the state entering it. Roles:
 //
-//   warp 0      TMA producer: B/C tiles of a unit (one ring slot per 128-token
-//               tile), x tile of each item (2-deep ring)
+//   warp 0      TMA producer: B/C tile of each unit (2-slot ring), x tile of
+//               each item (3-slot ring)
 //   warp 1      TMEM owner and MMA issuer (one thread)
 //   warp 2      per item: dt loads, cumulative sum of dt*A (log2 units) and the
-//               per-token factors exp(cs_last - cs_i) dt_i and exp(cs_j)
+//               per-token factors
 //   warp 3      lane 0 releases chain flags
-//   warps 4-7   mask group: P = (C B^T) o mask from TMEM G into TMEM P (bf16,
-//               the A operand of the Y product), and w o x into shared memory
+//   warps 4-7   mask group: P = (C B^T) o L into TMEM (bf16, A operand of Y)
 //   warps 8-15  state/epilogue group, two warps per TMEM lane quarter, each
-//               owning half of the head dim: drains S, Y, R from TMEM, then
-//               h <- e h + S, the bf16 state operand, w o x of the next item,
-//               y = Y + exp(cs) R + D x to global memory, state hand-off
+//               owning half of the head dim: the head's state after the tile
+//               out of TMEM onto the chain, the next item's operands (bf16
+//               entering state for C h^T, exp(cs_last) h preloaded into the S
+//               accumulator, w o x), then y = Y + exp(cs) R + D x
 //
-// Work: persistent CTAs take units (chunk c, batch row b, block of k heads of
-// one group) round-robin in chunk-major order. An item is (unit, head, tile);
-// a unit's items run head-major so that each head's state stays in registers
-// between the tiles of its chunk.
+// Work: persistent CTAs take units (tile t, batch row b, block of k heads of
+// one group) round-robin in tile-major order; an item is (unit, head), so
+// consecutive items never share a state. The state of (b, h) after tile t
+// goes to tile t+1 through one L2-resident buffer and a release/acquire flag.
 //
-// Tensor memory (512 columns): G of tile slot 0 / 1 (128 each), P (64, bf16
-// pairs), Y (64), R (64), S (64).
+// Tensor memory (512 columns): G (128), P (64, bf16 pairs), S (64), R 2 x 64,
+// Y 2 x 64: R and Y are double-buffered so an item's products do not wait for
+// the previous item's epilogue.
 //
 // Every wait is bounded; a wait that gives up sets the error word and makes
 // every role leave its loop, after which the CTA drains its MMAs and exits.
@@ -46,7 +45,6 @@ constexpr int kP = 64;
 constexpr int kN = 128;
 constexpr int kThreads = 512;
 constexpr int kXStages = 3;
-constexpr int kWXStages = 1;
 constexpr int kCsStages = 4;
 constexpr int kPubStages = 4;
 
@@ -55,17 +53,17 @@ constexpr uint32_t kBCSlot = 2 * (kN / 64) * kAtom;  // B and C of one tile: 64 
 constexpr uint32_t kOffBC = 0;                   // 2 slots
 constexpr uint32_t kOffX = kOffBC + 2 * kBCSlot;    // kXStages x 16 KB
 constexpr uint32_t kOffWX = kOffX + kXStages * kAtom;
-constexpr uint32_t kOffH = kOffWX + kWXStages * kAtom;
-constexpr uint32_t kOffCs = kOffH + kN * 128;    // kCsStages x 4 arrays x 128 floats
-constexpr uint32_t kCsSlot = 6 * kTile * 4;   // cs, dt, w, u, v (per item), then D_h
+constexpr uint32_t kOffH = kOffWX + kAtom;
+constexpr uint32_t kOffCs = kOffH + kN * 128;    // kCsStages slots
+constexpr uint32_t kCsSlot = 6 * kTile * 4;   // cs, dt, w, u, v (per token), then D_h
 constexpr uint32_t kOffBar = kOffCs + kCsStages * kCsSlot;
 constexpr uint32_t kSmemBytes = kOffBar + 512;
 
-constexpr uint32_t kColG = 0;     // + 128 * slot
-constexpr uint32_t kColP = 256;
-constexpr uint32_t kColY = 320;
-constexpr uint32_t kColR = 384;
-constexpr uint32_t kColS = 448;
+constexpr uint32_t kColG = 0;
+constexpr uint32_t kColP = 128;
+constexpr uint32_t kColS = 192;
+constexpr uint32_t kColR = 256;   // + 64 * buffer
+constexpr uint32_t kColY = 384;   // + 64 * buffer
 
 constexpr float kLog2e = 1.4426950408889634f;
 // Widest cs range (log2 units) of a 32-row diagonal block for which the masked
@@ -83,20 +81,22 @@ struct Params {
     __nv_bfloat16* y;
     int* flags;
     int* error;
-    int64_t T, H, G, nc;
-    int Q, kheads, batch, nunits;
+    int64_t T;
+    int H, G, kheads, batch, nunits;
 };
 
 struct Bars {
-    uint64_t bc_full[2], bc_empty[2], g_full[2], g_empty[2];
+    uint64_t bc_full[2], bc_empty[2];
+    uint64_t g_full, g_empty;
     uint64_t x_full[kXStages], x_empty[kXStages];
     uint64_t cs_full[kCsStages], cs_empty[kCsStages];
-    uint64_t wx_full[kWXStages], wx_empty[kWXStages];
-    uint64_t p_full, p_empty, h_full, h_empty, fin;
-    uint64_t sr_full, s_empty;    // S and R done; S drained by the state group
-    uint64_t y_full, ry_empty;    // Y done; R and Y drained by the state group
-    uint64_t chain_ok;                          // chain flag observed (state group)
+    uint64_t wx_full, wx_empty;
+    uint64_t p_full, p_empty;
+    uint64_t h_full, h_empty;     // state operand and S preload written / operand read
+    uint64_t s_full;              // S complete: the head's state after the tile
+    uint64_t y_full[2], ry_empty[2];
     uint64_t pub_full[kPubStages], pub_empty[kPubStages];  // state stored / flag released
+    uint64_t fin;
     uint32_t tmem;
     int abort;
 };
@@ -178,18 +178,16 @@ __device__ __forceinline__ void write_h_half(uint8_t* sh, int n, int half, const
 }
 
 struct Unit {
-    int c, b, hb, nsub;
-    int64_t tc0;
+    int t, b, hb;     // tile, batch row, head block
+    int64_t t0;       // first token of the tile
 };
 __device__ __forceinline__ Unit decode(const Params& p, int u) {
-    const int nhb = (int)(p.H / p.kheads);
+    const int nhb = p.H / p.kheads;
     Unit r;
     r.hb = u % nhb;
     r.b = (u / nhb) % p.batch;
-    r.c = u / (nhb * p.batch);
-    r.tc0 = (int64_t)r.c * p.Q;
-    const int len = (int)min((int64_t)p.Q, p.T - r.tc0);
-    r.nsub = (len + kTile - 1) / kTile;
+    r.t = u / (nhb * p.batch);
+    r.t0 = (int64_t)r.t * kTile;
     return r;
 }
 
@@ -208,36 +206,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bs->bc_full[i], 1);
             mbar_init(&bs->bc_empty[i], 1);
-            mbar_init(&bs->g_full[i], 1);
-            mbar_init(&bs->g_empty[i], 128);
+            mbar_init(&bs->y_full[i], 1);
+            mbar_init(&bs->ry_empty[i], 256);
         }
+        mbar_init(&bs->g_full, 1);
+        mbar_init(&bs->g_empty, 128);
         for (int i = 0; i < kXStages; ++i) {
             mbar_init(&bs->x_full[i], 1);
-            // Y product (commit) + state group twice (w o x, then the skip term x)
-            mbar_init(&bs->x_empty[i], 1 + 256 + 256);
+            // Y product (commit) + mask group (w o x) + state group (skip term D x)
+            mbar_init(&bs->x_empty[i], 1 + 128 + 256);
         }
         for (int i = 0; i < kCsStages; ++i) {
             mbar_init(&bs->cs_full[i], 32);
             mbar_init(&bs->cs_empty[i], 128 + 256);
         }
+        mbar_init(&bs->wx_full, 128);
+        mbar_init(&bs->wx_empty, 1);
         mbar_init(&bs->p_full, 128);
         mbar_init(&bs->p_empty, 1);
-        for (int i = 0; i < kWXStages; ++i) {
-            mbar_init(&bs->wx_full[i], 256);
-            mbar_init(&bs->wx_empty[i], 1);   // S product (commit)
-        }
         mbar_init(&bs->h_full, 256);
         mbar_init(&bs->h_empty, 1);
-        mbar_init(&bs->sr_full, 1);
-        mbar_init(&bs->s_empty, 256);
-        mbar_init(&bs->y_full, 1);
-        mbar_init(&bs->ry_empty, 256);
-        mbar_init(&bs->fin, 1);
-        mbar_init(&bs->chain_ok, 1);
+        mbar_init(&bs->s_full, 1);
         for (int i = 0; i < kPubStages; ++i) {
             mbar_init(&bs->pub_full[i], 256);
             mbar_init(&bs->pub_empty[i], 1);
         }
+        mbar_init(&bs->fin, 1);
         bs->abort = 0;
         fence_barrier_init();
         prefetch_tmap(&tm_x);
@@ -254,7 +248,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool misaligned = (smem_u32(smem) & 1023u) != 0;
     const uint32_t tmem = bs->tmem;
     const int kh_n = prm.kheads;
-    const int64_t T = prm.T, H = prm.H;
+    const int64_t T = prm.T;
+    const int H = prm.H;
 
     if (misaligned) {
         // nothing
@@ -262,36 +257,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             int n = 0, m = 0;
-            for (int u = blockIdx.x; u < prm.nunits; u += gridDim.x) {
+            for (int u = blockIdx.x; u < prm.nunits; u += gridDim.x, ++m) {
                 const Unit U = decode(prm, u);
-                const int g = (int)((int64_t)U.hb * kh_n / (H / prm.G));
-                for (int kh = 0; kh < kh_n; ++kh) {
-                    const int h = U.hb * kh_n + kh;
-                    for (int s = 0; s < U.nsub; ++s, ++n) {
-                        if (kh == 0) {
-                            // B and C of tile s, shared by every head of the unit
-                            const int mm = m + s, sl = mm & 1;
-                            if (!wait_bar(&bs->bc_empty[sl], ((mm >> 1) & 1) ^ 1, bs, err))
-                                goto done;
-                            mbar_arrive_expect_tx(&bs->bc_full[sl], kBCSlot);
-                            uint8_t* base = smem + kOffBC + sl * kBCSlot;
-                            for (int a = 0; a < kN / 64; ++a) {
-                                tma_load_4d(base + a * kAtom, &tm_B, &bs->bc_full[sl], a * 64, g,
-                                            (int)(U.tc0 + s * kTile), U.b);
-                                tma_load_4d(base + kBCSlot / 2 + a * kAtom, &tm_C,
-                                            &bs->bc_full[sl], a * 64, g,
-                                            (int)(U.tc0 + s * kTile), U.b);
-                            }
-                        }
-                        const int xs = n % kXStages;
-                        if (!wait_bar(&bs->x_empty[xs], ((n / kXStages) & 1) ^ 1, bs, err))
-                            goto done;
-                        mbar_arrive_expect_tx(&bs->x_full[xs], kAtom);
-                        tma_load_4d(smem + kOffX + xs * kAtom, &tm_x, &bs->x_full[xs], 0, h,
-                                    (int)(U.tc0 + s * kTile), U.b);
-                    }
+                const int g = U.hb * kh_n / (H / prm.G);
+                // B and C of the tile, shared by every head of the unit
+                const int sl = m & 1;
+                if (!wait_bar(&bs->bc_empty[sl], ((m >> 1) & 1) ^ 1, bs, err)) goto done;
+                mbar_arrive_expect_tx(&bs->bc_full[sl], kBCSlot);
+                uint8_t* base = smem + kOffBC + sl * kBCSlot;
+                for (int a = 0; a < kN / 64; ++a) {
+                    tma_load_4d(base + a * kAtom, &tm_B, &bs->bc_full[sl], a * 64, g, (int)U.t0, U.b);
+                    tma_load_4d(base + kBCSlot / 2 + a * kAtom, &tm_C, &bs->bc_full[sl], a * 64, g,
+                                (int)U.t0, U.b);
                 }
-                m += U.nsub;
+                for (int kh = 0; kh < kh_n; ++kh, ++n) {
+                    const int xs = n % kXStages;
+                    if (!wait_bar(&bs->x_empty[xs], ((n / kXStages) & 1) ^ 1, bs, err)) goto done;
+                    mbar_arrive_expect_tx(&bs->x_full[xs], kAtom);
+                    tma_load_4d(smem + kOffX + xs * kAtom, &tm_x, &bs->x_full[xs], 0,
+                                U.hb * kh_n + kh, (int)U.t0, U.b);
+                }
             }
         }
     } else if (warp == 1) {
@@ -300,68 +285,75 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t idG = idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t idS = idesc_bf16(128, kP, 1, 1);
             constexpr uint32_t idY = idesc_bf16(128, kP, 0, 1);
-            int n = 0, m = 0;
-            for (int u = blockIdx.x; u < prm.nunits; u += gridDim.x) {
-                const Unit U = decode(prm, u);
-                for (int kh = 0; kh < kh_n; ++kh) {
-                    for (int s = 0; s < U.nsub; ++s, ++n) {
-                        const int sl = (m + s) & 1, xs = n % kXStages;
-                        if (kh == 0) {
-                            // G = C B^T of tile s (diagonal block), shared by the unit's heads
-                            const int ph = ((m + s) >> 1) & 1;
-                            if (!wait_bar(&bs->bc_full[sl], ph, bs, err)) goto drain;
-                            if (!wait_bar(&bs->g_empty[sl], ph ^ 1, bs, err)) goto drain;
-                            tc_fence_after();
-                            const uint32_t gB = smem_u32(smem + kOffBC + sl * kBCSlot);
-                            const uint64_t dGA = sw128_desc(gB + kBCSlot / 2, 16, 1024);
-                            const uint64_t dGB = sw128_desc(gB, 16, 1024);
+            const uint64_t dSB = sw128_desc(smem_u32(smem + kOffWX), kAtom, 1024);
+            const uint64_t dRB = sw128_desc(smem_u32(smem + kOffH), kAtom, 1024);
+            // G = C B^T of unit m's tile (the diagonal block), shared by the unit's
+            // heads; its slot is free once the mask group has used the previous G
+            auto issue_g = [&](int m) -> bool {
+                const int sl = m & 1;
+                if (!wait_bar(&bs->bc_full[sl], (m >> 1) & 1, bs, err)) return false;
+                if (!wait_bar(&bs->g_empty, (m & 1) ^ 1, bs, err)) return false;
+                tc_fence_after();
+                const uint32_t gB = smem_u32(smem + kOffBC + sl * kBCSlot);
+                const uint64_t dGA = sw128_desc(gB + kBCSlot / 2, 16, 1024);
+                const uint64_t dGB = sw128_desc(gB, 16, 1024);
 #pragma unroll
-                            for (int kk = 0; kk < kN / 16; ++kk) {
-                                // start address advances by (kk/4) atoms + (kk%4) x 32 bytes
-                                const uint64_t off = (uint64_t)(((kk >> 2) * kAtom + (kk & 3) * 32) >> 4);
-                                mma_bf16(tmem + kColG + 128 * sl, dGA + off, dGB + off, idG, kk > 0);
-                            }
-                            mma_commit(&bs->g_full[sl]);
-                        }
-                        const uint32_t pn = n & 1;
-                        const int ws = n % kWXStages;
-                        // S = B^T (w o x) and R = C h^T first: the state update waits on them
-                        if (!wait_bar(&bs->wx_full[ws], (n / kWXStages) & 1, bs, err)) goto drain;
-                        if (!wait_bar(&bs->h_full, pn, bs, err)) goto drain;
-                        if (!wait_bar(&bs->s_empty, pn ^ 1, bs, err)) goto drain;
-                        if (!wait_bar(&bs->ry_empty, pn ^ 1, bs, err)) goto drain;
-                        tc_fence_after();
-                        const uint32_t aB = smem_u32(smem + kOffBC + sl * kBCSlot);
-                        const uint64_t dSA = sw128_desc(aB, kAtom, 1024);
-                        const uint64_t dSB = sw128_desc(smem_u32(smem + kOffWX + ws * kAtom), kAtom, 1024);
-                        const uint64_t dRA = sw128_desc(aB + kBCSlot / 2, 16, 1024);
-                        const uint64_t dRB = sw128_desc(smem_u32(smem + kOffH), kAtom, 1024);
-#pragma unroll
-                        for (int kk = 0; kk < kTile / 16; ++kk) {
-                            const uint64_t rows = (uint64_t)(kk * (2048 >> 4));   // 16 rows of 128 B
-                            const uint64_t kofs = (uint64_t)(((kk >> 2) * kAtom + (kk & 3) * 32) >> 4);
-                            mma_bf16(tmem + kColS, dSA + rows, dSB + rows, idS, kk > 0);
-                            mma_bf16(tmem + kColR, dRA + kofs, dRB + rows, idY, kk > 0);
-                        }
-                        mma_commit(&bs->wx_empty[ws]);
-                        mma_commit(&bs->h_empty);
-                        mma_commit(&bs->sr_full);
-                        // Y = P x (P straight from TMEM)
-                        if (!wait_bar(&bs->p_full, pn, bs, err)) goto drain;
-                        if (!wait_bar(&bs->x_full[xs], (n / kXStages) & 1, bs, err)) goto drain;
-                        tc_fence_after();
-                        const uint64_t dXB = sw128_desc(smem_u32(smem + kOffX + xs * kAtom), kAtom, 1024);
-#pragma unroll
-                        for (int kk = 0; kk < kTile / 16; ++kk)
-                            mma_bf16_tmem_a(tmem + kColY, tmem + kColP + 8 * kk,
-                                            dXB + (uint64_t)(kk * (2048 >> 4)), idY, kk > 0);
-                        mma_commit(&bs->p_empty);
-                        mma_commit(&bs->x_empty[xs]);
-                        mma_commit(&bs->y_full);
-                        if (kh == kh_n - 1) mma_commit(&bs->bc_empty[sl]);
-                    }
+                for (int kk = 0; kk < kN / 16; ++kk) {
+                    // start address advances by (kk/4) atoms + (kk%4) x 32 bytes
+                    const uint64_t off = (uint64_t)(((kk >> 2) * kAtom + (kk & 3) * 32) >> 4);
+                    mma_bf16(tmem + kColG, dGA + off, dGB + off, idG, kk > 0);
                 }
-                m += U.nsub;
+                mma_commit(&bs->g_full);
+                return true;
+            };
+            int n = 0, m = 0;
+            if (blockIdx.x < prm.nunits && !issue_g(0)) goto drain;
+            for (int u = blockIdx.x; u < prm.nunits; u += gridDim.x, ++m) {
+                const int sl = m & 1;
+                const uint32_t aB = smem_u32(smem + kOffBC + sl * kBCSlot);
+                const uint64_t dSA = sw128_desc(aB, kAtom, 1024);
+                const uint64_t dRA = sw128_desc(aB + kBCSlot / 2, 16, 1024);
+                for (int kh = 0; kh < kh_n; ++kh, ++n) {
+                    const uint32_t pn = n & 1;
+                    const int yb = n & 1, xs = n % kXStages;
+                    // S += B^T (w o x) onto the preloaded exp(cs_last) h: the head's state
+                    // after the tile, which the state group waits on first
+                    if (!wait_bar(&bs->wx_full, pn, bs, err)) goto drain;
+                    if (!wait_bar(&bs->h_full, pn, bs, err)) goto drain;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < kTile / 16; ++kk) {
+                        const uint64_t rows = (uint64_t)(kk * (2048 >> 4));   // 16 rows of 128 B
+                        mma_bf16(tmem + kColS, dSA + rows, dSB + rows, idS, 1u);
+                    }
+                    mma_commit(&bs->wx_empty);
+                    mma_commit(&bs->s_full);
+                    // R = C h^T into buffer yb (free once item n-2's epilogue drained it)
+                    if (!wait_bar(&bs->ry_empty[yb], ((n >> 1) & 1) ^ 1, bs, err)) goto drain;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < kN / 16; ++kk) {
+                        const uint64_t rows = (uint64_t)(kk * (2048 >> 4));
+                        const uint64_t kofs = (uint64_t)(((kk >> 2) * kAtom + (kk & 3) * 32) >> 4);
+                        mma_bf16(tmem + kColR + 64 * yb, dRA + kofs, dRB + rows, idY, kk > 0);
+                    }
+                    mma_commit(&bs->h_empty);
+                    // Y = P x (P straight from TMEM)
+                    if (!wait_bar(&bs->p_full, pn, bs, err)) goto drain;
+                    if (!wait_bar(&bs->x_full[xs], (n / kXStages) & 1, bs, err)) goto drain;
+                    tc_fence_after();
+                    const uint64_t dXB = sw128_desc(smem_u32(smem + kOffX + xs * kAtom), kAtom, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < kTile / 16; ++kk)
+                        mma_bf16_tmem_a(tmem + kColY + 64 * yb, tmem + kColP + 8 * kk,
+                                        dXB + (uint64_t)(kk * (2048 >> 4)), idY, kk > 0);
+                    mma_commit(&bs->p_empty);
+                    mma_commit(&bs->x_empty[xs]);
+                    mma_commit(&bs->y_full[yb]);
+                }
+                // every product reading this unit's B/C has been issued
+                mma_commit(&bs->bc_empty[sl]);
+                if (u + (int)gridDim.x < prm.nunits && !issue_g(m + 1)) goto drain;
             }
         drain:
             // every MMA issued so far is complete before TMEM is released
@@ -373,66 +365,79 @@ __global__ void __launch_bounds__(kThreads, 1)
         int n = 0;
         for (int u = blockIdx.x; u < prm.nunits; u += gridDim.x) {
             const Unit U = decode(prm, u);
-            for (int kh = 0; kh < kh_n; ++kh) {
+            const int len = (int)min((int64_t)kTile, T - U.t0);
+            for (int kh = 0; kh < kh_n; ++kh, ++n) {
                 const int h = U.hb * kh_n + kh;
                 const float a2 = prm.A[h] * kLog2e;
                 const float d_h = prm.D ? prm.D[h] : 0.f;
-                for (int s = 0; s < U.nsub; ++s, ++n) {
-                    const int cb = n % kCsStages;
-                    if (!wait_bar_all(&bs->cs_empty[cb], ((n / kCsStages) & 1) ^ 1, bs, err)) goto done;
-                    const int64_t t0 = U.tc0 + (int64_t)s * kTile;
-                    const int len = (int)min((int64_t)kTile, T - t0);
-                    float dtv[4], v[4];
+                const int cb = n % kCsStages;
+                if (!wait_bar_all(&bs->cs_empty[cb], ((n / kCsStages) & 1) ^ 1, bs, err)) goto done;
+                float dtv[4], v[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int t = lane * 4 + e;
-                        dtv[e] = t < len ? __ldg(prm.dt + ((int64_t)U.b * T + t0 + t) * H + h) : 0.f;
-                    }
-                    float run = 0.f;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        run += dtv[e] * a2;
-                        v[e] = run;
-                    }
-                    float incl = run;
-#pragma unroll
-                    for (int off = 1; off < 32; off <<= 1) {
-                        const float o = __shfl_up_sync(0xffffffffu, incl, off);
-                        if (lane >= off) incl += o;
-                    }
-                    const float excl = incl - run;
-                    const float last = __shfl_sync(0xffffffffu, incl, 31);
-                    float* cs = reinterpret_cast<float*>(smem + kOffCs + cb * kCsSlot);
-                    float* dts = cs + kTile;
-                    float* w = dts + kTile;
-                    float* uu = w + kTile;
-                    float* vv = uu + kTile;
-                    // cs at the last row of this lane's 32-column block (lanes 8b..8b+7 hold block b)
-                    const float cref = __shfl_sync(0xffffffffu, incl, (lane | 7));
-                    float4 c4, d4, w4, u4, v4;
-                    float* cp = &c4.x;
-                    float* dp = &d4.x;
-                    float* wp = &w4.x;
-                    float* up = &u4.x;
-                    float* vp = &v4.x;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float ce = excl + v[e];
-                        cp[e] = ce;
-                        dp[e] = dtv[e];
-                        wp[e] = exp2f(last - ce) * dtv[e];
-                        up[e] = exp2f(ce);
-                        vp[e] = exp2f(cref - ce) * dtv[e];
-                    }
-                    reinterpret_cast<float4*>(cs)[lane] = c4;
-                    reinterpret_cast<float4*>(dts)[lane] = d4;
-                    reinterpret_cast<float4*>(w)[lane] = w4;
-                    reinterpret_cast<float4*>(uu)[lane] = u4;
-                    reinterpret_cast<float4*>(vv)[lane] = v4;
-                    if (lane == 0) vv[kTile] = d_h;
-                    __syncwarp();
-                    mbar_arrive(&bs->cs_full[cb]);
+                for (int e = 0; e < 4; ++e) {
+                    const int t = lane * 4 + e;
+                    dtv[e] = t < len ? __ldg(prm.dt + ((int64_t)U.b * T + U.t0 + t) * H + h) : 0.f;
                 }
+                // The state entering tile t of (b, h) is tile t-1's: wait for its flag here,
+                // ahead of the consumers (cs_full, arrived after this acquire, orders the
+                // state group's loads of that state after it).
+                if (U.t > 0 && lane == 0) {
+                    const int* f = prm.flags + (int64_t)U.b * H + h;
+                    bool ok = false;
+                    const uint64_t t0 = global_ns();
+                    for (uint32_t it = 0;; ++it) {
+                        if (ld_acquire(f) >= U.t) { ok = true; break; }
+                        if (it >= 4) __nanosleep(64);
+                        if ((it & 15) == 15 &&
+                            (*(volatile int*)&bs->abort || global_ns() - t0 > 2000000000ull))
+                            break;
+                    }
+                    if (!ok) {
+                        *(volatile int*)&bs->abort = 1;
+                        atomicExch(err, 1);
+                    }
+                }
+                __syncwarp();
+                float run = 0.f;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    run += dtv[e] * a2;
+                    v[e] = run;
+                }
+                float incl = run;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float o = __shfl_up_sync(0xffffffffu, incl, off);
+                    if (lane >= off) incl += o;
+                }
+                const float excl = incl - run;
+                const float last = __shfl_sync(0xffffffffu, incl, 31);
+                float* cs = reinterpret_cast<float*>(smem + kOffCs + cb * kCsSlot);
+                // cs at the last row of this lane's 32-column block (lanes 8b..8b+7 hold block b)
+                const float cref = __shfl_sync(0xffffffffu, incl, (lane | 7));
+                float4 c4, d4, w4, u4, v4;
+                float* cp = &c4.x;
+                float* dp = &d4.x;
+                float* wp = &w4.x;
+                float* up = &u4.x;
+                float* vp = &v4.x;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float ce = excl + v[e];
+                    cp[e] = ce;
+                    dp[e] = dtv[e];
+                    wp[e] = exp2f(last - ce) * dtv[e];
+                    up[e] = exp2f(ce);
+                    vp[e] = exp2f(cref - ce) * dtv[e];
+                }
+                reinterpret_cast<float4*>(cs)[lane] = c4;
+                reinterpret_cast<float4*>(cs + kTile)[lane] = d4;
+                reinterpret_cast<float4*>(cs + 2 * kTile)[lane] = w4;
+                reinterpret_cast<float4*>(cs + 3 * kTile)[lane] = u4;
+                reinterpret_cast<float4*>(cs + 4 * kTile)[lane] = v4;
+                if (lane == 0) cs[5 * kTile] = d_h;
+                __syncwarp();
+                mbar_arrive(&bs->cs_full[cb]);
             }
         }
     } else if (warp == 3) {
@@ -445,257 +450,231 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int u = blockIdx.x; u < prm.nunits; u += gridDim.x) {
                 const Unit U = decode(prm, u);
                 for (int kh = 0; kh < kh_n; ++kh, ++np) {
-                    const int h = U.hb * kh_n + kh;
                     const int ps = np % kPubStages;
                     if (!wait_bar(&bs->pub_full[ps], (np / kPubStages) & 1, bs, err)) goto done;
                     __threadfence();
-                    st_release(prm.flags + (int64_t)U.b * H + h, U.c + 1);
+                    st_release(prm.flags + (int64_t)U.b * H + U.hb * kh_n + kh, U.t + 1);
                     mbar_arrive(&bs->pub_empty[ps]);
                 }
             }
         }
     } else if (warp >= 4 && warp < 8) {
         // ------------------------------------------------------------ mask group
+        // per item: w o x (the S product's operand), then P = G o L
         const int wq = warp - 4;
         const int j = tid - 128;  // row of the tile == TMEM lane
+        const int jj = j & 31;    // row within this warp's diagonal block
         const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
         int n = 0, m = 0;
-        for (int u = blockIdx.x; u < prm.nunits; u += gridDim.x) {
-            const Unit U = decode(prm, u);
-            for (int kh = 0; kh < kh_n; ++kh) {
-                for (int s = 0; s < U.nsub; ++s, ++n) {
-                    const int mm = m + s, sl = mm & 1;
-                    const uint32_t pn = n & 1;
-                    const int cb = n % kCsStages;
-                    if (!wait_bar_all(&bs->cs_full[cb], (n / kCsStages) & 1, bs, err)) goto done;
-                    const float* cs = reinterpret_cast<const float*>(smem + kOffCs + cb * kCsSlot);
-                    const float* dts = cs + kTile;
-                    const float* vv = dts + 3 * kTile;
-                    // masked diagonal block P = G o mask into TMEM
-                    if (kh == 0 && !wait_bar_all(&bs->g_full[sl], (mm >> 1) & 1, bs, err)) goto done;
-                    if (!wait_bar_all(&bs->p_empty, pn ^ 1, bs, err)) goto done;
-                    tc_fence_after();
-                    __syncwarp();
-                    const float csj = cs[j];
-                    const int jj = j & 31;   // row within this warp's diagonal block
+        for (int u = blockIdx.x; u < prm.nunits; u += gridDim.x, ++m) {
+            if (!wait_bar_all(&bs->g_full, m & 1, bs, err)) goto done;
+            for (int kh = 0; kh < kh_n; ++kh, ++n) {
+                const int cb = n % kCsStages;
+                if (!wait_bar_all(&bs->cs_full[cb], (n / kCsStages) & 1, bs, err)) goto done;
+                const float* cs = reinterpret_cast<const float*>(smem + kOffCs + cb * kCsSlot);
+                const float* dts = cs + kTile;
+                const float* vv = cs + 4 * kTile;
+                // w o x: row j of the x tile scaled by w_j = exp(cs_last - cs_j) dt_j, the
+                // B operand of the S product
+                {
+                    const int xs = n % kXStages;
+                    if (!wait_bar_all(&bs->x_full[xs], (n / kXStages) & 1, bs, err)) goto done;
+                    if (!wait_bar_all(&bs->wx_empty, (n & 1) ^ 1, bs, err)) goto done;
+                    const float w = cs[2 * kTile + j];
+                    const float2 w2 = make_float2(w, w);
+                    const uint8_t* sx = smem + kOffX + xs * kAtom;
+                    uint8_t* swx = smem + kOffWX;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint32_t off = sw128_off(j, c);
+                        const uint4 xv = *reinterpret_cast<const uint4*>(sx + off);
+                        *reinterpret_cast<uint4*>(swx + off) =
+                            make_uint4(pack_bf16(mul2(w2, unpack_bf16(xv.x))), pack_bf16(mul2(w2, unpack_bf16(xv.y))),
+                                       pack_bf16(mul2(w2, unpack_bf16(xv.z))), pack_bf16(mul2(w2, unpack_bf16(xv.w))));
+                    }
+                    fence_proxy_async_smem();
+                    mbar_arrive(&bs->wx_full);
+                    mbar_arrive(&bs->x_empty[xs]);
+                }
+                if (!wait_bar_all(&bs->p_empty, (n & 1) ^ 1, bs, err)) goto done;
+                tc_fence_after();
+                __syncwarp();
+                const float csj = cs[j];
 #pragma unroll 1
-                    for (int blk = 0; blk < 4; ++blk) {
-                        uint32_t pk[16];
-                        if (blk > wq) {
+                for (int blk = 0; blk < 4; ++blk) {
+                    uint32_t pk[16];
+                    if (blk > wq) {
 #pragma unroll
-                            for (int q = 0; q < 16; ++q) pk[q] = 0u;
+                        for (int q = 0; q < 16; ++q) pk[q] = 0u;
+                    } else {
+                        float gv[32];
+                        tmem_ld32(tmem + lane_base + kColG + 32 * blk, gv);
+                        // exp(cs_j - cs_i) dt_i = exp(cs_j - cs_e) * v_i with e the last row of
+                        // column block blk and v_i = exp(cs_e - cs_i) dt_i (<= dt_i). Below the
+                        // diagonal block the first factor is <= 1 too; on it, it is >= 1 and
+                        // bounded by the block's own cs range, which decides whether the
+                        // factored form is safe in fp32 or the exponent is taken per element.
+                        const float ce = cs[32 * blk + 31];
+                        const float a = exp2f(csj - ce);
+                        const bool exact = blk == wq && cs[32 * blk] - ce > kFactorRangeLog2;
+                        const float2 a2 = make_float2(a, a);
+                        tmem_ld_wait();
+                        if (blk < wq) {
+#pragma unroll
+                            for (int e4 = 0; e4 < 8; ++e4) {
+                                const float4 v4 = reinterpret_cast<const float4*>(vv)[blk * 8 + e4];
+                                pk[e4 * 2] = pack_bf16(mul2(make_float2(gv[e4 * 4], gv[e4 * 4 + 1]),
+                                                            mul2(make_float2(v4.x, v4.y), a2)));
+                                pk[e4 * 2 + 1] = pack_bf16(mul2(make_float2(gv[e4 * 4 + 2], gv[e4 * 4 + 3]),
+                                                                mul2(make_float2(v4.z, v4.w), a2)));
+                            }
+                        } else if (!exact) {
+#pragma unroll
+                            for (int e4 = 0; e4 < 8; ++e4) {
+                                const float4 v4 = reinterpret_cast<const float4*>(vv)[blk * 8 + e4];
+                                float2 p01 = mul2(make_float2(gv[e4 * 4], gv[e4 * 4 + 1]),
+                                                  mul2(make_float2(v4.x, v4.y), a2));
+                                float2 p23 = mul2(make_float2(gv[e4 * 4 + 2], gv[e4 * 4 + 3]),
+                                                  mul2(make_float2(v4.z, v4.w), a2));
+                                const int i0 = e4 * 4;   // causal mask: column i kept while i <= row
+                                p01.x = i0 <= jj ? p01.x : 0.f;
+                                p01.y = i0 + 1 <= jj ? p01.y : 0.f;
+                                p23.x = i0 + 2 <= jj ? p23.x : 0.f;
+                                p23.y = i0 + 3 <= jj ? p23.y : 0.f;
+                                pk[e4 * 2] = pack_bf16(p01);
+                                pk[e4 * 2 + 1] = pack_bf16(p23);
+                            }
                         } else {
-                            float gv[32];
-                            tmem_ld32(tmem + lane_base + kColG + 128 * sl + 32 * blk, gv);
-                            // exp(cs_j - cs_i) dt_i = exp(cs_j - cs_e) * v_i with e the last row of
-                            // column block blk and v_i = exp(cs_e - cs_i) dt_i (<= dt_i). Below the
-                            // diagonal block the first factor is <= 1 too; on it, it is >= 1 and
-                            // bounded by the block's own cs range, which decides whether the
-                            // factored form is safe in fp32 or the exponent is taken per element.
-                            const float ce = cs[32 * blk + 31];
-                            const float a = exp2f(csj - ce);
-                            const bool exact = blk == wq && cs[32 * blk] - ce > kFactorRangeLog2;
-                            const float2 a2 = make_float2(a, a);
-                            tmem_ld_wait();
-                            if (blk < wq) {
 #pragma unroll
-                                for (int e4 = 0; e4 < 8; ++e4) {
-                                    const float4 v4 = reinterpret_cast<const float4*>(vv)[blk * 8 + e4];
-                                    pk[e4 * 2] = pack_bf16(mul2(make_float2(gv[e4 * 4], gv[e4 * 4 + 1]),
-                                                                mul2(make_float2(v4.x, v4.y), a2)));
-                                    pk[e4 * 2 + 1] = pack_bf16(mul2(make_float2(gv[e4 * 4 + 2], gv[e4 * 4 + 3]),
-                                                                    mul2(make_float2(v4.z, v4.w), a2)));
-                                }
-                            } else if (!exact) {
-#pragma unroll
-                                for (int e4 = 0; e4 < 8; ++e4) {
-                                    const float4 v4 = reinterpret_cast<const float4*>(vv)[blk * 8 + e4];
-                                    float2 p01 = mul2(make_float2(gv[e4 * 4], gv[e4 * 4 + 1]),
-                                                      mul2(make_float2(v4.x, v4.y), a2));
-                                    float2 p23 = mul2(make_float2(gv[e4 * 4 + 2], gv[e4 * 4 + 3]),
-                                                      mul2(make_float2(v4.z, v4.w), a2));
-                                    const int i0 = e4 * 4;   // causal mask: column i kept while i <= row
-                                    p01.x = i0 <= jj ? p01.x : 0.f;
-                                    p01.y = i0 + 1 <= jj ? p01.y : 0.f;
-                                    p23.x = i0 + 2 <= jj ? p23.x : 0.f;
-                                    p23.y = i0 + 3 <= jj ? p23.y : 0.f;
-                                    pk[e4 * 2] = pack_bf16(p01);
-                                    pk[e4 * 2 + 1] = pack_bf16(p23);
-                                }
-                            } else {
-#pragma unroll
-                                for (int e4 = 0; e4 < 8; ++e4) {
-                                    const float4 c4 = reinterpret_cast<const float4*>(cs)[blk * 8 + e4];
-                                    const float4 d4 = reinterpret_cast<const float4*>(dts)[blk * 8 + e4];
-                                    const int i0 = blk * 32 + e4 * 4;
-                                    const float m0 = exp2f(csj - c4.x) * d4.x;
-                                    const float m1 = exp2f(csj - c4.y) * d4.y;
-                                    const float m2 = exp2f(csj - c4.z) * d4.z;
-                                    const float m3 = exp2f(csj - c4.w) * d4.w;
-                                    const float p0 = (i0 <= j) ? gv[e4 * 4] * m0 : 0.f;
-                                    const float p1 = (i0 + 1 <= j) ? gv[e4 * 4 + 1] * m1 : 0.f;
-                                    const float p2 = (i0 + 2 <= j) ? gv[e4 * 4 + 2] * m2 : 0.f;
-                                    const float p3 = (i0 + 3 <= j) ? gv[e4 * 4 + 3] * m3 : 0.f;
-                                    pk[e4 * 2] = pack_bf16(p0, p1);
-                                    pk[e4 * 2 + 1] = pack_bf16(p2, p3);
-                                }
+                            for (int e4 = 0; e4 < 8; ++e4) {
+                                const float4 c4 = reinterpret_cast<const float4*>(cs)[blk * 8 + e4];
+                                const float4 d4 = reinterpret_cast<const float4*>(dts)[blk * 8 + e4];
+                                const int i0 = blk * 32 + e4 * 4;
+                                const float m0 = exp2f(csj - c4.x) * d4.x;
+                                const float m1 = exp2f(csj - c4.y) * d4.y;
+                                const float m2 = exp2f(csj - c4.z) * d4.z;
+                                const float m3 = exp2f(csj - c4.w) * d4.w;
+                                const float p0 = (i0 <= j) ? gv[e4 * 4] * m0 : 0.f;
+                                const float p1 = (i0 + 1 <= j) ? gv[e4 * 4 + 1] * m1 : 0.f;
+                                const float p2 = (i0 + 2 <= j) ? gv[e4 * 4 + 2] * m2 : 0.f;
+                                const float p3 = (i0 + 3 <= j) ? gv[e4 * 4 + 3] * m3 : 0.f;
+                                pk[e4 * 2] = pack_bf16(p0, p1);
+                                pk[e4 * 2 + 1] = pack_bf16(p2, p3);
                             }
                         }
-                        tmem_st16(tmem + lane_base + kColP + 16 * blk, pk);
                     }
-                    tmem_st_wait();
-                    tc_fence_before();
-                    mbar_arrive(&bs->p_full);
-                    if (kh == kh_n - 1) mbar_arrive(&bs->g_empty[sl]);
-                    mbar_arrive(&bs->cs_empty[cb]);
+                    tmem_st16(tmem + lane_base + kColP + 16 * blk, pk);
                 }
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(&bs->p_full);
+                if (kh == kh_n - 1) mbar_arrive(&bs->g_empty);
+                mbar_arrive(&bs->cs_empty[cb]);
             }
-            m += U.nsub;
         }
     } else if (warp >= 8) {
         // ------------------------------------------------------------ state / epilogue group
-        // Iteration n finishes item n and prepares item n+1: drain S_n as soon as it is
-        // done (so the next S and R can follow Y on the tensor pipe), update the state,
-        // stage the next state operand (next tile of this head, or publish this head and
-        // enter the next one), build w o x of item n+1, then drain Y_n and R_n into y_n.
+        // Iteration n finishes item n and prepares item n+1:
+        //   1. the next head's entering state is fetched (its loads in flight),
+        //   2. S_n, the state of item n's head after its tile, goes from TMEM onto the chain,
+        //   3. the bf16 state operand and exp(cs_last) h preloaded into S, both for item
+        //      n+1, so its products run on the tensor pipe during step 4,
+        //   4. y_n = Y_n + exp(cs) R_n + D x_n.
         const int q = warp & 3;                 // TMEM lane quarter
         const int ph = (warp - 8) >> 2;         // half of the head dim this warp owns
         const int r = q * 32 + lane;            // tile row for outputs, state index n
-        const bool leader = (warp == 8 && lane == 0);
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         const int64_t PN = (int64_t)kP * kN;
-        int nchain = 0, npub = 0;
-        float hreg[32];  // h[32 ph + i][r] of the head being processed
-        // State entering chunk U.c of head h into hreg, and its bf16 copy as the B operand
-        // of the first tile's C h^T (item `item`). Returns false on abort.
-        auto enter_head = [&](const Unit& U, int h, int item) -> bool {
-            if (U.c == 0) {
+        // Fetching the next unit's state before this item's state is handed on is safe
+        // only if that state's predecessors are all earlier units than this one (more
+        // units per tile than CTAs); otherwise it waits for the hand-off.
+        const bool early_ok = prm.batch * (H / kh_n) > (int)gridDim.x;
+        int npub = 0;
+        float hn[32];    // h[32 ph + i][r] entering the next item's tile
+        // the state of head h entering tile U.t (item `item`); returns false on abort.
+        // Tile t-1's flag was acquired by the cumsum warp before it released the item's
+        // cs slot, so waiting for that slot orders these loads after the flag.
+        auto fetch = [&](const Unit& U, int h, int item) -> bool {
+            if (!wait_bar_all(&bs->cs_full[item % kCsStages], (item / kCsStages) & 1, bs, err))
+                return false;
+            if (U.t == 0) {
                 const float* src =
                     prm.init ? prm.init + ((int64_t)U.b * H + h) * PN + (int64_t)(32 * ph) * kN + r : nullptr;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) hreg[i] = src ? __ldg(src + (int64_t)i * kN) : 0.f;
-            } else {
-                if (leader) {
-                    const int* f = prm.flags + (int64_t)U.b * H + h;
-                    bool ok = false;
-                    const uint64_t t0 = global_ns();
-                    for (uint32_t it = 0;; ++it) {
-                        if (ld_acquire(f) >= U.c) { ok = true; break; }
-                        if (it >= 8) __nanosleep(32);
-                        if ((it & 15) == 15 &&
-                            (*(volatile int*)&bs->abort || global_ns() - t0 > 2000000000ull))
-                            break;
-                    }
-                    if (!ok) {
-                        *(volatile int*)&bs->abort = 1;
-                        atomicExch(err, 1);
-                    }
-                    mbar_arrive(&bs->chain_ok);
-                }
-                if (!wait_bar_all(&bs->chain_ok, nchain & 1, bs, err)) return false;
-                ++nchain;
-                if (*(volatile int*)&bs->abort) return false;
-                __threadfence();
-                const float* src = prm.chain + ((int64_t)U.b * H + h) * PN + (int64_t)(32 * ph) * kN + r;
-#pragma unroll
-                for (int i = 0; i < 32; ++i) hreg[i] = __ldcg(src + (int64_t)i * kN);
+                for (int i = 0; i < 32; ++i) hn[i] = src ? __ldg(src + (int64_t)i * kN) : 0.f;
+                return true;
             }
-            if (!wait_bar_all(&bs->h_empty, (item & 1) ^ 1, bs, err)) return false;
-            write_h_half(smem + kOffH, r, ph, hreg);
-            fence_proxy_async_smem();
-            mbar_arrive(&bs->h_full);
+            const float* src = prm.chain + ((int64_t)U.b * H + h) * PN + (int64_t)(32 * ph) * kN + r;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) hn[i] = __ldcg(src + (int64_t)i * kN);
             return true;
         };
-        // items in the order every role walks them: nx is the next one (unit, head,
-        // tile), cur the one being finished (batch row, head, first token, last tile
-        // of its chunk or not)
-        int nx_u = blockIdx.x, nx_kh = 0, nx_s = 0;
+        // items in the order every role walks them: nx is the next one (unit, head),
+        // cur the one being finished
+        int nx_u = blockIdx.x, nx_kh = 0;
         bool nx_ok = nx_u < prm.nunits;
         Unit nxU{};
         if (nx_ok) nxU = decode(prm, nx_u);
-        bool cur_ok = false, cur_last = false;
+        bool cur_ok = false;
         int cur_b = 0, cur_h = 0;
         int64_t cur_t0 = 0;
         for (int n = -1; cur_ok || nx_ok; ++n) {
-            const int nn = n < 0 ? 0 : n;
-            const uint32_t pn = nn & 1;
-            const int cb = nn % kCsStages, xs = nn % kXStages;
-            const float* cs = reinterpret_cast<const float*>(smem + kOffCs + cb * kCsSlot);
-            const float* uu = cs + 3 * kTile;
+            const int item = n + 1;
+            const int nh = nxU.hb * kh_n + nx_kh;   // head of the next item
+            // 1. the next item's entering state
+            const bool early = nx_ok && (nx_kh != 0 || early_ok);
+            if (early && !fetch(nxU, nh, item)) goto done;
+            // 2. S_n (this warp's 32 columns) is the state after item n's tile: hand it on
             if (cur_ok) {
-                if (!wait_bar_all(&bs->cs_full[cb], (nn / kCsStages) & 1, bs, err)) goto done;
-                if (!wait_bar_all(&bs->sr_full, pn, bs, err)) goto done;
+                if (!wait_bar_all(&bs->s_full, n & 1, bs, err)) goto done;
                 tc_fence_after();
                 __syncwarp();
-                // drain S (this warp's 32 columns), release it, update the state
-                {
-                    const float e = uu[kTile - 1];   // exp(cs_last): decay over the whole tile
-                    const float2 e2 = make_float2(e, e);
-                    float sv[32];
-                    tmem_ld32(tmem + lane_base + kColS + 32 * ph, sv);
-                    tmem_ld_wait();
-                    tc_fence_before();
-                    mbar_arrive(&bs->s_empty);
+                float sv[32];
+                tmem_ld32(tmem + lane_base + kColS + 32 * ph, sv);
+                tmem_ld_wait();
+                const int ps = npub % kPubStages;
+                if (!wait_bar_all(&bs->pub_empty[ps], ((npub / kPubStages) & 1) ^ 1, bs, err))
+                    goto done;
+                float* dst = prm.chain + ((int64_t)cur_b * H + cur_h) * PN + (int64_t)(32 * ph) * kN + r;
 #pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        const float2 t = fma2(e2, make_float2(hreg[i], hreg[i + 1]),
-                                              make_float2(sv[i], sv[i + 1]));
-                        hreg[i] = t.x;
-                        hreg[i + 1] = t.y;
-                    }
-                }
-                if (!cur_last) {
-                    // R of this item is complete, so the operand buffer is free:
-                    // stage the state entering the next tile
-                    write_h_half(smem + kOffH, r, ph, hreg);
-                    fence_proxy_async_smem();
-                    mbar_arrive(&bs->h_full);
-                } else {
-                    // hand the state of head h on (flag released by warp 3)
-                    const int ps = npub % kPubStages;
-                    if (!wait_bar_all(&bs->pub_empty[ps], ((npub / kPubStages) & 1) ^ 1, bs, err))
-                        goto done;
-                    float* dst = prm.chain + ((int64_t)cur_b * H + cur_h) * PN + (int64_t)(32 * ph) * kN + r;
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) __stcg(dst + (int64_t)i * kN, hreg[i]);
-                    mbar_arrive(&bs->pub_full[ps]);
-                    ++npub;
-                }
+                for (int i = 0; i < 32; ++i) __stcg(dst + (int64_t)i * kN, sv[i]);
+                mbar_arrive(&bs->pub_full[ps]);
+                ++npub;
             }
+            if (nx_ok && !early && !fetch(nxU, nh, item)) goto done;
+            // 3. operands of the next item
             if (nx_ok) {
-                const int item = n + 1;
-                // a new head: its entering state, so the next item's products can start
-                if (nx_s == 0 && !enter_head(nxU, nxU.hb * kh_n + nx_kh, item)) goto done;
-                // w o x of the next item: row r of its x tile scaled by
-                // w_r = exp(cs_last - cs_r) dt_r, this warp's half of the head dim
-                const int xs1 = item % kXStages, ws1 = item % kWXStages, cb1 = item % kCsStages;
-                if (!wait_bar_all(&bs->cs_full[cb1], (item / kCsStages) & 1, bs, err)) goto done;
-                if (!wait_bar_all(&bs->x_full[xs1], (item / kXStages) & 1, bs, err)) goto done;
-                if (!wait_bar_all(&bs->wx_empty[ws1], ((item / kWXStages) & 1) ^ 1, bs, err)) goto done;
-                const float w = reinterpret_cast<const float*>(smem + kOffCs + cb1 * kCsSlot)[2 * kTile + r];
-                const float2 w2 = make_float2(w, w);
-                const uint8_t* sx = smem + kOffX + xs1 * kAtom;
-                uint8_t* swx = smem + kOffWX + ws1 * kAtom;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const uint32_t off = sw128_off(r, 4 * ph + c);
-                    const uint4 xv = *reinterpret_cast<const uint4*>(sx + off);
-                    *reinterpret_cast<uint4*>(swx + off) =
-                        make_uint4(pack_bf16(mul2(w2, unpack_bf16(xv.x))), pack_bf16(mul2(w2, unpack_bf16(xv.y))),
-                                   pack_bf16(mul2(w2, unpack_bf16(xv.z))), pack_bf16(mul2(w2, unpack_bf16(xv.w))));
-                }
+                const float* cs1 = reinterpret_cast<const float*>(smem + kOffCs + (item % kCsStages) * kCsSlot);
+                // bf16 entering state, the B operand of C h^T (free once R_n is done) ...
+                if (!wait_bar_all(&bs->h_empty, (item & 1) ^ 1, bs, err)) goto done;
+                write_h_half(smem + kOffH, r, ph, hn);
                 fence_proxy_async_smem();
-                mbar_arrive(&bs->wx_full[ws1]);
-                mbar_arrive(&bs->x_empty[xs1]);
+                // ... and exp(cs_last) h preloaded into S (drained in step 2), which the
+                // S product then accumulates onto
+                {
+                    const float e = cs1[4 * kTile - 1];   // exp(cs_last): decay over the tile
+                    uint32_t pre[16];
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) pre[i] = __float_as_uint(e * hn[16 * hf + i]);
+                        tmem_st16(tmem + lane_base + kColS + 32 * ph + 16 * hf, pre);
+                    }
+                    tmem_st_wait();
+                }
+                tc_fence_before();
+                mbar_arrive(&bs->h_full);
             }
+            // 4. y of item n from R and Y (this warp's 32 columns):
+            // y_j = Y_j + exp(cs_j) R_j + D x_j, this thread's bytes of row r
             if (cur_ok) {
-                // R and Y (this warp's 32 columns) in two halves of 16:
-                // y_j = Y_j + exp(cs_j) R_j + D x_j, this thread's bytes of row r
-                if (!wait_bar_all(&bs->y_full, pn, bs, err)) goto done;
+                const int yb = n & 1, xs = n % kXStages, cb = n % kCsStages;
+                const float* cs = reinterpret_cast<const float*>(smem + kOffCs + cb * kCsSlot);
+                if (!wait_bar_all(&bs->y_full[yb], (n >> 1) & 1, bs, err)) goto done;
                 tc_fence_after();
                 __syncwarp();
-                const float uj = uu[r];
-                const float D_h = uu[2 * kTile];
+                const float uj = cs[3 * kTile + r];
+                const float D_h = cs[5 * kTile];
                 const float2 u2 = make_float2(uj, uj), d2 = make_float2(D_h, D_h);
                 const uint8_t* sx = smem + kOffX + xs * kAtom;
                 uint4* dst = reinterpret_cast<uint4*>(
@@ -704,8 +683,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     float yv[16], rv[16];
-                    tmem_ld16(tmem + lane_base + kColY + 32 * ph + 16 * hf, yv);
-                    tmem_ld16(tmem + lane_base + kColR + 32 * ph + 16 * hf, rv);
+                    tmem_ld16(tmem + lane_base + kColY + 64 * yb + 32 * ph + 16 * hf, yv);
+                    tmem_ld16(tmem + lane_base + kColR + 64 * yb + 32 * ph + 16 * hf, rv);
                     uint4 xq[2];
 #pragma unroll
                     for (int c = 0; c < 2; ++c)
@@ -713,13 +692,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld_wait();
                     if (hf == 1) {
                         tc_fence_before();
-                        mbar_arrive(&bs->ry_empty);
+                        mbar_arrive(&bs->ry_empty[yb]);
                         // generic-proxy reads of the x slot are done before the next
                         // TMA load into it
                         fence_proxy_async_smem();
                         mbar_arrive(&bs->x_empty[xs]);
                     }
-                    uint4 out[2];
 #pragma unroll
                     for (int c = 0; c < 2; ++c) {
                         const uint32_t xw[4] = {xq[c].x, xq[c].y, xq[c].z, xq[c].w};
@@ -731,11 +709,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                   make_float2(yv[i0], yv[i0 + 1]));
                             o[e2] = pack_bf16(fma2(d2, unpack_bf16(xw[e2]), t));
                         }
-                        out[c] = make_uint4(o[0], o[1], o[2], o[3]);
-                    }
-                    if (valid) {
-                        dst[2 * hf] = out[0];
-                        dst[2 * hf + 1] = out[1];
+                        if (valid) dst[2 * hf + c] = make_uint4(o[0], o[1], o[2], o[3]);
                     }
                 }
                 mbar_arrive(&bs->cs_empty[cb]);
@@ -744,17 +718,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             cur_ok = nx_ok;
             if (nx_ok) {
                 cur_b = nxU.b;
-                cur_h = nxU.hb * kh_n + nx_kh;
-                cur_t0 = nxU.tc0 + (int64_t)nx_s * kTile;
-                cur_last = nx_s + 1 >= nxU.nsub;
-                if (++nx_s >= nxU.nsub) {
-                    nx_s = 0;
-                    if (++nx_kh >= kh_n) {
-                        nx_kh = 0;
-                        nx_u += gridDim.x;
-                        nx_ok = nx_u < prm.nunits;
-                        if (nx_ok) nxU = decode(prm, nx_u);
-                    }
+                cur_h = nh;
+                cur_t0 = nxU.t0;
+                if (++nx_kh >= kh_n) {
+                    nx_kh = 0;
+                    nx_u += gridDim.x;
+                    nx_ok = nx_u < prm.nunits;
+                    if (nx_ok) nxU = decode(prm, nx_u);
                 }
             }
         }
@@ -791,13 +761,14 @@ cudaError_t launch_fused_ws(const Dims& d, const CUtensorMap* maps, const void* 
     prm.error = sync_ints + 1;
     prm.flags = sync_ints + 2;
     prm.T = d.T;
-    prm.H = d.H;
-    prm.G = d.G;
-    prm.nc = d.nc;
-    prm.Q = (int)d.Q;
+    prm.H = (int)d.H;
+    prm.G = (int)d.G;
     prm.kheads = kheads;
     prm.batch = (int)d.b;
-    prm.nunits = (int)(d.nc * d.b * (d.H / kheads));
+    const int64_t ntiles = (d.T + kTile - 1) / kTile;
+    const int64_t nunits = ntiles * d.b * (d.H / kheads);
+    if (nunits > INT32_MAX || d.T > INT32_MAX) return cudaErrorInvalidValue;
+    prm.nunits = (int)nunits;
     e = cudaFuncSetAttribute(ssd_fused_ws_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemBytes);
     if (e != cudaSuccess) return e;
