@@ -143,6 +143,20 @@ SSD_API ssd_status_t ssd_fwd_no_alloc(const ssd_shape_t* shape,
                                       const float* initial_states,
                                       void* y, float* final_states, void* stream);
 
+/*
+ * Device-side status of the last ssd_fwd that ran with `workspace` (same shape
+ * and workspace as that call). Waits for `stream`, so call it after the outputs
+ * are needed anyway. Returns SSD_OK, or SSD_ERR_TIMEOUT when a bounded wait
+ * inside the fused kernel gave up (about 2 s: a chain hand-off or a hand-off
+ * between the kernel's warp roles that never completed); that kernel then left
+ * its outputs incomplete but the CUDA context usable, and ssd_last_error_detail()
+ * names the wait. The step paths have no device-side waits and always report
+ * SSD_OK. There is no counterpart in the pages; it exists because the fused
+ * kernel's waits are bounded instead of hanging the GPU.
+ */
+SSD_API ssd_status_t ssd_fwd_check(const ssd_shape_t* shape, const void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
 /* Bytes of device workspace ssd_fwd_host needs (inputs, outputs and ssd_fwd's
  * own workspace are staged there). */
 SSD_API ssd_status_t ssd_fwd_host_workspace_size(const ssd_shape_t* shape, size_t* bytes);
@@ -153,7 +167,8 @@ SSD_API ssd_status_t ssd_fwd_host_workspace_size(const ssd_shape_t* shape, size_
  * non-NULL) back, and synchronizes `stream` before returning, so the host
  * outputs are ready on return. Host buffers should be page-locked for full
  * copy bandwidth; pageable memory works but is slower. The device workspace
- * must hold ssd_fwd_host_workspace_size() bytes.
+ * must hold ssd_fwd_host_workspace_size() bytes. Returns SSD_ERR_TIMEOUT (as
+ * ssd_fwd_check) when the fused kernel's bounded waits gave up.
  */
 SSD_API ssd_status_t ssd_fwd_host(const ssd_shape_t* shape,
                           const void* x, const float* dt, const float* A,

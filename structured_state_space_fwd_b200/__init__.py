@@ -22,7 +22,8 @@ import torch
 from ._lib import (SSD_BF16, SSD_F32, SSDError, ShapeT, check, lib, lib_path,  # noqa: F401
                    status_string)
 
-__all__ = ["ssd_fwd", "ssd_fwd_host", "ssd_fwd_workspace_size", "ssd_fwd_plan", "ssd_chunk_cumsum",
+__all__ = ["ssd_fwd", "ssd_fwd_host", "ssd_fwd_workspace_size", "ssd_fwd_plan", "ssd_fwd_check",
+           "ssd_chunk_cumsum",
            "ssd_chunk_state", "ssd_state_passing", "ssd_chunk_scan", "SSDError", "make_shape",
            "lib_path"]
 
@@ -99,6 +100,14 @@ def ssd_fwd(x, dt, A, B, C, D=None, chunk_size: int = 256, initial_states=None,
                         _p(initial_states), _p(y), _p(final_states), _p(workspace),
                         ctypes.c_size_t(nbytes), _stream(stream)), "ssd_fwd")
     return (y, final_states) if return_final_states else y
+
+
+def ssd_fwd_check(shape: ShapeT, workspace, stream=None):
+    """Device-side status of the last ssd_fwd on `workspace` (waits for the stream);
+    raises SSDError with SSD_ERR_TIMEOUT when the fused kernel's bounded waits gave up."""
+    nbytes = ssd_fwd_workspace_size(shape)
+    check(lib().ssd_fwd_check(ctypes.byref(shape), _p(workspace), ctypes.c_size_t(nbytes),
+                              _stream(stream)), "ssd_fwd_check")
 
 
 def ssd_fwd_host(x, dt, A, B, C, D=None, chunk_size: int = 256, initial_states=None,

@@ -203,6 +203,27 @@ ssd_status_t run_fwd(const ssd::Dims& d, const void* x, const float* dt, const f
                           : ssd::launch_chunk_scan_simt(d, x, dt, B, C, D, cs, entry, y, stream));
 }
 
+// The fused kernel's device status word (sync ints [1]) of the launch that last
+// used this workspace: waits for `s`, then maps a nonzero word to SSD_ERR_TIMEOUT.
+ssd_status_t read_device_status(const ssd::Dims& d, const void* workspace, cudaStream_t s) {
+    const FwdWorkspace w = fwd_workspace(d);
+    if (w.path != Path::Fused || w.total == 0 || d.b == 0 || d.T == 0) return SSD_OK;
+    int word = 0;
+    ssd_status_t st;
+    const int* dev = (const int*)((const char*)workspace + w.off_sync) + 1;
+    if ((st = cuda_status("status read", cudaMemcpyAsync(&word, dev, sizeof(int),
+                                                         cudaMemcpyDeviceToHost, s))) != SSD_OK)
+        return st;
+    if ((st = cuda_status("stream synchronize", cudaStreamSynchronize(s))) != SSD_OK) return st;
+    if (word == 0) return SSD_OK;
+    snprintf(g_detail, sizeof(g_detail), "%s",
+             word == 1   ? "fused kernel: a tile's entering state was not handed on in time (chain flag wait)"
+             : word == 3 ? "fused kernel: an mbarrier wait between warp roles timed out"
+             : word == 4 ? "fused kernel: shared memory base not 1024-byte aligned"
+                         : "fused kernel: device error");
+    return SSD_ERR_TIMEOUT;
+}
+
 }  // namespace
 
 void ssd::set_error_detail(const char* msg) { snprintf(g_detail, sizeof(g_detail), "%s", msg); }
@@ -320,7 +341,18 @@ ssd_status_t ssd_fwd_host(const ssd_shape_t* shape, const void* x, const float* 
         (st = cuda_status("device to host copy",
                           cudaMemcpyAsync(final_states, dfinal, z.st, cudaMemcpyDeviceToHost, s))) != SSD_OK)
         return st;
-    return cuda_status("stream synchronize", cudaStreamSynchronize(s));
+    if ((st = cuda_status("stream synchronize", cudaStreamSynchronize(s))) != SSD_OK) return st;
+    return read_device_status(d, base, s);
+}
+
+ssd_status_t ssd_fwd_check(const ssd_shape_t* shape, const void* workspace, size_t workspace_bytes,
+                           void* stream) {
+    ssd_status_t st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    const ssd::Dims d = ssd::make_dims(*shape);
+    const FwdWorkspace w = fwd_workspace(d);
+    if (workspace_bytes < w.total || (w.total > 0 && !workspace)) return SSD_ERR_INVALID_ARG;
+    return read_device_status(d, workspace, (cudaStream_t)stream);
 }
 
 ssd_status_t ssd_chunk_cumsum(const ssd_shape_t* shape, const float* dt, const float* A,

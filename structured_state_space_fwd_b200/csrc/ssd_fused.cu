@@ -28,6 +28,8 @@
 //
 // Every wait is bounded; a wait that gives up sets the error word and makes
 // every role leave its loop, after which the CTA drains its MMAs and exits.
+#include <cstdlib>
+
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -83,6 +85,7 @@ struct Params {
     int* error;
     int64_t T;
     int H, G, kheads, batch, nunits;
+    int stall;   // test hook: chain flags are awaited at a value never reached
 };
 
 struct Bars {
@@ -128,6 +131,9 @@ __device__ __forceinline__ uint64_t global_ns() {
     return t;
 }
 
+#ifndef SSD_IDLE_SLEEP_NS
+#define SSD_IDLE_SLEEP_NS 100
+#endif
 // A suspend-time hint on try_wait measured slower here (the woken thread
 // resumes later than a spinning one notices), so waits spin by default.
 #ifndef SSD_WAIT_HINT_NS
@@ -158,6 +164,32 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Bars* b
         }
     }
 }
+
+// Same for roles that run ahead of their consumers (TMA producer, cumsum warp,
+// chain publisher): between polls the thread sleeps, so that its warp leaves the
+// issue slots of its scheduler to the compute warps that share it.
+__device__ __forceinline__ bool wait_bar_idle(uint64_t* bar, uint32_t parity, Bars* bs, int* err) {
+    if (try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 1;; ++i) {
+        __nanosleep(SSD_IDLE_SLEEP_NS);
+        if (try_wait(bar, parity)) return true;
+        if ((i & 15) == 0) {
+            if (*(volatile int*)&bs->abort) return false;
+            if (global_ns() - t0 > 2000000000ull) {
+                *(volatile int*)&bs->abort = 1;
+                atomicExch(err, 3);
+                return false;
+            }
+        }
+    }
+}
+
+#ifdef SSD_MMA_IDLE
+#define MMA_WAIT wait_bar_idle
+#else
+#define MMA_WAIT wait_bar
+#endif
 
 // Same, called by all 32 lanes of a warp together: the outcome is made
 // warp-uniform so that no lane leaves a loop its warp-mates stay in (the
@@ -256,13 +288,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            int n = 0, m = 0;
-            for (int u = blockIdx.x; u < prm.nunits; u += gridDim.x, ++m) {
+            int n = 0, m = 0;    // x tiles and B/C tiles issued
+            for (int u = blockIdx.x; u < prm.nunits; u += gridDim.x) {
                 const Unit U = decode(prm, u);
                 const int g = U.hb * kh_n / (H / prm.G);
                 // B and C of the tile, shared by every head of the unit
                 const int sl = m & 1;
-                if (!wait_bar(&bs->bc_empty[sl], ((m >> 1) & 1) ^ 1, bs, err)) goto done;
+                if (!wait_bar_idle(&bs->bc_empty[sl], ((m >> 1) & 1) ^ 1, bs, err)) goto pdrain;
                 mbar_arrive_expect_tx(&bs->bc_full[sl], kBCSlot);
                 uint8_t* base = smem + kOffBC + sl * kBCSlot;
                 for (int a = 0; a < kN / 64; ++a) {
@@ -270,14 +302,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_load_4d(base + kBCSlot / 2 + a * kAtom, &tm_C, &bs->bc_full[sl], a * 64, g,
                                 (int)U.t0, U.b);
                 }
-                for (int kh = 0; kh < kh_n; ++kh, ++n) {
+                ++m;
+                for (int kh = 0; kh < kh_n; ++kh) {
                     const int xs = n % kXStages;
-                    if (!wait_bar(&bs->x_empty[xs], ((n / kXStages) & 1) ^ 1, bs, err)) goto done;
+                    if (!wait_bar_idle(&bs->x_empty[xs], ((n / kXStages) & 1) ^ 1, bs, err)) goto pdrain;
                     mbar_arrive_expect_tx(&bs->x_full[xs], kAtom);
                     tma_load_4d(smem + kOffX + xs * kAtom, &tm_x, &bs->x_full[xs], 0,
                                 U.hb * kh_n + kh, (int)U.t0, U.b);
+                    ++n;
                 }
             }
+        pdrain:
+            // No TMA load may still be writing shared memory when the CTA exits: wait for
+            // the last load issued into each slot (already complete unless a role aborted).
+            for (int i = 0; i < kXStages && i < n; ++i)
+                mbar_wait(&bs->x_full[i], ((n - 1 - i) / kXStages) & 1, 1u << 22);
+            for (int i = 0; i < 2 && i < m; ++i) mbar_wait(&bs->bc_full[i], ((m - 1 - i) / 2) & 1, 1u << 22);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -291,8 +331,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // heads; its slot is free once the mask group has used the previous G
             auto issue_g = [&](int m) -> bool {
                 const int sl = m & 1;
-                if (!wait_bar(&bs->bc_full[sl], (m >> 1) & 1, bs, err)) return false;
-                if (!wait_bar(&bs->g_empty, (m & 1) ^ 1, bs, err)) return false;
+                if (!MMA_WAIT(&bs->bc_full[sl], (m >> 1) & 1, bs, err)) return false;
+                if (!MMA_WAIT(&bs->g_empty, (m & 1) ^ 1, bs, err)) return false;
                 tc_fence_after();
                 const uint32_t gB = smem_u32(smem + kOffBC + sl * kBCSlot);
                 const uint64_t dGA = sw128_desc(gB + kBCSlot / 2, 16, 1024);
@@ -318,8 +358,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int yb = n & 1, xs = n % kXStages;
                     // S += B^T (w o x) onto the preloaded exp(cs_last) h: the head's state
                     // after the tile, which the state group waits on first
-                    if (!wait_bar(&bs->wx_full, pn, bs, err)) goto drain;
-                    if (!wait_bar(&bs->h_full, pn, bs, err)) goto drain;
+                    if (!MMA_WAIT(&bs->wx_full, pn, bs, err)) goto drain;
+                    if (!MMA_WAIT(&bs->h_full, pn, bs, err)) goto drain;
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < kTile / 16; ++kk) {
@@ -329,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mma_commit(&bs->wx_empty);
                     mma_commit(&bs->s_full);
                     // R = C h^T into buffer yb (free once item n-2's epilogue drained it)
-                    if (!wait_bar(&bs->ry_empty[yb], ((n >> 1) & 1) ^ 1, bs, err)) goto drain;
+                    if (!MMA_WAIT(&bs->ry_empty[yb], ((n >> 1) & 1) ^ 1, bs, err)) goto drain;
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < kN / 16; ++kk) {
@@ -339,8 +379,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     mma_commit(&bs->h_empty);
                     // Y = P x (P straight from TMEM)
-                    if (!wait_bar(&bs->p_full, pn, bs, err)) goto drain;
-                    if (!wait_bar(&bs->x_full[xs], (n / kXStages) & 1, bs, err)) goto drain;
+                    if (!MMA_WAIT(&bs->p_full, pn, bs, err)) goto drain;
+                    if (!MMA_WAIT(&bs->x_full[xs], (n / kXStages) & 1, bs, err)) goto drain;
                     tc_fence_after();
                     const uint64_t dXB = sw128_desc(smem_u32(smem + kOffX + xs * kAtom), kAtom, 1024);
 #pragma unroll
@@ -371,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float a2 = prm.A[h] * kLog2e;
                 const float d_h = prm.D ? prm.D[h] : 0.f;
                 const int cb = n % kCsStages;
-                if (!wait_bar_all(&bs->cs_empty[cb], ((n / kCsStages) & 1) ^ 1, bs, err)) goto done;
+                if (!__all_sync(0xffffffffu, wait_bar_idle(&bs->cs_empty[cb], ((n / kCsStages) & 1) ^ 1, bs, err))) goto done;
                 float dtv[4], v[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -381,12 +421,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // The state entering tile t of (b, h) is tile t-1's: wait for its flag here,
                 // ahead of the consumers (cs_full, arrived after this acquire, orders the
                 // state group's loads of that state after it).
+                int bad = 0;
                 if (U.t > 0 && lane == 0) {
                     const int* f = prm.flags + (int64_t)U.b * H + h;
                     bool ok = false;
                     const uint64_t t0 = global_ns();
                     for (uint32_t it = 0;; ++it) {
-                        if (ld_acquire(f) >= U.t) { ok = true; break; }
+                        if (ld_acquire(f) >= U.t + (prm.stall ? (1 << 30) : 0)) { ok = true; break; }
                         if (it >= 4) __nanosleep(64);
                         if ((it & 15) == 15 &&
                             (*(volatile int*)&bs->abort || global_ns() - t0 > 2000000000ull))
@@ -395,8 +436,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!ok) {
                         *(volatile int*)&bs->abort = 1;
                         atomicExch(err, 1);
+                        bad = 1;
                     }
                 }
+                if (__any_sync(0xffffffffu, bad)) goto done;
                 __syncwarp();
                 float run = 0.f;
 #pragma unroll
@@ -451,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const Unit U = decode(prm, u);
                 for (int kh = 0; kh < kh_n; ++kh, ++np) {
                     const int ps = np % kPubStages;
-                    if (!wait_bar(&bs->pub_full[ps], (np / kPubStages) & 1, bs, err)) goto done;
+                    if (!wait_bar_idle(&bs->pub_full[ps], (np / kPubStages) & 1, bs, err)) goto done;
                     __threadfence();
                     st_release(prm.flags + (int64_t)U.b * H + U.hb * kh_n + kh, U.t + 1);
                     mbar_arrive(&bs->pub_empty[ps]);
@@ -769,6 +812,10 @@ cudaError_t launch_fused_ws(const Dims& d, const CUtensorMap* maps, const void* 
     const int64_t nunits = ntiles * d.b * (d.H / kheads);
     if (nunits > INT32_MAX || d.T > INT32_MAX) return cudaErrorInvalidValue;
     prm.nunits = (int)nunits;
+    // SSD_TEST_STALL_CHAIN=1 makes every chain hand-off wait run out (about 2 s), so
+    // that tests can check the device status path without faulting the GPU
+    const char* stall = getenv("SSD_TEST_STALL_CHAIN");
+    prm.stall = (stall && stall[0] == '1') ? 1 : 0;
     e = cudaFuncSetAttribute(ssd_fused_ws_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemBytes);
     if (e != cudaSuccess) return e;
