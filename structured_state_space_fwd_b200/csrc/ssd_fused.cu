@@ -57,7 +57,7 @@ constexpr uint32_t kOffX = kOffBC + 2 * kBCSlot;    // kXStages x 16 KB
 constexpr uint32_t kOffWX = kOffX + kXStages * kAtom;
 constexpr uint32_t kOffH = kOffWX + kAtom;
 constexpr uint32_t kOffCs = kOffH + kN * 128;    // kCsStages slots
-constexpr uint32_t kCsSlot = 6 * kTile * 4;   // cs, dt, w, u, v (per token), then D_h
+constexpr uint32_t kCsSlot = 7 * kTile * 4;   // cs, dt, w, u, v, u' (per token), then D_h, unit flag
 constexpr uint32_t kOffBar = kOffCs + kCsStages * kCsSlot;
 constexpr uint32_t kSmemBytes = kOffBar + 512;
 
@@ -72,6 +72,11 @@ constexpr float kLog2e = 1.4426950408889634f;
 // product is formed as exp2(cs_j - cs_e) * exp2(cs_e - cs_i): both factors then
 // stay within 2^+-64, far from fp32 overflow for any finite G.
 constexpr float kFactorRangeLog2 = 64.f;
+// Widest decay over one tile (log2 units) for which the tile's masked product is
+// formed head-independently, Y' = tril(C B^T) (w o x) with y = exp2(cs - cs_last) Y':
+// both exp2(cs_last - cs) dt (in w o x, bf16) and its inverse stay inside the
+// normal fp32/bf16 exponent range with a wide margin.
+constexpr float kSharedMaskRangeLog2 = 96.f;
 
 struct Params {
     const __nv_bfloat16* x;
@@ -346,13 +351,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_commit(&bs->g_full);
                 return true;
             };
-            int n = 0, m = 0;
+            int n = 0, m = 0, pph = 0;
             if (blockIdx.x < prm.nunits && !issue_g(0)) goto drain;
             for (int u = blockIdx.x; u < prm.nunits; u += gridDim.x, ++m) {
                 const int sl = m & 1;
                 const uint32_t aB = smem_u32(smem + kOffBC + sl * kBCSlot);
                 const uint64_t dSA = sw128_desc(aB, kAtom, 1024);
                 const uint64_t dRA = sw128_desc(aB + kBCSlot / 2, 16, 1024);
+                // one head-independent masked product for the whole unit, or one per head
+                if (!MMA_WAIT(&bs->cs_full[n % kCsStages], (n / kCsStages) & 1, bs, err)) goto drain;
+                const bool shared =
+                    reinterpret_cast<const float*>(smem + kOffCs + (n % kCsStages) * kCsSlot)[6 * kTile + 1] != 0.f;
                 for (int kh = 0; kh < kh_n; ++kh, ++n) {
                     const uint32_t pn = n & 1;
                     const int yb = n & 1, xs = n % kXStages;
@@ -366,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint64_t rows = (uint64_t)(kk * (2048 >> 4));   // 16 rows of 128 B
                         mma_bf16(tmem + kColS, dSA + rows, dSB + rows, idS, 1u);
                     }
-                    mma_commit(&bs->wx_empty);
+                    if (!shared) mma_commit(&bs->wx_empty);
                     mma_commit(&bs->s_full);
                     // R = C h^T into buffer yb (free once item n-2's epilogue drained it)
                     if (!MMA_WAIT(&bs->ry_empty[yb], ((n >> 1) & 1) ^ 1, bs, err)) goto drain;
@@ -378,16 +387,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_bf16(tmem + kColR + 64 * yb, dRA + kofs, dRB + rows, idY, kk > 0);
                     }
                     mma_commit(&bs->h_empty);
-                    // Y = P x (P straight from TMEM)
-                    if (!MMA_WAIT(&bs->p_full, pn, bs, err)) goto drain;
-                    if (!MMA_WAIT(&bs->x_full[xs], (n / kXStages) & 1, bs, err)) goto drain;
+                    // Y = P x, or Y' = P' (w o x) with the unit's shared P' (P straight from TMEM)
+                    if (!shared || kh == 0) {
+                        if (!MMA_WAIT(&bs->p_full, pph & 1, bs, err)) goto drain;
+                    }
+                    if (!shared && !MMA_WAIT(&bs->x_full[xs], (n / kXStages) & 1, bs, err)) goto drain;
                     tc_fence_after();
-                    const uint64_t dXB = sw128_desc(smem_u32(smem + kOffX + xs * kAtom), kAtom, 1024);
+                    const uint64_t dXB =
+                        shared ? dSB : sw128_desc(smem_u32(smem + kOffX + xs * kAtom), kAtom, 1024);
 #pragma unroll
                     for (int kk = 0; kk < kTile / 16; ++kk)
                         mma_bf16_tmem_a(tmem + kColY + 64 * yb, tmem + kColP + 8 * kk,
                                         dXB + (uint64_t)(kk * (2048 >> 4)), idY, kk > 0);
-                    mma_commit(&bs->p_empty);
+                    if (!shared || kh == kh_n - 1) {
+                        mma_commit(&bs->p_empty);
+                        ++pph;
+                    }
+                    if (shared) mma_commit(&bs->wx_empty);
                     mma_commit(&bs->x_empty[xs]);
                     mma_commit(&bs->y_full[yb]);
                 }
@@ -406,6 +422,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int u = blockIdx.x; u < prm.nunits; u += gridDim.x) {
             const Unit U = decode(prm, u);
             const int len = (int)min((int64_t)kTile, T - U.t0);
+            // Does every head of the unit decay by at most kSharedMaskRangeLog2 over this
+            // tile? Then the unit shares one head-independent masked product.
+            float worst = 0.f;
+            for (int k2 = 0; k2 < kh_n; ++k2) {
+                const int h2 = U.hb * kh_n + k2;
+                float sdt = 0.f;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int t = lane * 4 + e;
+                    sdt += t < len ? __ldg(prm.dt + ((int64_t)U.b * T + U.t0 + t) * H + h2) : 0.f;
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) sdt += __shfl_xor_sync(0xffffffffu, sdt, off);
+                worst = fmaxf(worst, sdt * fabsf(prm.A[h2]) * kLog2e);
+            }
+            const float unit_shared = worst <= kSharedMaskRangeLog2 ? 1.f : 0.f;
             for (int kh = 0; kh < kh_n; ++kh, ++n) {
                 const int h = U.hb * kh_n + kh;
                 const float a2 = prm.A[h] * kLog2e;
@@ -458,12 +490,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float* cs = reinterpret_cast<float*>(smem + kOffCs + cb * kCsSlot);
                 // cs at the last row of this lane's 32-column block (lanes 8b..8b+7 hold block b)
                 const float cref = __shfl_sync(0xffffffffu, incl, (lane | 7));
-                float4 c4, d4, w4, u4, v4;
+                float4 c4, d4, w4, u4, v4, q4;
                 float* cp = &c4.x;
                 float* dp = &d4.x;
                 float* wp = &w4.x;
                 float* up = &u4.x;
                 float* vp = &v4.x;
+                float* qp = &q4.x;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float ce = excl + v[e];
@@ -472,13 +505,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     wp[e] = exp2f(last - ce) * dtv[e];
                     up[e] = exp2f(ce);
                     vp[e] = exp2f(cref - ce) * dtv[e];
+                    qp[e] = exp2f(ce - last);
                 }
                 reinterpret_cast<float4*>(cs)[lane] = c4;
                 reinterpret_cast<float4*>(cs + kTile)[lane] = d4;
                 reinterpret_cast<float4*>(cs + 2 * kTile)[lane] = w4;
                 reinterpret_cast<float4*>(cs + 3 * kTile)[lane] = u4;
                 reinterpret_cast<float4*>(cs + 4 * kTile)[lane] = v4;
-                if (lane == 0) cs[5 * kTile] = d_h;
+                reinterpret_cast<float4*>(cs + 5 * kTile)[lane] = q4;
+                if (lane == 0) {
+                    cs[6 * kTile] = d_h;
+                    cs[6 * kTile + 1] = unit_shared;
+                }
                 __syncwarp();
                 mbar_arrive(&bs->cs_full[cb]);
             }
@@ -503,14 +541,51 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp >= 4 && warp < 8) {
         // ------------------------------------------------------------ mask group
-        // per item: w o x (the S product's operand), then P = G o L
+        // Per unit: when every head's decay over the tile is within range, one
+        // head-independent P' = tril(G) (bf16) serves all the unit's heads (their decay
+        // goes into w o x and the epilogue); otherwise, per item, P = G o L of the head.
+        // Per item: w o x (the S product's operand, and Y's with P').
         const int wq = warp - 4;
         const int j = tid - 128;  // row of the tile == TMEM lane
         const int jj = j & 31;    // row within this warp's diagonal block
         const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
-        int n = 0, m = 0;
+        int n = 0, m = 0, pph = 0;
         for (int u = blockIdx.x; u < prm.nunits; u += gridDim.x, ++m) {
             if (!wait_bar_all(&bs->g_full, m & 1, bs, err)) goto done;
+            if (!wait_bar_all(&bs->cs_full[n % kCsStages], (n / kCsStages) & 1, bs, err)) goto done;
+            const bool shared =
+                reinterpret_cast<const float*>(smem + kOffCs + (n % kCsStages) * kCsSlot)[6 * kTile + 1] != 0.f;
+            if (shared) {
+                if (!wait_bar_all(&bs->p_empty, (pph & 1) ^ 1, bs, err)) goto done;
+                tc_fence_after();
+                __syncwarp();
+#pragma unroll 1
+                for (int blk = 0; blk < 4; ++blk) {
+                    uint32_t pk[16];
+                    if (blk > wq) {
+#pragma unroll
+                        for (int q = 0; q < 16; ++q) pk[q] = 0u;
+                    } else {
+                        float gv[32];
+                        tmem_ld32(tmem + lane_base + kColG + 32 * blk, gv);
+                        tmem_ld_wait_regs(gv);
+                        if (blk < wq) {
+#pragma unroll
+                            for (int q = 0; q < 16; ++q) pk[q] = pack_bf16(gv[2 * q], gv[2 * q + 1]);
+                        } else {
+#pragma unroll
+                            for (int q = 0; q < 16; ++q)   // causal mask: column i kept while i <= row
+                                pk[q] = pack_bf16(2 * q <= jj ? gv[2 * q] : 0.f, 2 * q + 1 <= jj ? gv[2 * q + 1] : 0.f);
+                        }
+                    }
+                    tmem_st16(tmem + lane_base + kColP + 16 * blk, pk);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(&bs->p_full);
+                ++pph;
+                mbar_arrive(&bs->g_empty);
+            }
             for (int kh = 0; kh < kh_n; ++kh, ++n) {
                 const int cb = n % kCsStages;
                 if (!wait_bar_all(&bs->cs_full[cb], (n / kCsStages) & 1, bs, err)) goto done;
@@ -539,7 +614,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive(&bs->wx_full);
                     mbar_arrive(&bs->x_empty[xs]);
                 }
-                if (!wait_bar_all(&bs->p_empty, (n & 1) ^ 1, bs, err)) goto done;
+                if (shared) {
+                    mbar_arrive(&bs->cs_empty[cb]);
+                    continue;
+                }
+                if (!wait_bar_all(&bs->p_empty, (pph & 1) ^ 1, bs, err)) goto done;
                 tc_fence_after();
                 __syncwarp();
                 const float csj = cs[j];
@@ -611,6 +690,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(&bs->p_full);
+                ++pph;
                 if (kh == kh_n - 1) mbar_arrive(&bs->g_empty);
                 mbar_arrive(&bs->cs_empty[cb]);
             }
@@ -717,8 +797,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 __syncwarp();
                 const float uj = cs[3 * kTile + r];
-                const float D_h = cs[5 * kTile];
-                const float2 u2 = make_float2(uj, uj), d2 = make_float2(D_h, D_h);
+                const float D_h = cs[6 * kTile];
+                // shared-mask units produced Y' = tril(C B^T) (w o x): row r scales by
+                // exp2(cs_r - cs_last)
+                const float qj = cs[6 * kTile + 1] != 0.f ? cs[5 * kTile + r] : 1.f;
+                const float2 u2 = make_float2(uj, uj), d2 = make_float2(D_h, D_h), q2 = make_float2(qj, qj);
                 const uint8_t* sx = smem + kOffX + xs * kAtom;
                 uint4* dst = reinterpret_cast<uint4*>(
                     prm.y + (((int64_t)cur_b * T + cur_t0 + r) * H + cur_h) * kP + 32 * ph);
@@ -749,7 +832,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int e2 = 0; e2 < 4; ++e2) {
                             const int i0 = 8 * c + 2 * e2;
                             const float2 t = fma2(u2, make_float2(rv[i0], rv[i0 + 1]),
-                                                  make_float2(yv[i0], yv[i0 + 1]));
+                                                  mul2(q2, make_float2(yv[i0], yv[i0 + 1])));
                             o[e2] = pack_bf16(fma2(d2, unpack_bf16(xw[e2]), t));
                         }
                         if (valid) dst[2 * hf + c] = make_uint4(o[0], o[1], o[2], o[3]);
