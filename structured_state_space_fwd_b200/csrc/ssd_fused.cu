@@ -103,6 +103,7 @@ struct Bars {
     uint64_t h_full, h_empty;     // state operand and S preload written / operand read
     uint64_t s_full;              // S complete: the head's state after the tile
     uint64_t y_full[2], ry_empty[2];
+    uint64_t y_staged[8];         // a lane quarter's y rows written (warp 12+q to 8+q), per item parity
     uint64_t pub_full[kPubStages], pub_empty[kPubStages];  // state stored / flag released
     uint64_t fin;
     uint32_t tmem;
@@ -246,12 +247,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bs->y_full[i], 1);
             mbar_init(&bs->ry_empty[i], 256);
         }
+        for (int i = 0; i < 8; ++i) mbar_init(&bs->y_staged[i], 32);
         mbar_init(&bs->g_full, 1);
         mbar_init(&bs->g_empty, 128);
         for (int i = 0; i < kXStages; ++i) {
             mbar_init(&bs->x_full[i], 1);
-            // Y product (commit) + mask group (w o x) + state group (skip term D x)
-            mbar_init(&bs->x_empty[i], 1 + 128 + 256);
+            // Y product (commit) + mask group (w o x) + the 4 lanes that store y from it
+            mbar_init(&bs->x_empty[i], 1 + 128 + 4);
         }
         for (int i = 0; i < kCsStages; ++i) {
             mbar_init(&bs->cs_full[i], 32);
@@ -713,6 +715,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // units per tile than CTAs); otherwise it waits for the hand-off.
         const bool early_ok = prm.batch * (H / kh_n) > (int)gridDim.x;
         int npub = 0;
+        int ystore_xs = -1;   // x slot of this quarter's last y store (issuing lanes)
         float hn[32];    // h[32 ph + i][r] entering the next item's tile
         // the state of head h entering tile U.t (item `item`); returns false on abort.
         // Tile t-1's flag was acquired by the cumsum warp before it released the item's
@@ -789,7 +792,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(&bs->h_full);
             }
             // 4. y of item n from R and Y (this warp's 32 columns):
-            // y_j = Y_j + exp(cs_j) R_j + D x_j, this thread's bytes of row r
+            // y_j = Y_j + exp(cs_j) R_j + D x_j, this thread's bytes of row r, written over
+            // the same bytes of the item's x tile; each lane quarter's 32 rows then go
+            // out as one TMA store
             if (cur_ok) {
                 const int yb = n & 1, xs = n % kXStages, cb = n % kCsStages;
                 const float* cs = reinterpret_cast<const float*>(smem + kOffCs + cb * kCsSlot);
@@ -802,10 +807,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // exp2(cs_r - cs_last)
                 const float qj = cs[6 * kTile + 1] != 0.f ? cs[5 * kTile + r] : 1.f;
                 const float2 u2 = make_float2(uj, uj), d2 = make_float2(D_h, D_h), q2 = make_float2(qj, qj);
-                const uint8_t* sx = smem + kOffX + xs * kAtom;
-                uint4* dst = reinterpret_cast<uint4*>(
-                    prm.y + (((int64_t)cur_b * T + cur_t0 + r) * H + cur_h) * kP + 32 * ph);
-                const bool valid = cur_t0 + r < T;
+                uint8_t* sx = smem + kOffX + xs * kAtom;
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     float yv[16], rv[16];
@@ -816,13 +818,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int c = 0; c < 2; ++c)
                         xq[c] = *reinterpret_cast<const uint4*>(sx + sw128_off(r, 4 * ph + 2 * hf + c));
                     tmem_ld_wait();
-                    if (hf == 1) {
+                    if (hf == 1 && ph == 1) {
                         tc_fence_before();
                         mbar_arrive(&bs->ry_empty[yb]);
-                        // generic-proxy reads of the x slot are done before the next
-                        // TMA load into it
-                        fence_proxy_async_smem();
-                        mbar_arrive(&bs->x_empty[xs]);
                     }
 #pragma unroll
                     for (int c = 0; c < 2; ++c) {
@@ -835,8 +833,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                   mul2(q2, make_float2(yv[i0], yv[i0 + 1])));
                             o[e2] = pack_bf16(fma2(d2, unpack_bf16(xw[e2]), t));
                         }
-                        if (valid) dst[2 * hf + c] = make_uint4(o[0], o[1], o[2], o[3]);
+                        *reinterpret_cast<uint4*>(sx + sw128_off(r, 4 * ph + 2 * hf + c)) =
+                            make_uint4(o[0], o[1], o[2], o[3]);
                     }
+                }
+                // y bytes visible to the async proxy, then the quarter's store: warp 12+q
+                // signals (one barrier per item parity), the first lane of warp 8+q issues
+                // once both halves are written. Warp 8+q releases R and Y only after that
+                // wait, so item n+2's products (and warp 12+q's next arrival on this
+                // parity's barrier) cannot come before it.
+                fence_proxy_async_smem();
+                if (ph == 1) {
+                    mbar_arrive(&bs->y_staged[2 * q + (n & 1)]);
+                } else {
+                    __syncwarp();
+                    int ok = 1;
+                    if (lane == 0) {
+                        ok = wait_bar(&bs->y_staged[2 * q + (n & 1)], (n >> 1) & 1, bs, err);
+                        if (ok) {
+                            // the previous store from this quarter has read its slot: release it
+                            if (ystore_xs >= 0) {
+                                bulk_wait_group_read0();
+                                mbar_arrive(&bs->x_empty[ystore_xs]);
+                                ystore_xs = -1;
+                            }
+                            if (cur_t0 + 32 * q < T) {   // rows past T are clipped by the store
+                                tma_store_4d(&tm_y, sx + q * (kAtom / 4), 0, cur_h, (int)(cur_t0 + 32 * q),
+                                             cur_b);
+                                bulk_commit_group();
+                                ystore_xs = xs;
+                            } else {
+                                mbar_arrive(&bs->x_empty[xs]);
+                            }
+                        }
+                    }
+                    if (!__shfl_sync(0xffffffffu, ok, 0)) goto done;
+                    tc_fence_before();
+                    mbar_arrive(&bs->ry_empty[yb]);
                 }
                 mbar_arrive(&bs->cs_empty[cb]);
             }
@@ -856,6 +889,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
 done:
+    // bulk stores still reading shared memory (y tiles) finish before the CTA exits
+    if (warp >= 8 && warp < 12 && lane == 0) bulk_wait_group0();
     tc_fence_before();
     __syncthreads();
     if (warp == 1) tmem_dealloc(tmem, 512);

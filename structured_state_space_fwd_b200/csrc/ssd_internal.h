@@ -46,7 +46,8 @@ cudaError_t launch_fused_tc(const Dims& d, const void* x, const float* dt, const
                             void* y, float* chain, int* sync_ints, cudaStream_t st);
 
 int pick_kheads(int64_t heads_per_group);
-// TMA maps of x, B, C, y (bf16, 4-D, 64 x 1 x 128 x 1 boxes, 128-byte swizzle).
+// TMA maps of x, B, C (bf16, 4-D, 64 x 1 x 128 x 1 boxes) and y (64 x 1 x 32 x 1 boxes),
+// 128-byte swizzle.
 bool make_tc_maps(const Dims& d, const void* x, const void* B, const void* C, const void* y,
                   CUtensorMap* maps);
 cudaError_t launch_fused_ws(const Dims& d, const CUtensorMap* maps, const void* x, const float* dt,

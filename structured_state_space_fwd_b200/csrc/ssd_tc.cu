@@ -473,12 +473,13 @@ EncodeTiledFn encode_fn() {
 }
 
 // 4-D bf16 map over [d3][d2][d1][d0] (d0 innermost), box {64, 1, 128, 1}, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3) {
+bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3,
+              uint32_t box_rows = kTile) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[4] = {d0, d1, d2, d3};
     const cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};
-    const cuuint32_t box[4] = {64, 1, kTile, 1};
+    const cuuint32_t box[4] = {64, 1, box_rows, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -497,7 +498,7 @@ bool make_tc_maps(const Dims& d, const void* x, const void* B, const void* C, co
                   CUtensorMap* maps) {
     return make_map(&maps[0], x, d.P, d.H, d.T, d.b) && make_map(&maps[1], B, d.N, d.G, d.T, d.b) &&
            make_map(&maps[2], C ? C : B, d.N, d.G, d.T, d.b) &&
-           make_map(&maps[3], y ? y : x, d.P, d.H, d.T, d.b);
+           make_map(&maps[3], y ? y : x, d.P, d.H, d.T, d.b, 32);
 }
 
 namespace {
