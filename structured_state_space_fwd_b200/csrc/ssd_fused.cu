@@ -155,8 +155,7 @@ __device__ __forceinline__ bool try_wait(uint64_t* bar, uint32_t parity) {
 
 // Bounded mbarrier wait (about 2 s) that also gives up once another role
 // aborted (checked every 16 polls).
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Bars* bs, int* err) {
-    if (try_wait(bar, parity)) return true;
+__device__ __noinline__ bool wait_bar_slow(uint64_t* bar, uint32_t parity, Bars* bs, int* err) {
     const uint64_t t0 = global_ns();
     for (uint32_t i = 1;; ++i) {
         if (try_wait(bar, parity)) return true;
@@ -170,12 +169,18 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Bars* b
         }
     }
 }
+// Fast path inline, the polling loop shared by every call site (one copy in the
+// instruction caches).
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Bars* bs, int* err) {
+    if (try_wait(bar, parity)) return true;
+    return wait_bar_slow(bar, parity, bs, err);
+}
+
 
 // Same for roles that run ahead of their consumers (TMA producer, cumsum warp,
 // chain publisher): between polls the thread sleeps, so that its warp leaves the
 // issue slots of its scheduler to the compute warps that share it.
-__device__ __forceinline__ bool wait_bar_idle(uint64_t* bar, uint32_t parity, Bars* bs, int* err) {
-    if (try_wait(bar, parity)) return true;
+__device__ __noinline__ bool wait_bar_idle_slow(uint64_t* bar, uint32_t parity, Bars* bs, int* err) {
     const uint64_t t0 = global_ns();
     for (uint32_t i = 1;; ++i) {
         __nanosleep(SSD_IDLE_SLEEP_NS);
@@ -190,6 +195,11 @@ __device__ __forceinline__ bool wait_bar_idle(uint64_t* bar, uint32_t parity, Ba
         }
     }
 }
+__device__ __forceinline__ bool wait_bar_idle(uint64_t* bar, uint32_t parity, Bars* bs, int* err) {
+    if (try_wait(bar, parity)) return true;
+    return wait_bar_idle_slow(bar, parity, bs, err);
+}
+
 
 #ifdef SSD_MMA_IDLE
 #define MMA_WAIT wait_bar_idle
@@ -213,6 +223,14 @@ __device__ __forceinline__ void write_h_half(uint8_t* sh, int n, int half, const
         *reinterpret_cast<uint4*>(sh + sw128_off(n, 4 * half + c)) =
             make_uint4(pack_bf16(hh[8 * c], hh[8 * c + 1]), pack_bf16(hh[8 * c + 2], hh[8 * c + 3]),
                        pack_bf16(hh[8 * c + 4], hh[8 * c + 5]), pack_bf16(hh[8 * c + 6], hh[8 * c + 7]));
+}
+
+// 2^x on the special-function unit (a few ulp; results below 2^-126 flush to
+// zero, i.e. decays too small to matter).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 struct Unit {
@@ -504,10 +522,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float ce = excl + v[e];
                     cp[e] = ce;
                     dp[e] = dtv[e];
-                    wp[e] = exp2f(last - ce) * dtv[e];
-                    up[e] = exp2f(ce);
-                    vp[e] = exp2f(cref - ce) * dtv[e];
-                    qp[e] = exp2f(ce - last);
+                    wp[e] = ex2(last - ce) * dtv[e];
+                    up[e] = ex2(ce);
+                    vp[e] = ex2(cref - ce) * dtv[e];
+                    qp[e] = ex2(ce - last);
                 }
                 reinterpret_cast<float4*>(cs)[lane] = c4;
                 reinterpret_cast<float4*>(cs + kTile)[lane] = d4;
@@ -639,7 +657,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         // bounded by the block's own cs range, which decides whether the
                         // factored form is safe in fp32 or the exponent is taken per element.
                         const float ce = cs[32 * blk + 31];
-                        const float a = exp2f(csj - ce);
+                        const float a = ex2(csj - ce);
                         const bool exact = blk == wq && cs[32 * blk] - ce > kFactorRangeLog2;
                         const float2 a2 = make_float2(a, a);
                         tmem_ld_wait();
@@ -674,10 +692,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 const float4 c4 = reinterpret_cast<const float4*>(cs)[blk * 8 + e4];
                                 const float4 d4 = reinterpret_cast<const float4*>(dts)[blk * 8 + e4];
                                 const int i0 = blk * 32 + e4 * 4;
-                                const float m0 = exp2f(csj - c4.x) * d4.x;
-                                const float m1 = exp2f(csj - c4.y) * d4.y;
-                                const float m2 = exp2f(csj - c4.z) * d4.z;
-                                const float m3 = exp2f(csj - c4.w) * d4.w;
+                                const float m0 = ex2(csj - c4.x) * d4.x;
+                                const float m1 = ex2(csj - c4.y) * d4.y;
+                                const float m2 = ex2(csj - c4.z) * d4.z;
+                                const float m3 = ex2(csj - c4.w) * d4.w;
                                 const float p0 = (i0 <= j) ? gv[e4 * 4] * m0 : 0.f;
                                 const float p1 = (i0 + 1 <= j) ? gv[e4 * 4 + 1] * m1 : 0.f;
                                 const float p2 = (i0 + 2 <= j) ? gv[e4 * 4 + 2] * m2 : 0.f;
@@ -808,7 +826,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float qj = cs[6 * kTile + 1] != 0.f ? cs[5 * kTile + r] : 1.f;
                 const float2 u2 = make_float2(uj, uj), d2 = make_float2(D_h, D_h), q2 = make_float2(qj, qj);
                 uint8_t* sx = smem + kOffX + xs * kAtom;
-#pragma unroll
+#pragma unroll 1
                 for (int hf = 0; hf < 2; ++hf) {
                     float yv[16], rv[16];
                     tmem_ld16(tmem + lane_base + kColY + 64 * yb + 32 * ph + 16 * hf, yv);
