@@ -248,7 +248,8 @@ def run_ours(args):
     import structured_state_space_fwd_b200 as ssd
 
     w = WORKLOAD
-    inp = W.workload_inputs(w, seed=0)
+    # each rank's shard: its own batch of the workload (seeded by rank)
+    inp = W.workload_inputs(w, seed=rank)
     d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
     b, T, H, P, G, N, Q = w.batch, w.seqlen, w.nheads, w.headdim, w.ngroups, w.dstate, w.chunk_size
     nc = -(-T // Q)

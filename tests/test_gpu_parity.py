@@ -292,6 +292,16 @@ def test_tensor_steps_against_oracle(ssd, path_env):
     assert oracle.rel_err(y.float().cpu(), y_ref) <= 5e-3
 
 
+def test_phase_sequential_fused_kernel(ssd, path_env, monkeypatch):
+    # The phase-sequential predecessor of the fused kernel (SSD_FUSED=v0), kept as
+    # an independent second single-pass implementation, against the oracle.
+    path_env("fused")
+    monkeypatch.setenv("SSD_FUSED", "v0")
+    inp = make_inputs(batch=2, seqlen=700, nheads=8, headdim=64, ngroups=2, dstate=128,
+                      dtype="bf16", initial_states=True, seed=41)
+    check_full(ssd, inp, 256, "bf16")
+
+
 def test_paths_agree(ssd, path_env):
     inp = make_inputs(batch=2, seqlen=900, nheads=4, headdim=64, ngroups=1, dstate=128,
                       dtype="bf16", initial_states=True, seed=33)
