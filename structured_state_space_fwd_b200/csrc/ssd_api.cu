@@ -224,6 +224,31 @@ ssd_status_t read_device_status(const ssd::Dims& d, const void* workspace, cudaS
     return SSD_ERR_TIMEOUT;
 }
 
+// ssd_fwd_host works through the batch in slices of rows so that the copies in,
+// the forward and the copies out of different slices overlap (the two copy
+// directions use separate copy engines). Each slice has its own forward
+// workspace, so every slice's device status word survives until it is read.
+struct HostPlan {
+    int64_t nslices, rows;     // slices of `rows` batch rows (the last may be shorter)
+    size_t ws_slice;           // forward workspace of one full slice
+};
+HostPlan host_plan(const ssd::Dims& d) {
+    HostPlan hp;
+    hp.nslices = d.b < 8 ? (d.b > 0 ? d.b : 1) : 8;
+    // slices start at row boundaries: keep the 16-byte alignment of every tensor
+    if (d.b > 0) {
+        const Sizes z = sizes_of(d);
+        for (size_t bytes : {z.x, z.dt, z.bc, z.st})
+            if ((bytes / d.b) % 16 != 0) hp.nslices = 1;
+    }
+    hp.rows = d.b > 0 ? (d.b + hp.nslices - 1) / hp.nslices : 0;
+    if (hp.rows > 0) hp.nslices = (d.b + hp.rows - 1) / hp.rows;
+    ssd::Dims ds = d;
+    ds.b = hp.rows;
+    hp.ws_slice = align_up(fwd_workspace(ds).total, 256);
+    return hp;
+}
+
 }  // namespace
 
 void ssd::set_error_detail(const char* msg) { snprintf(g_detail, sizeof(g_detail), "%s", msg); }
@@ -282,7 +307,8 @@ ssd_status_t ssd_fwd_host_workspace_size(const ssd_shape_t* shape, size_t* bytes
     if (st != SSD_OK) return st;
     const ssd::Dims d = ssd::make_dims(*shape);
     const Sizes z = sizes_of(d);
-    size_t tot = align_up(fwd_workspace(d).total, 256);
+    const HostPlan hp = host_plan(d);
+    size_t tot = (size_t)hp.nslices * hp.ws_slice;
     for (size_t s : {z.x, z.dt, z.hv, z.bc, z.bc, z.hv, z.st, z.x, z.st}) tot += align_up(s, 256);
     *bytes = tot;
     return SSD_OK;
@@ -305,44 +331,99 @@ ssd_status_t ssd_fwd_host(const ssd_shape_t* shape, const void* x, const float* 
     if (workspace_bytes < need) return SSD_ERR_INVALID_ARG;
     const ssd::Dims d = ssd::make_dims(*shape);
     const Sizes z = sizes_of(d);
+    const HostPlan hp = host_plan(d);
     cudaStream_t s = (cudaStream_t)stream;
     char* base = (char*)device_workspace;
-    size_t off = align_up(fwd_workspace(d).total, 256);
+    size_t off = (size_t)hp.nslices * hp.ws_slice;
     auto take = [&](size_t bytes) {
         char* p = base + off;
         off += align_up(bytes, 256);
         return p;
     };
-    void* dx = take(z.x);
-    float* ddt = (float*)take(z.dt);
+    char* dx = take(z.x);
+    char* ddt = take(z.dt);
     float* dA = (float*)take(z.hv);
-    void* dB = take(z.bc);
-    void* dC = take(z.bc);
+    char* dB = take(z.bc);
+    char* dC = take(z.bc);
     float* dD = (float*)take(z.hv);
-    float* dinit = (float*)take(z.st);
-    void* dy = take(z.x);
-    float* dfinal = (float*)take(z.st);
-    struct Cp { void* dst; const void* src; size_t n; };
-    const Cp h2d[] = {{dx, x, z.x}, {ddt, dt, z.dt}, {dA, A, z.hv}, {dB, B, z.bc}, {dC, C, z.bc},
-                      {dD, D, D ? z.hv : 0}, {dinit, initial_states, initial_states ? z.st : 0}};
-    for (const Cp& c : h2d) {
-        if (c.n == 0) continue;
-        if ((st = cuda_status("host to device copy",
-                              cudaMemcpyAsync(c.dst, c.src, c.n, cudaMemcpyHostToDevice, s))) != SSD_OK)
-            return st;
+    char* dinit = take(z.st);
+    char* dy = take(z.x);
+    char* dfinal = take(z.st);
+    if (d.b == 0) return SSD_OK;
+    // bytes of one batch row of each batch-major tensor
+    const size_t rx = z.x / d.b, rdt = z.dt / d.b, rbc = z.bc / d.b, rst = z.st / d.b;
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    cudaEvent_t ev[2 * 8] = {};
+    auto cleanup = [&]() {
+        for (cudaEvent_t e : ev)
+            if (e) cudaEventDestroy(e);
+        if (s_in) cudaStreamDestroy(s_in);
+        if (s_out) cudaStreamDestroy(s_out);
+    };
+    auto fail = [&](ssd_status_t r) {
+        cudaStreamSynchronize(s);
+        if (s_in) cudaStreamSynchronize(s_in);
+        if (s_out) cudaStreamSynchronize(s_out);
+        cleanup();
+        return r;
+    };
+    if ((st = cuda_status("stream create", cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking))) != SSD_OK ||
+        (st = cuda_status("stream create", cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking))) != SSD_OK)
+        return fail(st);
+    for (int64_t k = 0; k < 2 * hp.nslices; ++k)
+        if ((st = cuda_status("event create", cudaEventCreateWithFlags(&ev[k], cudaEventDisableTiming))) != SSD_OK)
+            return fail(st);
+    // s_in starts after whatever the caller queued on `stream` before this call
+    if ((st = cuda_status("event record", cudaEventRecord(ev[0], s))) != SSD_OK ||
+        (st = cuda_status("stream wait", cudaStreamWaitEvent(s_in, ev[0], 0))) != SSD_OK)
+        return fail(st);
+    auto h2d = [&](void* dst, const void* src, size_t n) -> ssd_status_t {
+        if (n == 0) return SSD_OK;
+        return cuda_status("host to device copy", cudaMemcpyAsync(dst, src, n, cudaMemcpyHostToDevice, s_in));
+    };
+    auto d2h = [&](void* dst, const void* src, size_t n) -> ssd_status_t {
+        if (n == 0) return SSD_OK;
+        return cuda_status("device to host copy", cudaMemcpyAsync(dst, src, n, cudaMemcpyDeviceToHost, s_out));
+    };
+    if ((st = h2d(dA, A, z.hv)) != SSD_OK || (st = h2d(dD, D, D ? z.hv : 0)) != SSD_OK) return fail(st);
+    for (int64_t k = 0; k < hp.nslices; ++k) {
+        const int64_t r0 = k * hp.rows, nr = std::min(hp.rows, d.b - r0);
+        ssd::Dims ds = d;
+        ds.b = nr;
+        if ((st = h2d(dx + r0 * rx, (const char*)x + r0 * rx, nr * rx)) != SSD_OK ||
+            (st = h2d(ddt + r0 * rdt, (const char*)dt + r0 * rdt, nr * rdt)) != SSD_OK ||
+            (st = h2d(dB + r0 * rbc, (const char*)B + r0 * rbc, nr * rbc)) != SSD_OK ||
+            (st = h2d(dC + r0 * rbc, (const char*)C + r0 * rbc, nr * rbc)) != SSD_OK ||
+            (st = h2d(dinit + r0 * rst, initial_states ? (const char*)initial_states + r0 * rst : nullptr,
+                      initial_states ? nr * rst : 0)) != SSD_OK)
+            return fail(st);
+        if ((st = cuda_status("event record", cudaEventRecord(ev[2 * k], s_in))) != SSD_OK ||
+            (st = cuda_status("stream wait", cudaStreamWaitEvent(s, ev[2 * k], 0))) != SSD_OK)
+            return fail(st);
+        st = run_fwd(ds, dx + r0 * rx, (const float*)(ddt + r0 * rdt), dA, dB + r0 * rbc, dC + r0 * rbc,
+                     D ? dD : nullptr, initial_states ? (const float*)(dinit + r0 * rst) : nullptr,
+                     dy + r0 * rx, final_states ? (float*)(dfinal + r0 * rst) : nullptr,
+                     base + (size_t)k * hp.ws_slice, s);
+        if (st != SSD_OK) return fail(st);
+        if ((st = cuda_status("event record", cudaEventRecord(ev[2 * k + 1], s))) != SSD_OK ||
+            (st = cuda_status("stream wait", cudaStreamWaitEvent(s_out, ev[2 * k + 1], 0))) != SSD_OK)
+            return fail(st);
+        if ((st = d2h((char*)y + r0 * rx, dy + r0 * rx, nr * rx)) != SSD_OK ||
+            (st = d2h(final_states ? (char*)final_states + r0 * rst : nullptr, dfinal + r0 * rst,
+                      final_states ? nr * rst : 0)) != SSD_OK)
+            return fail(st);
     }
-    st = run_fwd(d, dx, ddt, dA, dB, dC, D ? dD : nullptr, initial_states ? dinit : nullptr, dy,
-                 final_states ? dfinal : nullptr, base, s);
-    if (st != SSD_OK) return st;
-    if (z.x && (st = cuda_status("device to host copy",
-                                 cudaMemcpyAsync(y, dy, z.x, cudaMemcpyDeviceToHost, s))) != SSD_OK)
-        return st;
-    if (final_states && z.st &&
-        (st = cuda_status("device to host copy",
-                          cudaMemcpyAsync(final_states, dfinal, z.st, cudaMemcpyDeviceToHost, s))) != SSD_OK)
-        return st;
-    if ((st = cuda_status("stream synchronize", cudaStreamSynchronize(s))) != SSD_OK) return st;
-    return read_device_status(d, base, s);
+    if ((st = cuda_status("stream synchronize", cudaStreamSynchronize(s_out))) != SSD_OK ||
+        (st = cuda_status("stream synchronize", cudaStreamSynchronize(s))) != SSD_OK)
+        return fail(st);
+    cleanup();
+    // every slice's fused kernel reports through its own status word
+    for (int64_t k = 0; k < hp.nslices; ++k) {
+        ssd::Dims ds = d;
+        ds.b = std::min(hp.rows, d.b - k * hp.rows);
+        if ((st = read_device_status(ds, base + (size_t)k * hp.ws_slice, s)) != SSD_OK) return st;
+    }
+    return SSD_OK;
 }
 
 ssd_status_t ssd_fwd_check(const ssd_shape_t* shape, const void* workspace, size_t workspace_bytes,
