@@ -163,9 +163,12 @@ SSD_API ssd_status_t ssd_fwd_host_workspace_size(const ssd_shape_t* shape, size_
 
 /*
  * Same computation as ssd_fwd on HOST buffers: copies the inputs to the device
- * workspace on `stream`, runs ssd_fwd there, copies y (and final_states when
- * non-NULL) back, and synchronizes `stream` before returning, so the host
- * outputs are ready on return. Host buffers should be page-locked for full
+ * workspace, runs ssd_fwd there, copies y (and final_states when non-NULL)
+ * back, and returns when everything is done, so the host outputs are ready on
+ * return. The batch is processed in up to 8 slices of rows: the forward of a
+ * slice runs on `stream` while two streams the call creates (and destroys
+ * before returning) copy the next slice in and the previous one out; the
+ * copies start after the work already queued on `stream`. Host buffers should be page-locked for full
  * copy bandwidth; pageable memory works but is slower. The device workspace
  * must hold ssd_fwd_host_workspace_size() bytes. Returns SSD_ERR_TIMEOUT (as
  * ssd_fwd_check) when the fused kernel's bounded waits gave up.
