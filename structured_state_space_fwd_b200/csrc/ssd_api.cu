@@ -90,12 +90,28 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 // each other); by default the fused tensor-core kernel runs where supported.
 enum class Path { Fused, Steps, Simt };
 
+// The fused kernel hands each head's state from tile to tile through a chain
+// across CTAs, so a sequence's tiles are processed one after another. With few
+// independent chains (batch rows x head blocks) and long sequences that chain,
+// not the work, sets the time, and the four separate steps (whose chunk states
+// are computed for all chunks in parallel) are faster: measured on B200 at
+// 32K tokens x 32 heads, fused 454 vs steps 567 us with 32 chains of 64 tiles,
+// fused 866 vs steps 571 us with 16 chains of 128 tiles.
+bool chain_bound(const ssd::Dims& d) {
+    const int64_t kh = ssd::pick_kheads(d.H / d.G);
+    const int64_t chains = d.b * (d.H / kh);
+    const int64_t tiles = (d.T + 127) / 128;
+    return chains < 24 && tiles >= 32;
+}
+
 Path pick_path(const ssd::Dims& d) {
     const char* e = getenv("SSD_PATH");
     const bool tc = ssd::tc_supported(d);
     if (e && strcmp(e, "simt") == 0) return Path::Simt;
     if (e && strcmp(e, "steps") == 0) return tc ? Path::Steps : Path::Simt;
-    return tc ? Path::Fused : Path::Simt;
+    if (e && strcmp(e, "fused") == 0) return tc ? Path::Fused : Path::Simt;
+    if (!tc) return Path::Simt;
+    return chain_bound(d) ? Path::Steps : Path::Fused;
 }
 
 bool steps_use_tc(const ssd::Dims& d) {

@@ -227,14 +227,12 @@ def test_full_long_context(ssd):
 
 # ---------------------------------------------------------------- tensor-core path
 # bf16, head dim 64, state dim 128, chunk 128 or 256 run on the tcgen05 kernels:
-# the fused kernel by default, the separate tensor-core steps with SSD_PATH=steps.
+# the fused kernel (SSD_PATH=fused forces it; by default it is chosen unless the
+# shape has few long chains), the separate tensor-core steps with SSD_PATH=steps.
 @pytest.fixture
 def path_env(monkeypatch):
     def set_path(p):
-        if p == "fused":
-            monkeypatch.delenv("SSD_PATH", raising=False)
-        else:
-            monkeypatch.setenv("SSD_PATH", p)
+        monkeypatch.setenv("SSD_PATH", p)
     return set_path
 
 
@@ -290,6 +288,18 @@ def test_tensor_steps_against_oracle(ssd, path_env):
     y = ssd.ssd_chunk_scan(d["x"], d["dt"], d["B"], d["C"], d["D"], cs, e_dev, shp)
     torch.cuda.synchronize()
     assert oracle.rel_err(y.float().cpu(), y_ref) <= 5e-3
+
+
+def test_path_choice(ssd, monkeypatch):
+    # fused kernel unless the shape has few independent chains of many tiles
+    monkeypatch.delenv("SSD_PATH", raising=False)
+    def plan(w):
+        return ssd.ssd_fwd_plan(ssd.ShapeT(w.batch, w.seqlen, w.nheads, w.headdim, w.ngroups,
+                                           w.dstate, w.chunk_size, ssd.SSD_BF16, 0))[0]
+    assert plan(W.MAMBA2_27B_LAYER) == "fused"
+    assert plan(W.seqlen_sweep()[4]) == "fused"     # 32 chains of 64 tiles
+    assert plan(W.seqlen_sweep()[5]) == "steps"     # 16 chains of 128 tiles
+    assert plan(W.LONG_CONTEXT) == "steps"          # 8 chains of 512 tiles
 
 
 def test_phase_sequential_fused_kernel(ssd, path_env, monkeypatch):
