@@ -204,6 +204,213 @@ def run_reference(args):
     return 0
 
 
+# ------------------------------------------------------------------ decoding step
+DECODE = W.DECODE_STEP_27B
+DECODE_METRIC = "SSD decode step (recurrent form) Mtokens/s at 2.7B layer shape, 128 sequences"
+# dram__bytes_read.sum + dram__bytes_write.sum of one ssd_step_kernel launch on this
+# workload, from one ncu capture (profiles/); None once the kernel changes
+DECODE_TRAFFIC = 614916608
+
+
+def decode_bytes(w: W.Workload) -> float:
+    """Algorithmic bytes of one decoding step: the fp32 state read and written
+    (8 b H P N) plus the token's x, y, dt, B, C and A, D."""
+    b, T, H, P, G, N = w.batch, w.seqlen, w.nheads, w.headdim, w.ngroups, w.dstate
+    s = 2 if w.dtype == "bf16" else 4
+    return 8.0 * b * H * P * N + b * T * (H * P * 2 * s + 4 * H + 2 * G * N * s) + 8.0 * H
+
+
+def measure_decode(ssd, dev, stream, steps, warmup, rank, with_cpu):
+    """Decoding steps on the 2.7B layer shape for 128 sequences: each step runs
+    ssd_step once, updating a carried fp32 state (335 MB) in place. Two state sets
+    are alternated so that a step never finds its state in L2 from the step before."""
+    w = DECODE
+    inp = W.workload_inputs(w, seed=rank)
+    d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+    states = [d["initial_states"].clone(), d["initial_states"].clone()]
+    y = torch.empty_like(d["x"])
+
+    def step(i):
+        ssd.ssd_step(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], states[i & 1], y=y,
+                     stream=stream)
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    by = decode_bytes(w)
+    pk, pk_kind = peaks()
+    achieved = by / (ms / 1e3) / 1e9
+    out = {"metric": DECODE_METRIC, "value": w.tokens / (ms / 1e3) / 1e6, "unit": UNIT,
+           "ms_per_step": ms, "steps": steps, "warmup": warmup, "dtype": "bf16",
+           "config": {"workload": w.name, **w.shape_dict(), "input_dtype": w.dtype,
+                      "state_mb": 4.0 * w.batch * w.nheads * w.headdim * w.dstate / 1e6,
+                      "l2": "two 335 MB state sets alternated, no flush"},
+           "roofline": {"kernel": "ssd_step_kernel", "bound": "hbm", "achieved": achieved,
+                        "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
+                        "traffic": DECODE_TRAFFIC, "alg_bytes_per_launch": by,
+                        "peak_source": pk_kind + " (burst copy, MEASURED_PEAKS hbm_gbs)"},
+           "gpu_launches": steps}
+    if with_cpu:
+        import oracle
+        f64 = {k: (v.double().numpy() if v is not None else None) for k, v in inp.items()}
+        t0 = time.perf_counter()
+        reps = 0
+        while time.perf_counter() - t0 < 3.0 or reps == 0:
+            oracle.recurrence(**f64)
+            reps += 1
+        el = time.perf_counter() - t0
+        out["cpu_baseline"] = {"value": w.tokens * reps / el / 1e6, "unit": UNIT,
+                               "cores": oracle.max_threads(), "kind": "oracle",
+                               "sample": f"fp64 recurrence, the whole step (128 sequences x 80 "
+                                         f"heads, one token); {reps} runs in {el:.1f} s"}
+    return out
+
+
+# ------------------------------------------------------------------ context parallelism
+CP = W.LONG_CONTEXT
+CP_METRIC = ("SSD fwd Mtokens/s, long context (b1 T65536 H32 P64 N128 G8) split over the "
+             "ranks along the sequence")
+
+
+def cp_slice_bytes(w: W.Workload, T_slice: int, nranks: int) -> float:
+    """Algorithmic bytes of one rank's slice: its x, y, dt, B, C (and A, D), the
+    initial and final states, and the gathered records it reads."""
+    ws = W.Workload(w.name, w.batch, T_slice, w.nheads, w.headdim, w.ngroups, w.dstate,
+                    w.chunk_size, w.dtype, w.dt_dist, w.initial_states)
+    _, by = alg_counts(ws, with_final=True, with_init=True)
+    return by + 4.0 * nranks * w.batch * w.nheads * (w.headdim * w.dstate + 1)
+
+
+def cp_setup(ssd, dev, w, nranks, rank, seed=0):
+    """Inputs of rank `rank`'s slice of the long-context sequence (the whole
+    sequence is drawn once with `seed`, then sliced)."""
+    inp = W.workload_inputs(w, seed=seed)
+    Ts = w.seqlen // nranks
+    sl = slice(rank * Ts, (rank + 1) * Ts)
+    d = {k: (inp[k][:, sl].contiguous().to(dev)) for k in ("x", "dt", "B", "C")}
+    d.update({k: (inp[k].to(dev) if inp[k] is not None else None) for k in ("A", "D", "initial_states")})
+    return d, Ts
+
+
+def measure_cp_slice(ssd, dev, stream, steps, warmup, nranks=8):
+    """One rank's work in an nranks-way split of the long-context sequence, timed on
+    one GPU: ssd_cp_begin, then ssd_cp_end of the last rank (which folds the most
+    records) with a records buffer standing in for the all-gather's result. The
+    collective itself needs several GPUs and is not in this number."""
+    w = CP
+    rank = nranks - 1
+    d, Ts = cp_setup(ssd, dev, w, nranks, rank)
+    rec, ws = ssd.ssd_cp_begin(d["x"], d["dt"], d["A"], d["B"], w.chunk_size)
+    records = rec.repeat(nranks)
+    y = torch.empty_like(d["x"])
+    fin = torch.empty_like(d["initial_states"])
+
+    def step():
+        ssd.ssd_cp_begin(d["x"], d["dt"], d["A"], d["B"], w.chunk_size, record=rec, workspace=ws,
+                         stream=stream)
+        ssd.ssd_cp_end(d["x"], d["dt"], d["B"], d["C"], d["D"], records, nranks, rank, ws,
+                       w.chunk_size, y=y, final_states=fin, stream=stream)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    by = cp_slice_bytes(w, Ts, nranks)
+    pk, pk_kind = peaks()
+    return {"what": f"one rank of {nranks}: ssd_cp_begin + ssd_cp_end on a {Ts}-token slice "
+                    f"(rank {rank}); the all-gather of {nranks} records of "
+                    f"{4 * w.batch * w.nheads * (w.headdim * w.dstate + 1) / 2**20:.2f} MiB is not timed",
+            "ms_per_rank_step": ms, "slice_tokens": Ts, "workload": w.name,
+            "kernels_per_rank_step": 7,
+            "roofline": {"bound": "hbm", "achieved": by / (ms / 1e3) / 1e9, "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": by / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
+                         "alg_bytes_per_rank_step": by, "traffic": None,
+                         "peak_source": pk_kind + " (burst copy, MEASURED_PEAKS hbm_gbs)"}}
+
+
+def run_cp(args):
+    """--workload long_context_cp: the long-context sequence split along its length
+    over the torchrun ranks (strong scaling: the sequence is fixed), one all-gather of
+    the per-rank records per step (NCCL), timed on the device, max over ranks."""
+    import datetime
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    import torch.distributed as dist
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    from structured_state_space_fwd_b200 import build as _b
+    _b.build()
+    import structured_state_space_fwd_b200 as ssd
+    w = CP
+    if w.seqlen % world:
+        raise SystemExit(f"seqlen {w.seqlen} does not split over {world} ranks")
+    d, Ts = cp_setup(ssd, dev, w, world, rank)
+    stream = torch.cuda.current_stream(dev)
+    init = d["initial_states"] if rank == 0 else None
+    rec, ws = ssd.ssd_cp_begin(d["x"], d["dt"], d["A"], d["B"], w.chunk_size, initial_states=init)
+    records = torch.empty(world * rec.numel(), dtype=torch.float32, device=dev)
+    y = torch.empty_like(d["x"])
+    fin = torch.empty_like(d["initial_states"])
+
+    def step():
+        ssd.ssd_cp_begin(d["x"], d["dt"], d["A"], d["B"], w.chunk_size, initial_states=init,
+                         record=rec, workspace=ws, stream=stream)
+        if world > 1:
+            dist.all_gather_into_tensor(records, rec)
+        else:
+            records.copy_(rec)
+        ssd.ssd_cp_end(d["x"], d["dt"], d["B"], d["C"], d["D"], records, world, rank, ws,
+                       w.chunk_size, initial_states=init, y=y, final_states=fin, stream=stream)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = ClockSampler(local)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.steps
+    by = cp_slice_bytes(w, Ts, world)
+    pk, pk_kind = peaks()
+    if rank == 0:
+        line = {"metric": CP_METRIC, "value": w.tokens / (ms / 1e3) / 1e6, "unit": UNIT,
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": w.name, **w.shape_dict(), "input_dtype": w.dtype,
+                           "slice_tokens": Ts, "exchange": "NCCL all-gather of per-rank records"
+                           if world > 1 else "none (one rank)",
+                           "l2": "per-rank slice inputs 34 MB + outputs; timed back to back"},
+                "roofline": {"kernel": "rank step (7 kernels + all-gather)", "bound": "hbm",
+                             "achieved": by / (ms / 1e3) / 1e9, "peak": pk["hbm_gbs"],
+                             "unit": "GB/s", "frac": by / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
+                             "traffic": None, "alg_bytes_per_rank_step": by,
+                             "peak_source": pk_kind + " (burst copy, MEASURED_PEAKS hbm_gbs)"},
+                "gpu_launches": 7 * args.steps, "clocks": clk}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 # ------------------------------------------------------------------ our arm
 def kernel_plan(ssd, w, d, bufs, stream):
     """The kernels of the unfused path as individually timed launches, with the
@@ -379,6 +586,13 @@ def run_ours(args):
         cpu = {"value": tok * reps / el / 1e6, "unit": UNIT, "cores": threads, "kind": "oracle",
                "sample": f"fp64 sequential recurrence, {desc}; {reps} runs in {el:.1f} s"}
 
+    decode = None
+    cp = None
+    if not args.profile:
+        decode = measure_decode(ssd, dev, stream, 200, 10, rank,
+                                rank == 0 and world == 1 and not args.no_cpu_baseline)
+        cp = measure_cp_slice(ssd, dev, stream, 50, 5)
+
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -396,11 +610,30 @@ def run_ours(args):
             "e2e": e2e,
             "gpu_launches": kernels_per_step * args.steps,
             "clocks": clk,
+            "next_rows": {"decode_step": decode, "context_parallel": cp},
         }
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+    return 0
+
+
+def run_decode_only(args):
+    """--workload decode_step: the decoding step alone, as the printed line."""
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from structured_state_space_fwd_b200 import build as _b
+    _b.build()
+    import structured_state_space_fwd_b200 as ssd
+    stream = torch.cuda.current_stream(dev)
+    out = measure_decode(ssd, dev, stream, args.steps, args.warmup, rank,
+                         world == 1 and not args.no_cpu_baseline and not args.profile)
+    if rank == 0:
+        out.update({"n_gpus": 1, "higher_is_better": True, "scaling": "weak",
+                    "vs_baseline": None, "data": "synthetic"})
+        print(json.dumps(out), flush=True)
     return 0
 
 
@@ -416,11 +649,19 @@ def main():
                     help="untimed load before the timed region, for the clock samples")
     ap.add_argument("--profile", action="store_true",
                     help="warmup and timed steps only (for ncu): no e2e, no CPU baseline")
+    ap.add_argument("--workload", choices=["layer", "decode_step", "long_context_cp"],
+                    default="layer",
+                    help="decode_step: time only the recurrent decoding step; long_context_cp: "
+                         "the long-context sequence split over the ranks (context parallel)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "decode_step":
+        return run_decode_only(args)
+    if args.workload == "long_context_cp":
+        return run_cp(args)
     return run_ours(args)
 
 

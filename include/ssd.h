@@ -180,6 +180,82 @@ SSD_API ssd_status_t ssd_fwd_host(const ssd_shape_t* shape,
                           void* y, float* final_states,
                           void* device_workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * Recurrent (linear) form for the decoding mode of the layer (Knowl 1, linear
+ * form: each new token costs O(P N) per head, however long the context): runs
+ * shape->seqlen tokens per batch row from `state` and leaves the state after
+ * the last one in `state`:
+ *     a = exp(dt[b,t,h] * A[h])
+ *     state[b,h,p,n] <- a * state[b,h,p,n] + dt[b,t,h] * x[b,t,h,p] * B[b,t,g,n]
+ *     y[b,t,h,p] = sum_n C[b,t,g,n] * state[b,h,p,n] + D[h] * x[b,t,h,p]
+ * i.e. ssd_fwd with initial_states = final_states = state, token by token.
+ *   x, dt, A, B, C, D, y   as for ssd_fwd (seqlen = tokens of this call, usually 1;
+ *                          seqlen 0 leaves state unchanged and writes no y).
+ *   state                  [b,H,P,N] fp32, read and overwritten in place; must
+ *                          not overlap any input or y.
+ *   shape->chunk_size      not used (any value).
+ * No workspace; one kernel launch (none when batch or seqlen is 0). The state
+ * is read once and written once per call, so a call is an HBM stream of
+ * 8 b H P N bytes plus the token's inputs; long prompts belong to ssd_fwd,
+ * whose final_states then seed this call.
+ */
+SSD_API ssd_status_t ssd_step(const ssd_shape_t* shape,
+                              const void* x, const float* dt, const float* A,
+                              const void* B, const void* C, const float* D,
+                              float* state, void* y, void* stream);
+
+/* ---- Sequence (context) parallelism (Knowl 8: the sequence is split along its
+ * length across workers; each runs its slice and only the boundary state
+ * travels). ----
+ * Rank r of R holds the contiguous slice r of every batch row's sequence (any
+ * lengths, zero allowed); all ranks share batch, nheads, headdim, ngroups,
+ * dstate, chunk_size and dtype, seqlen being the rank's own slice length. Per
+ * rank and call:
+ *   1. ssd_cp_begin: chunk cumsum and chunk states of the slice, then this
+ *      rank's record = [s (b H P N floats) | alpha (b H floats) | pad], where
+ *      s is the state the slice reaches from a zero state (rank 0: from the
+ *      sequence's initial_states) and alpha[b,h] = prod_{t in slice} a_t.
+ *   2. the caller all-gathers the records of every rank, in rank order, into
+ *      one buffer of R * record_floats floats (NCCL all-gather, or any
+ *      collective with that result);
+ *   3. ssd_cp_end: rank r's entering state h_in = fold over k < r of
+ *      h <- alpha_k h + s_k from h = 0 (rank 0: initial_states), then the state
+ *      passing from h_in and the chunk scan of the slice: y of the slice and,
+ *      in final_states, the state after the slice (on the last rank, the
+ *      sequence's final state).
+ * The result equals ssd_fwd over the whole sequence up to rounding. Each step
+ * runs the four-step kernels (tensor cores where ssd_fwd's steps path would);
+ * the exchange is one record per rank (about 1 MiB at 32 heads x 64 x 128). */
+
+/* Floats in one rank's record (b*H*P*N + b*H, rounded up to a multiple of 4). */
+SSD_API ssd_status_t ssd_cp_record_floats(const ssd_shape_t* shape, size_t* floats);
+
+/* Bytes of the device workspace ssd_cp_begin fills and ssd_cp_end reads. */
+SSD_API ssd_status_t ssd_cp_workspace_size(const ssd_shape_t* shape, size_t* bytes);
+
+/* Step 1 on this rank's slice. initial_states: the sequence's initial state on
+ * rank 0, NULL on every other rank (and NULL on rank 0 for a zero state).
+ * record: ssd_cp_record_floats() floats (16-byte aligned) receiving the record.
+ * workspace: ssd_cp_workspace_size() bytes, kept untouched until ssd_cp_end. */
+SSD_API ssd_status_t ssd_cp_begin(const ssd_shape_t* shape,
+                                  const void* x, const float* dt, const float* A,
+                                  const void* B, const float* initial_states,
+                                  float* record, void* workspace, size_t workspace_bytes,
+                                  void* stream);
+
+/* Step 3 on this rank's slice. records: the gathered records of all nranks
+ * ranks (nranks * record_floats floats, rank k's at offset k * record_floats);
+ * only those of ranks below `rank` are read. initial_states: as passed to
+ * ssd_cp_begin on rank 0 (ignored on other ranks). y: the slice's output
+ * [b, seqlen, H, P]. final_states (nullable): the state after the slice.
+ * workspace: the one ssd_cp_begin filled for this slice. */
+SSD_API ssd_status_t ssd_cp_end(const ssd_shape_t* shape, int nranks, int rank,
+                                const float* records, const float* initial_states,
+                                const void* x, const float* dt,
+                                const void* B, const void* C, const float* D,
+                                void* y, float* final_states,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
 /* ---- The four steps of the block-decomposition algorithm, one call each. ----
  * ssd_fwd runs the same steps (or a fused equivalent); these entry points
  * expose each one with its intermediate tensors for callers that need them:

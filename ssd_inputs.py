@@ -75,6 +75,12 @@ LONG_CONTEXT = Workload("long_context_b1_T65536_H32_P64_N128_G8_state_carry", 1,
                         64, 8, 128, 256, "bf16", "loguniform", initial_states=True)
 
 
+# one decoding step of the same layer for 128 sequences: the recurrent form on the
+# carried state [128, 80, 64, 128] fp32 (335 MB, larger than L2)
+DECODE_STEP_27B = Workload("decode_step_mamba2_2.7b_b128_H80_P64_N128_G1", 128, 1, 80, 64, 1,
+                           128, 256, "bf16", "loguniform", initial_states=True)
+
+
 def all_workloads() -> list[Workload]:
     return [TINY_FP32, MAMBA2_27B_LAYER, *seqlen_sweep(), *dstate_sweep(), LONG_CONTEXT]
 

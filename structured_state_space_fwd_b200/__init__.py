@@ -23,6 +23,7 @@ from ._lib import (SSD_BF16, SSD_F32, SSDError, ShapeT, check, lib, lib_path,  #
                    status_string)
 
 __all__ = ["ssd_fwd", "ssd_fwd_host", "ssd_fwd_workspace_size", "ssd_fwd_plan", "ssd_fwd_check",
+           "ssd_step", "ssd_fwd_cp", "ssd_cp_begin", "ssd_cp_end", "ssd_cp_record_floats",
            "ssd_chunk_cumsum",
            "ssd_chunk_state", "ssd_state_passing", "ssd_chunk_scan", "SSDError", "make_shape",
            "lib_path"]
@@ -127,6 +128,118 @@ def ssd_fwd_host(x, dt, A, B, C, D=None, chunk_size: int = 256, initial_states=N
                              _p(initial_states), _p(y), _p(final_states), _p(device_workspace),
                              ctypes.c_size_t(n.value), _stream(stream)), "ssd_fwd_host")
     return y, final_states
+
+
+def ssd_step(x, dt, A, B, C, D, state, y=None, stream=None):
+    """Recurrent form from `state` (updated in place) for the tokens in x; returns y.
+
+    x [b,T,H,P] (or [b,H,P] for one token), dt [b,T,H] (or [b,H]), B/C [b,T,G,N]
+    (or [b,G,N]), state [b,H,P,N] fp32. y has x's shape and dtype.
+    """
+    one = x.dim() == 3
+    if one:
+        x, dt, B, C = x.unsqueeze(1), dt.unsqueeze(1), B.unsqueeze(1), C.unsqueeze(1)
+    _need(x, "x")
+    _need(dt, "dt", torch.float32)
+    _need(A, "A", torch.float32)
+    _need(B, "B", x.dtype)
+    _need(C, "C", x.dtype)
+    _need(state, "state", torch.float32)
+    if D is not None:
+        _need(D, "D", torch.float32)
+    shape = make_shape(x, B, 0)
+    if y is None:
+        y = torch.empty_like(x)
+    elif one:
+        y = y.unsqueeze(1)
+    check(lib().ssd_step(ctypes.byref(shape), _p(x), _p(dt), _p(A), _p(B), _p(C), _p(D),
+                         _p(state), _p(y), _stream(stream)), "ssd_step")
+    return y.squeeze(1) if one else y
+
+
+def ssd_cp_record_floats(shape: ShapeT) -> int:
+    n = ctypes.c_size_t(0)
+    check(lib().ssd_cp_record_floats(ctypes.byref(shape), ctypes.byref(n)), "ssd_cp_record_floats")
+    return int(n.value)
+
+
+def ssd_cp_workspace_size(shape: ShapeT) -> int:
+    n = ctypes.c_size_t(0)
+    check(lib().ssd_cp_workspace_size(ctypes.byref(shape), ctypes.byref(n)), "ssd_cp_workspace_size")
+    return int(n.value)
+
+
+def ssd_cp_begin(x, dt, A, B, chunk_size: int = 256, initial_states=None, record=None,
+                 workspace=None, stream=None):
+    """Sequence-parallel step 1 on this rank's slice; returns (record, workspace)."""
+    _need(x, "x")
+    _need(dt, "dt", torch.float32)
+    _need(A, "A", torch.float32)
+    _need(B, "B", x.dtype)
+    if initial_states is not None:
+        _need(initial_states, "initial_states", torch.float32)
+    shape = make_shape(x, B, chunk_size)
+    if record is None:
+        record = torch.empty(max(ssd_cp_record_floats(shape), 4), dtype=torch.float32,
+                             device=x.device)
+    nbytes = ssd_cp_workspace_size(shape)
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=x.device)
+    check(lib().ssd_cp_begin(ctypes.byref(shape), _p(x), _p(dt), _p(A), _p(B), _p(initial_states),
+                             _p(record), _p(workspace), ctypes.c_size_t(nbytes), _stream(stream)),
+          "ssd_cp_begin")
+    return record, workspace
+
+
+def ssd_cp_end(x, dt, B, C, D, records, nranks: int, rank: int, workspace, chunk_size: int = 256,
+               initial_states=None, y=None, final_states=None, stream=None):
+    """Sequence-parallel step 3 on this rank's slice; returns (y, final_states)."""
+    _need(x, "x")
+    _need(dt, "dt", torch.float32)
+    _need(B, "B", x.dtype)
+    _need(C, "C", x.dtype)
+    _need(records, "records", torch.float32)
+    if D is not None:
+        _need(D, "D", torch.float32)
+    shape = make_shape(x, B, chunk_size)
+    if y is None:
+        y = torch.empty_like(x)
+    if final_states is None:
+        final_states = torch.empty((x.shape[0], x.shape[2], x.shape[3], B.shape[3]),
+                                   dtype=torch.float32, device=x.device)
+    nbytes = ssd_cp_workspace_size(shape)
+    check(lib().ssd_cp_end(ctypes.byref(shape), int(nranks), int(rank), _p(records),
+                           _p(initial_states), _p(x), _p(dt), _p(B), _p(C), _p(D), _p(y),
+                           _p(final_states), _p(workspace), ctypes.c_size_t(nbytes),
+                           _stream(stream)), "ssd_cp_end")
+    return y, final_states
+
+
+def _cp_exchange(record, world: int, group=None):
+    """All ranks' records, gathered in rank order (one collective)."""
+    import torch.distributed as dist
+    out = torch.empty(world * record.numel(), dtype=record.dtype, device=record.device)
+    dist.all_gather_into_tensor(out, record, group=group)
+    return out
+
+
+def ssd_fwd_cp(x, dt, A, B, C, D=None, chunk_size: int = 256, initial_states=None,
+               return_final_states: bool = False, group=None):
+    """Context-parallel SSD forward over the ranks of `group` (torch.distributed).
+
+    Every rank passes its own contiguous slice of the sequence (x [b, T_r, H, P],
+    dt, B, C likewise), rank order being sequence order; initial_states is read on
+    rank 0 only. Returns this slice's y (and the state after the slice, which on
+    the last rank is the sequence's final state).
+    """
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    init = initial_states if rank == 0 else None
+    record, ws = ssd_cp_begin(x, dt, A, B, chunk_size, initial_states=init)
+    records = _cp_exchange(record, world, group)
+    y, fin = ssd_cp_end(x, dt, B, C, D, records, world, rank, ws, chunk_size, initial_states=init)
+    return (y, fin) if return_final_states else y
 
 
 def ssd_chunk_cumsum(dt, A, chunk_size, shape: ShapeT, cs=None, stream=None):

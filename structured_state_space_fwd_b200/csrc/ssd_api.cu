@@ -240,6 +240,27 @@ ssd_status_t read_device_status(const ssd::Dims& d, const void* workspace, cudaS
     return SSD_ERR_TIMEOUT;
 }
 
+// Sequence-parallel workspace (ssd_cp_begin fills cs and S, ssd_cp_end reads them):
+//   [cs | chunk states S | entry states | entering state h_in], regions 256-byte aligned.
+struct CpWorkspace {
+    size_t off_cs, off_S, off_entry, off_hin, total;
+};
+CpWorkspace cp_workspace(const ssd::Dims& d) {
+    const Sizes z = sizes_of(d);
+    CpWorkspace w;
+    w.off_cs = 0;
+    w.off_S = align_up(z.cs, 256);
+    w.off_entry = w.off_S + align_up(z.chunk_states, 256);
+    w.off_hin = w.off_entry + align_up(z.chunk_states, 256);
+    w.total = w.off_hin + align_up(z.st, 256);
+    if (d.b == 0) w.total = 0;
+    return w;
+}
+// One rank's record: its slice's state [b,H,P,N], then alpha [b,H], padded to 16 bytes.
+size_t cp_record_floats(const ssd::Dims& d) {
+    return align_up((size_t)(d.b * d.H * d.P * d.N + d.b * d.H), 4);
+}
+
 // ssd_fwd_host works through the batch in slices of rows so that the copies in,
 // the forward and the copies out of different slices overlap (the two copy
 // directions use separate copy engines). Each slice has its own forward
@@ -450,6 +471,147 @@ ssd_status_t ssd_fwd_check(const ssd_shape_t* shape, const void* workspace, size
     const FwdWorkspace w = fwd_workspace(d);
     if (workspace_bytes < w.total || (w.total > 0 && !workspace)) return SSD_ERR_INVALID_ARG;
     return read_device_status(d, workspace, (cudaStream_t)stream);
+}
+
+ssd_status_t ssd_step(const ssd_shape_t* shape, const void* x, const float* dt, const float* A,
+                      const void* B, const void* C, const float* D, float* state, void* y,
+                      void* stream) {
+    if (!shape) return SSD_ERR_INVALID_ARG;
+    ssd_shape_t s = *shape;
+    s.chunk_size = 64;   // not used by the recurrent form
+    ssd_status_t st = check_shape(&s);
+    if (st != SSD_OK) return st;
+    const ssd::Dims d = ssd::make_dims(s);
+    const Sizes z = sizes_of(d);
+    if ((!x && z.x) || (!dt && z.dt) || !A || (!B && z.bc) || (!C && z.bc) || (!y && z.x) ||
+        (!state && z.st))
+        return SSD_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(y, 16) || !aligned(state, 16))
+        return SSD_ERR_INVALID_ARG;
+    if (!aligned(dt, 4) || !aligned(A, 4) || (D && !aligned(D, 4))) return SSD_ERR_INVALID_ARG;
+    const Range ins[] = {{x, z.x}, {dt, z.dt}, {A, z.hv}, {B, z.bc}, {C, z.bc}, {D, D ? z.hv : 0}};
+    const Range outs[] = {{state, z.st}, {y, z.x}};
+    for (const Range& o : outs)
+        for (const Range& i : ins)
+            if (overlaps(o, i)) return SSD_ERR_INVALID_ARG;
+    if (overlaps(outs[0], outs[1])) return SSD_ERR_INVALID_ARG;
+    return cuda_status("recurrent step", ssd::launch_step(d, x, dt, A, B, C, D, state, y,
+                                                          (cudaStream_t)stream));
+}
+
+ssd_status_t ssd_cp_record_floats(const ssd_shape_t* shape, size_t* floats) {
+    if (!floats) return SSD_ERR_INVALID_ARG;
+    ssd_status_t st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    *floats = cp_record_floats(ssd::make_dims(*shape));
+    return SSD_OK;
+}
+
+ssd_status_t ssd_cp_workspace_size(const ssd_shape_t* shape, size_t* bytes) {
+    if (!bytes) return SSD_ERR_INVALID_ARG;
+    ssd_status_t st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    *bytes = cp_workspace(ssd::make_dims(*shape)).total;
+    return SSD_OK;
+}
+
+ssd_status_t ssd_cp_begin(const ssd_shape_t* shape, const void* x, const float* dt, const float* A,
+                          const void* B, const float* initial_states, float* record,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+    ssd_status_t st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    const ssd::Dims d = ssd::make_dims(*shape);
+    const Sizes z = sizes_of(d);
+    const size_t rec_bytes = cp_record_floats(d) * 4;
+    const CpWorkspace w = cp_workspace(d);
+    if ((!x && z.x) || (!dt && z.dt) || !A || (!B && z.bc) || (!record && rec_bytes))
+        return SSD_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(B, 16) || !aligned(record, 16) || !aligned(workspace, 16) ||
+        (initial_states && !aligned(initial_states, 16)) || !aligned(dt, 4) || !aligned(A, 4))
+        return SSD_ERR_INVALID_ARG;
+    if (workspace_bytes < w.total || (w.total > 0 && !workspace)) return SSD_ERR_INVALID_ARG;
+    const Range ins[] = {{x, z.x}, {dt, z.dt}, {A, z.hv}, {B, z.bc},
+                         {initial_states, initial_states ? z.st : 0}};
+    const Range outs[] = {{record, rec_bytes}, {workspace, w.total}};
+    for (const Range& o : outs)
+        for (const Range& i : ins)
+            if (overlaps(o, i)) return SSD_ERR_INVALID_ARG;
+    if (overlaps(outs[0], outs[1])) return SSD_ERR_INVALID_ARG;
+    if (d.b == 0) return SSD_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    float* alpha = record + d.b * d.H * d.P * d.N;
+    if (d.T == 0) {
+        if ((st = cuda_status("slice state", ssd::launch_copy_or_zero_states(d, initial_states, record, s))) != SSD_OK)
+            return st;
+        return cuda_status("slice decay", ssd::launch_slice_decay(d, nullptr, alpha, s));
+    }
+    char* ws = (char*)workspace;
+    float* cs = (float*)(ws + w.off_cs);
+    float* S = (float*)(ws + w.off_S);
+    if ((st = cuda_status("chunk cumsum", ssd::launch_chunk_cumsum(d, dt, A, cs, s))) != SSD_OK) return st;
+    if ((st = cuda_status("chunk state",
+                          steps_use_tc(d) ? ssd::launch_chunk_state_tc(d, x, dt, B, cs, S, s)
+                                          : ssd::launch_chunk_state_simt(d, x, dt, B, cs, S, s))) != SSD_OK)
+        return st;
+    if ((st = cuda_status("slice state", ssd::launch_state_passing(d, S, cs, initial_states, nullptr,
+                                                                    record, s))) != SSD_OK)
+        return st;
+    return cuda_status("slice decay", ssd::launch_slice_decay(d, cs, alpha, s));
+}
+
+ssd_status_t ssd_cp_end(const ssd_shape_t* shape, int nranks, int rank, const float* records,
+                        const float* initial_states, const void* x, const float* dt,
+                        const void* B, const void* C, const float* D, void* y,
+                        float* final_states, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+    ssd_status_t st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    if (nranks < 1 || rank < 0 || rank >= nranks) return SSD_ERR_INVALID_ARG;
+    const ssd::Dims d = ssd::make_dims(*shape);
+    const Sizes z = sizes_of(d);
+    const size_t rec_floats = cp_record_floats(d);
+    const size_t recs_bytes = rec_floats * 4 * (size_t)nranks;
+    const CpWorkspace w = cp_workspace(d);
+    if ((!x && z.x) || (!dt && z.dt) || (!B && z.bc) || (!C && z.bc) || (!y && z.x) ||
+        (!records && recs_bytes))
+        return SSD_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(y, 16) ||
+        !aligned(records, 16) || !aligned(workspace, 16) ||
+        (initial_states && !aligned(initial_states, 16)) ||
+        (final_states && !aligned(final_states, 16)) || !aligned(dt, 4) || (D && !aligned(D, 4)))
+        return SSD_ERR_INVALID_ARG;
+    if (workspace_bytes < w.total || (w.total > 0 && !workspace)) return SSD_ERR_INVALID_ARG;
+    const Range ins[] = {{x, z.x}, {dt, z.dt}, {B, z.bc}, {C, z.bc}, {D, D ? z.hv : 0},
+                         {initial_states, initial_states ? z.st : 0}, {records, recs_bytes}};
+    const Range outs[] = {{y, z.x}, {final_states, final_states ? z.st : 0}, {workspace, w.total}};
+    for (const Range& o : outs)
+        for (const Range& i : ins)
+            if (overlaps(o, i)) return SSD_ERR_INVALID_ARG;
+    for (int i = 0; i < 3; ++i)
+        for (int j = i + 1; j < 3; ++j)
+            if (overlaps(outs[i], outs[j])) return SSD_ERR_INVALID_ARG;
+    if (d.b == 0) return SSD_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    char* ws = (char*)workspace;
+    const float* h_in = initial_states;
+    if (rank > 0) {
+        float* hin = (float*)(ws + w.off_hin);
+        if ((st = cuda_status("rank fold", ssd::launch_cp_fold(d, records, (int64_t)rec_floats, rank,
+                                                               hin, s))) != SSD_OK)
+            return st;
+        h_in = hin;
+    }
+    if (d.T == 0)
+        return cuda_status("final states", ssd::launch_copy_or_zero_states(d, h_in, final_states, s));
+    const float* cs = (const float*)(ws + w.off_cs);
+    const float* S = (const float*)(ws + w.off_S);
+    float* entry = (float*)(ws + w.off_entry);
+    if ((st = cuda_status("state passing", ssd::launch_state_passing(d, S, cs, h_in, entry,
+                                                                      final_states, s))) != SSD_OK)
+        return st;
+    return cuda_status("chunk scan",
+                       steps_use_tc(d) ? ssd::launch_chunk_scan_tc(d, x, dt, B, C, D, cs, entry, y, s)
+                                       : ssd::launch_chunk_scan_simt(d, x, dt, B, C, D, cs, entry, y, s));
 }
 
 ssd_status_t ssd_chunk_cumsum(const ssd_shape_t* shape, const float* dt, const float* A,

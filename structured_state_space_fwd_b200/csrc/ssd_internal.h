@@ -54,6 +54,23 @@ cudaError_t launch_fused_ws(const Dims& d, const CUtensorMap* maps, const void* 
                             const float* A, const float* D, const float* init, void* y,
                             float* chain, int* sync_ints, int kheads, cudaStream_t st);
 
+// Recurrent form for a few tokens per sequence, state [b,H,P,N] updated in place.
+struct StepLayout {
+    int W;             // state elements per load (4 when N % 4 == 0, else 1)
+    int L;             // lanes sharing one state row
+    int K;             // W-wide pieces of a row per lane
+    int rows_per_cta;  // state rows one CTA owns
+};
+StepLayout step_layout(int64_t N);
+cudaError_t launch_step(const Dims& d, const void* x, const float* dt, const float* A, const void* B,
+                        const void* C, const float* D, float* state, void* y, cudaStream_t st);
+
+// Sequence parallelism: alpha[b,h] = prod of a_t over the slice (from cs), and the fold
+// of ranks 0..rank-1's records [state b*H*P*N | alpha b*H] into rank's entering state.
+cudaError_t launch_slice_decay(const Dims& d, const float* cs, float* alpha, cudaStream_t st);
+cudaError_t launch_cp_fold(const Dims& d, const float* records, int64_t rec_floats, int rank,
+                           float* h_in, cudaStream_t st);
+
 // Sets the message ssd_last_error_detail() returns on the calling host thread.
 void set_error_detail(const char* msg);
 

@@ -180,3 +180,72 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(_lib, "lib_path", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         _lib.lib()
+
+
+def test_recurrent_step_rejections(L):
+    """ssd_step: state is in/out, so it may overlap neither an input nor y; the other
+    rules are ssd_fwd's. chunk_size is not used by the recurrent form."""
+    s = shape(seqlen=1)
+    bufs = Bufs(s)
+    lib = L.lib()
+
+    def call(**over):
+        names = ["x", "dt", "A", "B", "C", "D", "init", "y"]
+        a = {k: bufs.p(k) for k in names}
+        a.update(over)
+        sh = over.pop("shape", s) if "shape" in over else s
+        return lib.ssd_step(ctypes.byref(sh), a["x"], a["dt"], a["A"], a["B"], a["C"], a["D"],
+                            a["init"], a["y"], None)
+    assert call(init=None) == 1                       # state required
+    assert call(x=None) == 1
+    assert call(init=bufs.p("x")) == 1                # state overlaps x
+    assert call(init=off(bufs, "B", 16)) == 1         # state overlaps B
+    assert call(y=bufs.p("init")) == 1                # y overlaps state
+    assert call(y=bufs.p("C")) == 1                   # y overlaps an input
+    assert call(init=off(bufs, "init", 4)) == 1       # state misaligned
+    assert call(shape=shape(seqlen=1, nheads=5, ngroups=2)) == 1
+    assert call(shape=shape(seqlen=1, dstate=300)) == 2
+    assert call(shape=shape(seqlen=1, dtype=5)) == 1
+
+
+def test_context_parallel_sizes_and_rejections(L):
+    """ssd_cp_*: record size is the documented layout; bad ranks, missing or
+    overlapping buffers and a short workspace are rejected before any launch."""
+    s = shape()
+    lib = L.lib()
+    n = ctypes.c_size_t(0)
+    assert lib.ssd_cp_record_floats(ctypes.byref(s), ctypes.byref(n)) == 0
+    bhpn, bh = s.batch * s.nheads * s.headdim * s.dstate, s.batch * s.nheads
+    assert n.value == (bhpn + bh + 3) // 4 * 4
+    rec_floats = n.value
+    ws = ctypes.c_size_t(0)
+    assert lib.ssd_cp_workspace_size(ctypes.byref(s), ctypes.byref(ws)) == 0 and ws.value > 0
+    bufs = Bufs(s)
+    # records of 4 ranks and one cp workspace, as placeholder or real device buffers
+    if bufs.real:
+        recs = torch.empty(4 * rec_floats, dtype=torch.float32, device="cuda")
+        cpws = torch.empty(ws.value, dtype=torch.uint8, device="cuda")
+        rp, wp = recs.data_ptr(), cpws.data_ptr()
+    else:
+        rp, wp = 1 << 44, 1 << 45
+    R = ctypes.c_void_p(rp)
+    WS = ctypes.c_void_p(wp)
+    p = bufs.p
+
+    def begin(record=R, x=None, ws_bytes=ws.value, workspace=WS):
+        return lib.ssd_cp_begin(ctypes.byref(s), x or p("x"), p("dt"), p("A"), p("B"), None,
+                                record, workspace, ctypes.c_size_t(ws_bytes), None)
+
+    def end(nranks=4, rank=1, records=R, y=None, final=None, ws_bytes=ws.value):
+        return lib.ssd_cp_end(ctypes.byref(s), nranks, rank, records, None, p("x"), p("dt"),
+                              p("B"), p("C"), p("D"), y or p("y"), final, WS,
+                              ctypes.c_size_t(ws_bytes), None)
+    assert begin(record=None) == 1
+    assert begin(record=p("x")) == 1                      # record overlaps x
+    assert begin(ws_bytes=ws.value - 1) == 1
+    assert begin(workspace=R) == 1                        # workspace overlaps the record
+    assert end(rank=4) == 1 and end(rank=-1) == 1 and end(nranks=0, rank=0) == 1
+    assert end(records=None) == 1
+    assert end(y=R) == 1                                  # y overlaps the records
+    assert end(final=p("x")) == 1
+    assert end(ws_bytes=0) == 1
