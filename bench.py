@@ -209,7 +209,7 @@ DECODE = W.DECODE_STEP_27B
 DECODE_METRIC = "SSD decode step (recurrent form) Mtokens/s at 2.7B layer shape, 128 sequences"
 # dram__bytes_read.sum + dram__bytes_write.sum of one ssd_step_kernel launch on this
 # workload, from one ncu capture (profiles/); None once the kernel changes
-DECODE_TRAFFIC = 614916608
+DECODE_TRAFFIC = 614314752
 
 
 def decode_bytes(w: W.Workload) -> float:

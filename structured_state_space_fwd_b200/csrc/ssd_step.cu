@@ -21,7 +21,7 @@ namespace ssd {
 namespace {
 
 constexpr int kStepWarps = 4;
-constexpr int kStepChunks = 8;   // W-wide pieces of state a thread holds
+constexpr int kStepChunks = 4;   // W-wide pieces of state a thread holds
 
 struct StepParams {
     const void* x;
