@@ -7,7 +7,8 @@ code with the CUDA path and never imports it.
 Source of every definition: "Transformers are SSMs: Generalized Models and
 Efficient Algorithms Through Structured State Space Duality" (summary page),
 Knowl 1 (linear and dual forms), Knowl 2 (block-decomposition algorithm) and
-Knowl 7 (head patterns); "Mamba-2 and State Space Duality (SSD)", section
+Knowl 6 (Mamba-2 block: gate and norm), Knowl 7 (head patterns); "Mamba-2 and
+State Space Duality (SSD)", section
 "The Concept of State Space Duality" (dual form Y = (L o C B^T) X).
 
 Functions
@@ -18,6 +19,7 @@ Functions
                   from a zero state (Knowl 2, "right factor chunk state").
   dual_form()     the quadratic (masked attention) form, tiny T only.
   chunked()       the block-decomposition algorithm, step by step, fp64.
+  gated_rmsnorm() the gate and RMSNorm after the layer (Knowl 6), fp64.
 Every function is pinned by ``tests/test_oracle.py`` against closed forms,
 library routines and the identities the pages state.
 """
@@ -255,6 +257,30 @@ def chunked(x, dt, A, B, C, D=None, chunk_size=64, initial_states=None):
             if D is not None:
                 y[bi, :, h, :] += D[h] * x[bi, :, h, :]
     return y, final, cs_all, S_all, entry
+
+
+def gated_rmsnorm(y, z, weight, group_size, eps):
+    """Gate and normalisation after the SSD layer, fp64.
+
+    "Transformers are SSMs" (summary page), Knowl 6, step 4 of the Mamba-2
+    block: the layer output is gated elementwise by the SiLU of the gate branch
+    z, Y_g = Y * SiLU(z) with SiLU(v) = v / (1 + exp(-v)), then normalised
+    (RMSNorm) before the output projection. Reading where the page is silent:
+    the channels of a token (H * P, head-major as in y) are split into
+    contiguous groups of ``group_size``; each group is divided by
+    sqrt(mean over the group of Y_g^2 + eps) and scaled by the per-channel
+    ``weight`` [H * P].
+    y, z: [..., H, P] (same shape); returns an array of that shape.
+    """
+    y, z, w = _f64(y), _f64(z), _f64(weight)
+    shape = y.shape
+    C = shape[-2] * shape[-1]
+    if C % group_size != 0:
+        raise ValueError("group_size must divide the channel count")
+    yg = (y * (z / (1.0 + np.exp(-z)))).reshape(-1, C // group_size, group_size)
+    ms = np.mean(yg * yg, axis=-1, keepdims=True)
+    out = yg / np.sqrt(ms + eps) * w.reshape(C // group_size, group_size)
+    return out.reshape(shape)
 
 
 def rel_err(a, ref) -> float:

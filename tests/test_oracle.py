@@ -282,3 +282,52 @@ def test_golden_fixture():
                                     arr["initial_states"])
     np.testing.assert_allclose(y, np.array(g["y"]), rtol=1e-13, atol=1e-15)
     np.testing.assert_allclose(final, np.array(g["final_states"]), rtol=1e-13, atol=1e-15)
+
+
+# ---------------------------------------------------------------- gate + norm (Knowl 6)
+def _gate_inputs(seed, rows=6, H=4, P=8):
+    rng = np.random.Generator(np.random.PCG64(seed))
+    y = rng.standard_normal((rows, H, P))
+    z = rng.standard_normal((rows, H, P)) * 2.0
+    w = rng.uniform(0.5, 1.5, size=(H * P,))
+    return y, z, w
+
+
+@pytest.mark.parametrize("group_size", [32, 16, 8, 1])
+def test_gated_rmsnorm_matches_library_rmsnorm(group_size):
+    """Against torch's own SiLU and RMSNorm routines (fp64), groups as reshapes."""
+    import torch
+    y, z, w = _gate_inputs(1)
+    eps = 1e-5
+    got = oracle.gated_rmsnorm(y, z, w, group_size, eps)
+    ty, tz = torch.from_numpy(y), torch.from_numpy(z)
+    g = (ty * torch.nn.functional.silu(tz)).reshape(y.shape[0], -1, group_size)
+    ref = torch.nn.functional.rms_norm(g, (group_size,), eps=eps)
+    ref = (ref * torch.from_numpy(w).reshape(-1, group_size)).reshape(y.shape).numpy()
+    assert np.max(np.abs(got - ref)) <= 1e-12 * np.max(np.abs(ref))
+
+
+def test_gated_rmsnorm_identities():
+    y, z, w = _gate_inputs(2)
+    ones = np.ones_like(w)
+    # eps = 0: scale invariant, odd in y, and every group comes out with unit RMS
+    a = oracle.gated_rmsnorm(y, z, w, 16, 0.0)
+    assert np.allclose(oracle.gated_rmsnorm(3.7 * y, z, w, 16, 0.0), a, rtol=1e-13, atol=0)
+    assert np.allclose(oracle.gated_rmsnorm(-y, z, w, 16, 0.0), -a, rtol=1e-13, atol=0)
+    u = oracle.gated_rmsnorm(y, z, ones, 16, 0.0).reshape(y.shape[0], -1, 16)
+    assert np.allclose(np.mean(u * u, axis=-1), 1.0, rtol=1e-13)
+    # a closed gate (z = 0) gives 0; SiLU(z) -> z for large z and -> 0 for very negative z
+    assert np.all(oracle.gated_rmsnorm(y, np.zeros_like(z), w, 16, 1e-5) == 0)
+    big = np.full_like(z, 40.0)
+    ref = oracle.gated_rmsnorm(y * 40.0, np.full_like(z, 1e9), w, 16, 0.0)
+    assert np.allclose(oracle.gated_rmsnorm(y, big, w, 16, 0.0), ref, rtol=1e-12)
+
+
+def test_gated_rmsnorm_hand_example():
+    """One group of two channels, gate open (SiLU(z) = z for z -> inf, here z = 60
+    where 1/(1+e^-60) = 1 in fp64): values 3*60 and 4*60; RMS = 60*sqrt((9+16)/2),
+    so the outputs are 3/sqrt(12.5) and 4/sqrt(12.5) times the weights 2 and 1."""
+    y = np.array([[[3.0, 4.0]]])
+    z = np.full_like(y, 60.0)
+    out = oracle.gated_rmsnorm(y, z, np.array([2.0, 1.0]), 2, 0.0)
+    assert np.allclose(out.ravel(), [2 * 3 / math.sqrt(12.5), 4 / math.sqrt(12.5)], rtol=1e-15)
