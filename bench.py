@@ -209,7 +209,7 @@ DECODE = W.DECODE_STEP_27B
 DECODE_METRIC = "SSD decode step (recurrent form) Mtokens/s at 2.7B layer shape, 128 sequences"
 # dram__bytes_read.sum + dram__bytes_write.sum of one ssd_step_kernel launch on this
 # workload, from one ncu capture (profiles/); None once the kernel changes
-DECODE_TRAFFIC = 614314752
+DECODE_TRAFFIC = 614955264
 
 
 def decode_bytes(w: W.Workload) -> float:
@@ -270,6 +270,50 @@ def measure_decode(ssd, dev, stream, steps, warmup, rank, with_cpu):
                                "sample": f"fp64 recurrence, the whole step (128 sequences x 80 "
                                          f"heads, one token); {reps} runs in {el:.1f} s"}
     return out
+
+
+# ------------------------------------------------------------------ gate + norm
+GATE_METRIC = "SSD gate + RMSNorm (y * SiLU(z), one group of 5120 channels) at 2.7B layer shape"
+
+
+def measure_gate(ssd, dev, stream, steps, warmup, seed=0):
+    """ssd_gated_rmsnorm on the layer output of the 2.7B shape: y, z bf16
+    [8, 2048, 80, 64] (168 MB each, larger than L2), weight [5120], one norm group
+    per token. Algorithmic bytes: y and z read, out written, weight read."""
+    w = WORKLOAD
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    shp = (w.batch, w.seqlen, w.nheads, w.headdim)
+    y = torch.randn(shp, generator=g).to(torch.bfloat16).to(dev)
+    z = (torch.randn(shp, generator=g) * 2.0).to(torch.bfloat16).to(dev)
+    wt = (torch.rand(w.nheads * w.headdim, generator=g) + 0.5).to(dev)
+    out = torch.empty_like(y)
+
+    def step():
+        ssd.ssd_gated_rmsnorm(y, z, wt, group_size=w.nheads * w.headdim, out=out, stream=stream)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    by = 3.0 * y.numel() * 2 + 4.0 * wt.numel()
+    pk, pk_kind = peaks()
+    return {"metric": GATE_METRIC, "value": w.tokens / (ms / 1e3) / 1e6, "unit": UNIT,
+            "ms_per_step": ms, "steps": steps, "warmup": warmup, "dtype": "bf16",
+            "config": {"workload": "gate_rmsnorm_b8_T2048_C5120_group5120", "batch": w.batch,
+                       "seqlen": w.seqlen, "channels": w.nheads * w.headdim,
+                       "group_size": w.nheads * w.headdim,
+                       "l2": "y and z 168 MB each, larger than L2, no flush"},
+            "roofline": {"kernel": "gated_rmsnorm_kernel", "bound": "hbm",
+                         "achieved": by / (ms / 1e3) / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": by / (ms / 1e3) / 1e9 / pk["hbm_gbs"], "traffic": None,
+                         "alg_bytes_per_launch": by,
+                         "peak_source": pk_kind + " (burst copy, MEASURED_PEAKS hbm_gbs)"},
+            "gpu_launches": steps}
 
 
 # ------------------------------------------------------------------ context parallelism
@@ -588,10 +632,12 @@ def run_ours(args):
 
     decode = None
     cp = None
+    gate = None
     if not args.profile:
         decode = measure_decode(ssd, dev, stream, 200, 10, rank,
                                 rank == 0 and world == 1 and not args.no_cpu_baseline)
         cp = measure_cp_slice(ssd, dev, stream, 50, 5)
+        gate = measure_gate(ssd, dev, stream, 100, 5, seed=rank)
 
     if rank == 0:
         line = {
@@ -610,7 +656,7 @@ def run_ours(args):
             "e2e": e2e,
             "gpu_launches": kernels_per_step * args.steps,
             "clocks": clk,
-            "next_rows": {"decode_step": decode, "context_parallel": cp},
+            "next_rows": {"decode_step": decode, "context_parallel": cp, "gate_norm": gate},
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -620,7 +666,7 @@ def run_ours(args):
 
 
 def run_decode_only(args):
-    """--workload decode_step: the decoding step alone, as the printed line."""
+    """--workload decode_step / gate_norm: that kernel alone, as the printed line."""
     world, rank, local = dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -628,8 +674,11 @@ def run_decode_only(args):
     _b.build()
     import structured_state_space_fwd_b200 as ssd
     stream = torch.cuda.current_stream(dev)
-    out = measure_decode(ssd, dev, stream, args.steps, args.warmup, rank,
-                         world == 1 and not args.no_cpu_baseline and not args.profile)
+    if args.workload == "gate_norm":
+        out = measure_gate(ssd, dev, stream, args.steps, args.warmup, seed=rank)
+    else:
+        out = measure_decode(ssd, dev, stream, args.steps, args.warmup, rank,
+                             world == 1 and not args.no_cpu_baseline and not args.profile)
     if rank == 0:
         out.update({"n_gpus": 1, "higher_is_better": True, "scaling": "weak",
                     "vs_baseline": None, "data": "synthetic"})
@@ -649,7 +698,7 @@ def main():
                     help="untimed load before the timed region, for the clock samples")
     ap.add_argument("--profile", action="store_true",
                     help="warmup and timed steps only (for ncu): no e2e, no CPU baseline")
-    ap.add_argument("--workload", choices=["layer", "decode_step", "long_context_cp"],
+    ap.add_argument("--workload", choices=["layer", "decode_step", "gate_norm", "long_context_cp"],
                     default="layer",
                     help="decode_step: time only the recurrent decoding step; long_context_cp: "
                          "the long-context sequence split over the ranks (context parallel)")
@@ -658,7 +707,7 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
-    if args.workload == "decode_step":
+    if args.workload in ("decode_step", "gate_norm"):
         return run_decode_only(args)
     if args.workload == "long_context_cp":
         return run_cp(args)

@@ -204,6 +204,26 @@ SSD_API ssd_status_t ssd_step(const ssd_shape_t* shape,
                               const void* B, const void* C, const float* D,
                               float* state, void* y, void* stream);
 
+/*
+ * Gate and normalisation that follow the layer in the Mamba-2 block (Knowl 6,
+ * step 4: the layer output is gated by SiLU of the gate branch z, then
+ * RMS-normalised before the output projection). Per token (b, t) and group of
+ * group_size contiguous channels of its H*P channels (head-major, as y):
+ *     v_c   = y_c * z_c / (1 + exp(-z_c))
+ *     out_c = v_c / sqrt(mean over the group of v^2 + eps) * weight_c
+ *   shape          batch, seqlen, nheads, headdim, dtype are used (the others
+ *                  only have to be valid for ssd_fwd, chunk_size excepted).
+ *   y, z, out      [b, T, H, P] in dtype (16-byte aligned); out must not overlap
+ *                  y, z or weight.
+ *   weight         [H * P] fp32.
+ *   group_size     divides H * P (H * P for one group per token).
+ *   eps            >= 0, finite.
+ * fp32 arithmetic, out rounded once to dtype. One kernel launch.
+ */
+SSD_API ssd_status_t ssd_gated_rmsnorm(const ssd_shape_t* shape, const void* y, const void* z,
+                                       const float* weight, int64_t group_size, float eps,
+                                       void* out, void* stream);
+
 /* ---- Sequence (context) parallelism (Knowl 8: the sequence is split along its
  * length across workers; each runs its slice and only the boundary state
  * travels). ----

@@ -24,7 +24,7 @@ from ._lib import (SSD_BF16, SSD_F32, SSDError, ShapeT, check, lib, lib_path,  #
 
 __all__ = ["ssd_fwd", "ssd_fwd_host", "ssd_fwd_workspace_size", "ssd_fwd_plan", "ssd_fwd_check",
            "ssd_step", "ssd_fwd_cp", "ssd_cp_begin", "ssd_cp_end", "ssd_cp_record_floats",
-           "ssd_chunk_cumsum",
+           "ssd_gated_rmsnorm", "ssd_chunk_cumsum",
            "ssd_chunk_state", "ssd_state_passing", "ssd_chunk_scan", "SSDError", "make_shape",
            "lib_path"]
 
@@ -155,6 +155,27 @@ def ssd_step(x, dt, A, B, C, D, state, y=None, stream=None):
     check(lib().ssd_step(ctypes.byref(shape), _p(x), _p(dt), _p(A), _p(B), _p(C), _p(D),
                          _p(state), _p(y), _stream(stream)), "ssd_step")
     return y.squeeze(1) if one else y
+
+
+def ssd_gated_rmsnorm(y, z, weight, group_size: int | None = None, eps: float = 1e-5, out=None,
+                      stream=None):
+    """out = RMSNorm over channel groups of (y * SiLU(z)), times weight (Knowl 6).
+
+    y, z [b, T, H, P] (same dtype), weight [H * P] fp32; group_size defaults to H * P.
+    """
+    _need(y, "y")
+    _need(z, "z", y.dtype)
+    _need(weight, "weight", torch.float32)
+    b, T, H, P = y.shape
+    if y.dtype not in _DT:
+        raise TypeError(f"y must be float32 or bfloat16, got {y.dtype}")
+    shape = ShapeT(b, T, H, P, 1, 1, 64, _DT[y.dtype], 0)
+    if out is None:
+        out = torch.empty_like(y)
+    gs = H * P if group_size is None else int(group_size)
+    check(lib().ssd_gated_rmsnorm(ctypes.byref(shape), _p(y), _p(z), _p(weight), ctypes.c_int64(gs),
+                                  ctypes.c_float(eps), _p(out), _stream(stream)), "ssd_gated_rmsnorm")
+    return out
 
 
 def ssd_cp_record_floats(shape: ShapeT) -> int:

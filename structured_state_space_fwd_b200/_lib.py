@@ -51,6 +51,8 @@ _SIGS = {
     "ssd_cp_begin": ([ctypes.POINTER(ShapeT)] + [_VP] * 7 + [ctypes.c_size_t, _VP], ctypes.c_int),
     "ssd_cp_end": ([ctypes.POINTER(ShapeT), ctypes.c_int, ctypes.c_int] + [_VP] * 10
                    + [ctypes.c_size_t, _VP], ctypes.c_int),
+    "ssd_gated_rmsnorm": ([ctypes.POINTER(ShapeT), _VP, _VP, _VP, ctypes.c_int64, ctypes.c_float,
+                           _VP, _VP], ctypes.c_int),
     "ssd_chunk_cumsum": ([ctypes.POINTER(ShapeT), _VP, _VP, _VP, _VP], ctypes.c_int),
     "ssd_chunk_state": ([ctypes.POINTER(ShapeT)] + [_VP] * 6, ctypes.c_int),
     "ssd_state_passing": ([ctypes.POINTER(ShapeT)] + [_VP] * 6, ctypes.c_int),

@@ -614,6 +614,31 @@ ssd_status_t ssd_cp_end(const ssd_shape_t* shape, int nranks, int rank, const fl
                                        : ssd::launch_chunk_scan_simt(d, x, dt, B, C, D, cs, entry, y, s));
 }
 
+ssd_status_t ssd_gated_rmsnorm(const ssd_shape_t* shape, const void* y, const void* z,
+                               const float* weight, int64_t group_size, float eps, void* out,
+                               void* stream) {
+    if (!shape) return SSD_ERR_INVALID_ARG;
+    ssd_shape_t s = *shape;
+    s.chunk_size = 64;   // not used
+    ssd_status_t st = check_shape(&s);
+    if (st != SSD_OK) return st;
+    const ssd::Dims d = ssd::make_dims(s);
+    const int64_t C = d.H * d.P;
+    if (group_size < 1 || C % group_size != 0) return SSD_ERR_INVALID_ARG;
+    if (!(eps >= 0.f) || eps > 3.0e38f) return SSD_ERR_INVALID_ARG;   // rejects NaN and inf
+    const Sizes z0 = sizes_of(d);
+    if ((!y && z0.x) || (!z && z0.x) || (!out && z0.x) || !weight) return SSD_ERR_INVALID_ARG;
+    if (!aligned(y, 16) || !aligned(z, 16) || !aligned(out, 16) || !aligned(weight, 4))
+        return SSD_ERR_INVALID_ARG;
+    const Range o{out, z0.x};
+    if (overlaps(o, {y, z0.x}) || overlaps(o, {z, z0.x}) || overlaps(o, {weight, (size_t)C * 4}))
+        return SSD_ERR_INVALID_ARG;
+    // one CTA per group at worst: keep the grid inside its x limit
+    if (d.b * d.T * (C / group_size) > 2147483647LL) return SSD_ERR_UNSUPPORTED;
+    return cuda_status("gated rmsnorm", ssd::launch_gated_rmsnorm(d, y, z, weight, group_size, eps, out,
+                                                                  (cudaStream_t)stream));
+}
+
 ssd_status_t ssd_chunk_cumsum(const ssd_shape_t* shape, const float* dt, const float* A,
                               float* cs, void* stream) {
     ssd_status_t st = check_shape(shape);

@@ -71,6 +71,11 @@ cudaError_t launch_slice_decay(const Dims& d, const float* cs, float* alpha, cud
 cudaError_t launch_cp_fold(const Dims& d, const float* records, int64_t rec_floats, int rank,
                            float* h_in, cudaStream_t st);
 
+// Gate and RMSNorm after the layer: out = (y * SiLU(z)) / rms over groups of group_size
+// channels * weight, for b*T rows of H*P channels.
+cudaError_t launch_gated_rmsnorm(const Dims& d, const void* y, const void* z, const float* w,
+                                 int64_t group_size, float eps, void* out, cudaStream_t st);
+
 // Sets the message ssd_last_error_detail() returns on the calling host thread.
 void set_error_detail(const char* msg);
 

@@ -86,9 +86,12 @@ __device__ __forceinline__ void store_state(float* p, const float (&v)[W]) {
 
 // Thread layout: a warp covers 32 / L rows at a time, L lanes per row; lane j of
 // a row holds the W-wide pieces n0 = (j + k L) W, k < K, of RS rows spaced
-// kStepWarps * 32 / L apart. Grid (row blocks, H, batch).
+// kStepWarps * 32 / L apart. Grid (row blocks, H, batch). With 16-byte pieces
+// the update runs on packed fp32x2 instructions and registers are capped so
+// that 7 CTAs fit on an SM: many small CTAs keep more of the DRAM stream busy
+// than few large ones.
 template <typename E, int W, int K>
-__global__ void __launch_bounds__(kStepWarps * 32) ssd_step_kernel(const StepParams prm) {
+__global__ void __launch_bounds__(kStepWarps * 32, W == 4 ? 7 : 1) ssd_step_kernel(const StepParams prm) {
     constexpr int RS = kStepChunks / K > 0 ? kStepChunks / K : 1;
     const int L = prm.L;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -149,13 +152,30 @@ __global__ void __launch_bounds__(kStepWarps * 32) ssd_step_kernel(const StepPar
             const float xv = row_ok[r] ? to_f32(xt[p]) : 0.f;
             const float u = dtv * xv;
             float acc = 0.f;
+            if constexpr (W == 4) {
+                // packed fp32x2: two state elements per instruction
+                const float2 a2 = make_float2(a, a), u2 = make_float2(u, u);
+                float2 acc2 = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int k = 0; k < K; ++k)
+                for (int k = 0; k < K; ++k)
 #pragma unroll
-                for (int w = 0; w < W; ++w) {
-                    hs[r][k][w] = fmaf(a, hs[r][k][w], u * Bv[k][w]);
-                    acc = fmaf(Cv[k][w], hs[r][k][w], acc);
-                }
+                    for (int w = 0; w < W; w += 2) {
+                        float2 h2 = make_float2(hs[r][k][w], hs[r][k][w + 1]);
+                        h2 = __ffma2_rn(a2, h2, __fmul2_rn(u2, make_float2(Bv[k][w], Bv[k][w + 1])));
+                        acc2 = __ffma2_rn(make_float2(Cv[k][w], Cv[k][w + 1]), h2, acc2);
+                        hs[r][k][w] = h2.x;
+                        hs[r][k][w + 1] = h2.y;
+                    }
+                acc = acc2.x + acc2.y;
+            } else {
+#pragma unroll
+                for (int k = 0; k < K; ++k)
+#pragma unroll
+                    for (int w = 0; w < W; ++w) {
+                        hs[r][k][w] = fmaf(a, hs[r][k][w], u * Bv[k][w]);
+                        acc = fmaf(Cv[k][w], hs[r][k][w], acc);
+                    }
+            }
             // sum over the L lanes of the row (aligned groups of L lanes)
             for (int off = L >> 1; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
             if (j == 0 && row_ok[r]) store_out(yt + p, fmaf(Dh, xv, acc));

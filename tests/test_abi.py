@@ -249,3 +249,21 @@ def test_context_parallel_sizes_and_rejections(L):
     assert end(y=R) == 1                                  # y overlaps the records
     assert end(final=p("x")) == 1
     assert end(ws_bytes=0) == 1
+
+
+def test_gated_rmsnorm_rejections(L):
+    s = shape()
+    bufs = Bufs(s)
+    lib = L.lib()
+
+    def call(y="x", z="C", w="A", gs=256, eps=1e-5, out="y", sh=None):
+        return lib.ssd_gated_rmsnorm(ctypes.byref(sh or s), bufs.p(y) if y else None,
+                                     bufs.p(z) if z else None, bufs.p(w) if w else None,
+                                     ctypes.c_int64(gs), ctypes.c_float(eps),
+                                     bufs.p(out) if out else None, None)
+    # H * P = 256 channels in this shape
+    assert call(gs=0) == 1 and call(gs=100) == 1 and call(gs=512) == 1
+    assert call(eps=-1.0) == 1 and call(eps=float("nan")) == 1 and call(eps=float("inf")) == 1
+    assert call(out=None) == 1 and call(w=None) == 1
+    assert call(out="x") == 1                           # out overlaps y
+    assert call(sh=shape(dtype=9)) == 1
