@@ -217,8 +217,10 @@ SSD_API ssd_status_t ssd_step(const ssd_shape_t* shape,
  *                  y, z or weight.
  *   weight         [H * P] fp32.
  *   group_size     divides H * P (H * P for one group per token).
- *   eps            >= 0, finite.
- * fp32 arithmetic, out rounded once to dtype. One kernel launch.
+ *   eps            >= 0, finite (with eps = 0 a group whose gated values are
+ *                  all 0 gives NaN, 0/0, as the formula does).
+ * fp32 arithmetic (SiLU's exponential and division on the special-function
+ * unit, a few ulp), out rounded once to dtype. One kernel launch.
  */
 SSD_API ssd_status_t ssd_gated_rmsnorm(const ssd_shape_t* shape, const void* y, const void* z,
                                        const float* weight, int64_t group_size, float eps,

@@ -256,6 +256,9 @@ CpWorkspace cp_workspace(const ssd::Dims& d) {
     if (d.b == 0) w.total = 0;
     return w;
 }
+// The rank fold and the state copies run one thread per state element in a 1-D grid.
+constexpr int64_t kMaxFlatStateElems = 256LL * 2147483647LL;
+
 // One rank's record: its slice's state [b,H,P,N], then alpha [b,H], padded to 16 bytes.
 size_t cp_record_floats(const ssd::Dims& d) {
     return align_up((size_t)(d.b * d.H * d.P * d.N + d.b * d.H), 4);
@@ -537,6 +540,7 @@ ssd_status_t ssd_cp_begin(const ssd_shape_t* shape, const void* x, const float* 
         for (const Range& i : ins)
             if (overlaps(o, i)) return SSD_ERR_INVALID_ARG;
     if (overlaps(outs[0], outs[1])) return SSD_ERR_INVALID_ARG;
+    if (d.b * d.H * d.P * d.N > kMaxFlatStateElems) return SSD_ERR_UNSUPPORTED;
     if (d.b == 0) return SSD_OK;
     cudaStream_t s = (cudaStream_t)stream;
     float* alpha = record + d.b * d.H * d.P * d.N;
@@ -590,6 +594,7 @@ ssd_status_t ssd_cp_end(const ssd_shape_t* shape, int nranks, int rank, const fl
     for (int i = 0; i < 3; ++i)
         for (int j = i + 1; j < 3; ++j)
             if (overlaps(outs[i], outs[j])) return SSD_ERR_INVALID_ARG;
+    if (d.b * d.H * d.P * d.N > kMaxFlatStateElems) return SSD_ERR_UNSUPPORTED;
     if (d.b == 0) return SSD_OK;
     cudaStream_t s = (cudaStream_t)stream;
     char* ws = (char*)workspace;
