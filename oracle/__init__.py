@@ -17,7 +17,10 @@ Functions
                   cumulative products of a_t, Knowl 2 step 2).
   chunk_states()  per-chunk states S_c: the recurrence run over chunk c alone
                   from a zero state (Knowl 2, "right factor chunk state").
-  dual_form()     the quadratic (masked attention) form, tiny T only.
+  dual_form()     the quadratic (masked attention) form, tiny T only; optional
+                  resets (a_t = 0) for packed documents.
+  recurrence_varlen()  packed variable-length documents (Knowl 8), each its own
+                  sequence.
   chunked()       the block-decomposition algorithm, step by step, fp64.
   gated_rmsnorm() the gate and RMSNorm after the layer (Knowl 6), fp64.
 Every function is pinned by ``tests/test_oracle.py`` against closed forms,
@@ -160,15 +163,18 @@ def chunk_states(x, dt, A, B, chunk_size):
     return final.reshape(b, nc, H, P, N)
 
 
-def dual_form(x, dt, A, B, C, D=None):
+def dual_form(x, dt, A, B, C, D=None, resets=None):
     """Quadratic (masked attention) form, fp64, one dense T x T matrix per (b, h).
 
     y = (L o (C B^T)) diag(dt) x + D x with the 1-semiseparable mask
     L_ji = prod_{s=i+1}^{j} a_s for j >= i and 0 above the diagonal
     (Knowl 1, dual form; "Mamba-2 and State Space Duality", Y = (L o C B^T) X).
     The products are taken directly, not through exponentials of sums.
+    ``resets`` (bool [b, T], optional) sets a_t = 0 where true, the document
+    boundaries of packed variable-length input (Knowl 8).
     """
     x, dt, A, B, C, D = map(_f64, (x, dt, A, B, C, D))
+    rs = None if resets is None else np.asarray(resets, dtype=bool)
     b, T, H, P = x.shape
     G = B.shape[2]
     hpg = H // G
@@ -177,6 +183,8 @@ def dual_form(x, dt, A, B, C, D=None):
         for h in range(H):
             g = h // hpg
             a = np.exp(dt[bi, :, h] * A[h])
+            if rs is not None:
+                a = np.where(rs[bi], 0.0, a)
             L = np.zeros((T, T))
             for j in range(T):
                 L[j, j] = 1.0
@@ -188,6 +196,32 @@ def dual_form(x, dt, A, B, C, D=None):
             if D is not None:
                 y[bi, :, h, :] += D[h] * x[bi, :, h, :]
     return y
+
+
+def recurrence_varlen(x, dt, A, B, C, D=None, cu_seqlens=None, initial_states=None):
+    """Packed variable-length input (Knowl 8): documents concatenated along the
+    sequence of batch row 0, document k at tokens cu_seqlens[k] .. cu_seqlens[k+1]-1,
+    each run as its own sequence (the state does not cross a boundary).
+
+    x [1, T, H, P], dt [1, T, H], B/C [1, T, G, N]; cu_seqlens [n_docs + 1] with
+    cu_seqlens[0] = 0, non-decreasing, cu_seqlens[-1] = T; initial_states
+    [n_docs, H, P, N] or None. Returns (y [1, T, H, P], final_states [n_docs, H, P, N]).
+    """
+    x, dt, A, B, C, D, init = map(_f64, (x, dt, A, B, C, D, initial_states))
+    cu = [int(v) for v in np.asarray(cu_seqlens).ravel()]
+    if x.shape[0] != 1 or cu[0] != 0 or cu[-1] != x.shape[1] or any(b < a for a, b in zip(cu, cu[1:])):
+        raise ValueError("packed input needs batch 1 and cu_seqlens from 0 to T, non-decreasing")
+    ndoc = len(cu) - 1
+    H, P, N = x.shape[2], x.shape[3], B.shape[3]
+    y = np.zeros_like(x)
+    final = np.zeros((ndoc, H, P, N))
+    for k in range(ndoc):
+        sl = slice(cu[k], cu[k + 1])
+        yk, fk, _ = recurrence(x[:, sl], dt[:, sl], A, B[:, sl], C[:, sl], D,
+                               init[k:k + 1] if init is not None else None)
+        y[:, sl] = yk
+        final[k] = fk[0]
+    return y, final
 
 
 def chunked(x, dt, A, B, C, D=None, chunk_size=64, initial_states=None):

@@ -331,3 +331,49 @@ def test_gated_rmsnorm_hand_example():
     z = np.full_like(y, 60.0)
     out = oracle.gated_rmsnorm(y, z, np.array([2.0, 1.0]), 2, 0.0)
     assert np.allclose(out.ravel(), [2 * 3 / math.sqrt(12.5), 4 / math.sqrt(12.5)], rtol=1e-15)
+
+
+# ---------------------------------------------------------------- packed documents (Knowl 8)
+def _packed(cu, seed, H=2, P=3, G=1, N=4):
+    T = cu[-1]
+    inp = make_inputs(1, T, H, P, G, N, dtype="f32", dt_dist="softplus", seed=seed)
+    inp.pop("initial_states")
+    rng = np.random.Generator(np.random.PCG64(seed + 1))
+    init = rng.standard_normal((len(cu) - 1, H, P, N)) * 0.1
+    return inp, init
+
+
+@pytest.mark.parametrize("cu", [[0, 7, 8, 20, 33], [0, 33], [0, 1, 2, 3, 33], [0, 12, 12, 33]])
+def test_packed_documents_equal_resets_in_dual_form(cu):
+    """Knowl 8 literally: a_t = 0 at each document start in one flat sequence. The dual
+    form with those resets (brute force, products of a) must equal running every
+    document as its own sequence; documents of length 0 and 1 included."""
+    inp, _ = _packed(cu, seed=31)
+    y, _ = oracle.recurrence_varlen(**inp, cu_seqlens=cu)
+    resets = np.zeros((1, cu[-1]), dtype=bool)
+    for s in cu[1:-1]:
+        if s < cu[-1]:
+            resets[0, s] = True
+    y_ref = oracle.dual_form(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"],
+                             resets=resets)
+    assert oracle.rel_err(y, y_ref) < 1e-12
+
+
+def test_packed_documents_are_independent():
+    cu = [0, 9, 21, 33]
+    inp, init = _packed(cu, seed=32)
+    y, fin = oracle.recurrence_varlen(**inp, cu_seqlens=cu, initial_states=init)
+    pert = dict(inp)
+    x = f64(inp["x"]).copy()
+    x[:, 9:21] += 1.0                       # change document 1 only
+    pert["x"] = x
+    init2 = init.copy()
+    init2[1] *= -2.0
+    y2, fin2 = oracle.recurrence_varlen(**pert, cu_seqlens=cu, initial_states=init2)
+    assert np.array_equal(y[:, :9], y2[:, :9]) and np.array_equal(y[:, 21:], y2[:, 21:])
+    assert np.array_equal(fin[[0, 2]], fin2[[0, 2]])
+    assert not np.array_equal(y[:, 9:21], y2[:, 9:21])
+    # one document is the plain recurrence
+    y1, f1 = oracle.recurrence_varlen(**inp, cu_seqlens=[0, 33], initial_states=init[:1])
+    y_ref, f_ref, _ = oracle.recurrence(**inp, initial_states=init[:1])
+    assert np.array_equal(y1, y_ref) and np.array_equal(f1, f_ref)
