@@ -634,10 +634,21 @@ def run_ours(args):
     cp = None
     gate = None
     if not args.profile:
-        decode = measure_decode(ssd, dev, stream, 200, 10, rank,
-                                rank == 0 and world == 1 and not args.no_cpu_baseline)
-        cp = measure_cp_slice(ssd, dev, stream, 50, 5)
-        gate = measure_gate(ssd, dev, stream, 100, 5, seed=rank)
+        # secondary rows, measured after the headline: a failure here is reported in
+        # its own entry and does not take the headline line down with it
+        def guarded(fn, *a, **k):
+            try:
+                return fn(*a, **k)
+            except Exception as e:  # noqa: BLE001
+                try:
+                    torch.cuda.synchronize()
+                except Exception:  # noqa: BLE001
+                    pass
+                return {"error": f"{type(e).__name__}: {e}"[:300]}
+        decode = guarded(measure_decode, ssd, dev, stream, 200, 10, rank,
+                         rank == 0 and world == 1 and not args.no_cpu_baseline)
+        cp = guarded(measure_cp_slice, ssd, dev, stream, 50, 5)
+        gate = guarded(measure_gate, ssd, dev, stream, 100, 5, seed=rank)
 
     if rank == 0:
         line = {
