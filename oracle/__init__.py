@@ -21,6 +21,8 @@ Functions
                   resets (a_t = 0) for packed documents.
   recurrence_varlen()  packed variable-length documents (Knowl 8), each its own
                   sequence.
+  chunked_varlen() the block-decomposition algorithm on packed documents, with
+                  segment-aware decays, step by step (the kernels' blueprint).
   chunked()       the block-decomposition algorithm, step by step, fp64.
   gated_rmsnorm() the gate and RMSNorm after the layer (Knowl 6), fp64.
 Every function is pinned by ``tests/test_oracle.py`` against closed forms,
@@ -315,6 +317,102 @@ def gated_rmsnorm(y, z, weight, group_size, eps):
     ms = np.mean(yg * yg, axis=-1, keepdims=True)
     out = yg / np.sqrt(ms + eps) * w.reshape(C // group_size, group_size)
     return out.reshape(shape)
+
+
+def chunked_varlen(x, dt, A, B, C, D=None, cu_seqlens=None, chunk_size=64, initial_states=None):
+    """Block-decomposition algorithm (Knowl 2) on packed documents (Knowl 8), fp64.
+
+    Same inputs and outputs as ``recurrence_varlen``. The chunk grid ignores the
+    documents; each token carries its document index seg_t, and with cs the plain
+    intra-chunk cumulative sum of dt*A (a_t = 0 at a document start is applied
+    by the segment tests, so no log-decay is ever -inf):
+      * mask: L_ji = exp(cs_j - cs_i) if seg_j == seg_i (j >= i), else 0;
+      * chunk state: only tokens of the chunk's last document count,
+        S_c = sum_{k: seg_k = seg_last} exp(cs_last - cs_k) dt_k x_k B_k^T;
+      * the state entering chunk c belongs to the document of token cQ - 1 and
+        survives to token j only if seg_j is that document: the off-diagonal term
+        exp(cs_j) C_j h_c and the chunk decay exp(cs_last) h_c are kept only then;
+      * a document starting at token s inside chunk c enters its initial state
+        there: tokens j >= s of that document add exp(cs_j - cs_{s-1}) C_j h0
+        (cs_{s-1} = 0 when s is the chunk's first token), and so does the chunk
+        state when that document is the chunk's last;
+      * the state at a document's last token e is the same sum stopped at e.
+    Returns (y, final_states).
+    """
+    x, dt, A, B, C, D, init = map(_f64, (x, dt, A, B, C, D, initial_states))
+    cu = [int(v) for v in np.asarray(cu_seqlens).ravel()]
+    _, T, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    hpg = H // G
+    Q = chunk_size
+    ndoc = len(cu) - 1
+    seg = np.zeros(T, dtype=np.int64)
+    start = np.zeros(T, dtype=bool)
+    for k in range(ndoc):
+        seg[cu[k]:cu[k + 1]] = k
+        if cu[k] < cu[k + 1]:
+            start[cu[k]] = True
+    y = np.zeros_like(x)
+    final = np.zeros((ndoc, H, P, N))
+    for k in range(ndoc):                       # empty documents keep their initial state
+        if cu[k] == cu[k + 1] and init is not None:
+            final[k] = init[k]
+    nc = -(-T // Q)
+    for h in range(H):
+        g = h // hpg
+        hc = np.zeros((P, N))                   # state entering the chunk
+        for c in range(nc):
+            t0, t1 = c * Q, min(T, (c + 1) * Q)
+            n_c = t1 - t0
+            sg = seg[t0:t1]
+            Xc, Bc, Cc = x[0, t0:t1, h], B[0, t0:t1, g], C[0, t0:t1, g]
+            dtc = dt[0, t0:t1, h]
+            cs = np.cumsum(dtc * A[h])
+            prev = seg[t0 - 1] if t0 > 0 else -1   # document of the entering state
+            # the state entering this chunk counts only for the document of token t0-1,
+            # and only until that document ends (a start at t0 ends it at once)
+            keep = (sg == prev) & ~np.logical_or.accumulate(start[t0:t1])
+            # diagonal block, segment-masked
+            L = np.zeros((n_c, n_c))
+            for j in range(n_c):
+                for i in range(j + 1):
+                    if sg[i] == sg[j]:
+                        L[j, i] = np.exp(cs[j] - cs[i])
+            Yc = (L * (Cc @ Bc.T)) @ (dtc[:, None] * Xc)
+            Yc += keep[:, None] * np.exp(cs)[:, None] * (Cc @ hc.T)
+            # initial states of documents starting inside this chunk
+            h0 = {}
+            for s in range(t0, t1):
+                if start[s]:
+                    k = seg[s]
+                    h0[k] = (s - t0, init[k, h] if init is not None else np.zeros((P, N)))
+            for k, (s, hk) in h0.items():
+                base = cs[s - 1] if s > 0 else 0.0
+                for j in range(s, n_c):
+                    if sg[j] == k:
+                        Yc[j] += np.exp(cs[j] - base) * (Cc[j] @ hk.T)
+            y[0, t0:t1, h] = Yc
+            # the state after token j of document k (for document ends and the chunk end)
+            def state_at(j):
+                k = sg[j]
+                st = np.zeros((P, N))
+                if keep[j]:
+                    st += np.exp(cs[j]) * hc
+                if k in h0:
+                    s, hk = h0[k]
+                    st += np.exp(cs[j] - (cs[s - 1] if s > 0 else 0.0)) * hk
+                for i in range(j + 1):
+                    if sg[i] == k:
+                        st += np.exp(cs[j] - cs[i]) * dtc[i] * np.outer(Xc[i], Bc[i])
+                return st
+            for k in set(sg.tolist()):
+                e = cu[k + 1] - 1
+                if t0 <= e < t1:
+                    final[k, h] = state_at(e - t0)
+            hc = state_at(n_c - 1)
+        if D is not None:
+            y[0, :, h] += D[h] * x[0, :, h]
+    return y, final
 
 
 def rel_err(a, ref) -> float:

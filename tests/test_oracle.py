@@ -377,3 +377,18 @@ def test_packed_documents_are_independent():
     y1, f1 = oracle.recurrence_varlen(**inp, cu_seqlens=[0, 33], initial_states=init[:1])
     y_ref, f_ref, _ = oracle.recurrence(**inp, initial_states=init[:1])
     assert np.array_equal(y1, y_ref) and np.array_equal(f1, f_ref)
+
+
+@pytest.mark.parametrize("cu,Q", [([0, 7, 8, 20, 33], 8), ([0, 16, 32, 33], 16), ([0, 1, 2, 3, 33], 4),
+                                  ([0, 12, 12, 33], 5), ([0, 5, 9, 30, 31, 33], 7), ([0, 0, 33], 33)])
+@pytest.mark.parametrize("with_init", [False, True])
+def test_chunked_algorithm_on_packed_documents(cu, Q, with_init):
+    """Knowl 2's chunked algorithm with segment-aware decays (the blueprint for the
+    kernels) equals every document run as its own sequence: documents starting on
+    and off chunk boundaries, several in one chunk, empty and one-token ones."""
+    inp, init = _packed(cu, seed=40 + Q, H=4, P=3, G=2, N=5)
+    ini = init if with_init else None
+    y, f = oracle.recurrence_varlen(**inp, cu_seqlens=cu, initial_states=ini)
+    y2, f2 = oracle.chunked_varlen(**inp, cu_seqlens=cu, chunk_size=Q, initial_states=ini)
+    assert oracle.rel_err(y2, y) < 1e-12
+    assert oracle.rel_err(f2, f) < 1e-12
