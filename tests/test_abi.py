@@ -267,3 +267,9 @@ def test_gated_rmsnorm_rejections(L):
     assert call(out=None) == 1 and call(w=None) == 1
     assert call(out="x") == 1                           # out overlaps y
     assert call(sh=shape(dtype=9)) == 1
+
+
+def test_binding_declares_every_entry_point(L):
+    """The Python binding gives every C entry point of include/ssd.h its signature."""
+    missing = [n for n in declared_functions() if n not in L._SIGS]
+    assert not missing, missing
