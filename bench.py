@@ -316,6 +316,55 @@ def measure_gate(ssd, dev, stream, steps, warmup, seed=0):
             "gpu_launches": steps}
 
 
+# ------------------------------------------------------------------ packed documents
+VARLEN_METRIC = ("SSD fwd Mtokens/s on packed variable-length documents (16 docs, 16384 tokens, "
+                 "2.7B head shape)")
+
+
+def measure_varlen(ssd, dev, stream, steps, warmup, seed=0):
+    """ssd_fwd_varlen on 16 packed documents of mixed lengths (16384 tokens, H80 P64
+    N128 G1 bf16), per-document final states returned. Algorithmic bytes: x, y, dt,
+    B, C of the pack and one final state per document."""
+    w = W.PACKED_DOCS_27B
+    cu = W.packed_cu_seqlens()
+    inp = W.workload_inputs(w, seed=seed)
+    d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+    ndoc = len(cu) - 1
+    y = torch.empty_like(d["x"])
+    fin = torch.empty((ndoc, w.nheads, w.headdim, w.dstate), dtype=torch.float32, device=dev)
+
+    def step():
+        ssd.ssd_fwd_varlen(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], cu_seqlens=cu,
+                           chunk_size=w.chunk_size, return_final_states=True, y=y,
+                           final_states=fin, stream=stream)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    _, by = alg_counts(w, with_final=False)
+    by += 4.0 * ndoc * w.nheads * w.headdim * w.dstate
+    pk, pk_kind = peaks()
+    return {"metric": VARLEN_METRIC, "value": w.tokens / (ms / 1e3) / 1e6, "unit": UNIT,
+            "ms_per_step": ms, "steps": steps, "warmup": warmup, "dtype": "bf16",
+            "config": {"workload": w.name, "documents": ndoc, "doc_lengths": list(W.PACKED_DOC_LENGTHS),
+                       **w.shape_dict(), "input_dtype": w.dtype,
+                       "dispatch": "one ssd_fwd per document on views of the pack"},
+            "roofline": {"kernel": "ssd_fwd per document (16 launches)", "bound": "hbm",
+                         "achieved": by / (ms / 1e3) / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": by / (ms / 1e3) / 1e9 / pk["hbm_gbs"], "traffic": None,
+                         "alg_bytes_per_step": by,
+                         "peak_source": pk_kind + " (burst copy, MEASURED_PEAKS hbm_gbs)"},
+            "gpu_launches": steps * sum(
+                ssd.ssd_fwd_plan(ssd.make_shape(d["x"][:, a:b], d["B"][:, a:b], w.chunk_size))[1]
+                for a, b in zip(cu, cu[1:]))}
+
+
 # ------------------------------------------------------------------ context parallelism
 CP = W.LONG_CONTEXT
 CP_METRIC = ("SSD fwd Mtokens/s, long context (b1 T65536 H32 P64 N128 G8) split over the "
@@ -633,6 +682,7 @@ def run_ours(args):
     decode = None
     cp = None
     gate = None
+    varlen = None
     if not args.profile:
         # secondary rows, measured after the headline: a failure here is reported in
         # its own entry and does not take the headline line down with it
@@ -649,6 +699,7 @@ def run_ours(args):
                          rank == 0 and world == 1 and not args.no_cpu_baseline)
         cp = guarded(measure_cp_slice, ssd, dev, stream, 50, 5)
         gate = guarded(measure_gate, ssd, dev, stream, 100, 5, seed=rank)
+        varlen = guarded(measure_varlen, ssd, dev, stream, 20, 3, seed=rank)
 
     if rank == 0:
         line = {
@@ -667,7 +718,8 @@ def run_ours(args):
             "e2e": e2e,
             "gpu_launches": kernels_per_step * args.steps,
             "clocks": clk,
-            "next_rows": {"decode_step": decode, "context_parallel": cp, "gate_norm": gate},
+            "next_rows": {"decode_step": decode, "context_parallel": cp, "gate_norm": gate,
+                          "packed_docs": varlen},
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -81,6 +81,21 @@ DECODE_STEP_27B = Workload("decode_step_mamba2_2.7b_b128_H80_P64_N128_G1", 128, 
                            128, 256, "bf16", "loguniform", initial_states=True)
 
 
+# packed documents (variable length): 16 documents of mixed lengths, 16384 tokens in
+# all (the 2.7B layer's b*T), at the 2.7B head shape, in batch row 0
+PACKED_DOC_LENGTHS = (2048, 512, 1024, 256, 3072, 768, 1536, 128, 2048, 640, 1408, 896, 1152,
+                      384, 320, 192)
+PACKED_DOCS_27B = Workload("packed_docs_mamba2_2.7b_16docs_T16384_H80_P64_N128_G1", 1,
+                           sum(PACKED_DOC_LENGTHS), 80, 64, 1, 128, 256, "bf16", "loguniform")
+
+
+def packed_cu_seqlens(lengths=PACKED_DOC_LENGTHS) -> list[int]:
+    cu = [0]
+    for n in lengths:
+        cu.append(cu[-1] + n)
+    return cu
+
+
 def all_workloads() -> list[Workload]:
     return [TINY_FP32, MAMBA2_27B_LAYER, *seqlen_sweep(), *dstate_sweep(), LONG_CONTEXT]
 
