@@ -6,7 +6,9 @@ import os
 import threading
 
 PKG = os.path.dirname(os.path.abspath(__file__))
-lib_path = os.path.join(PKG, "libssd.so")
+# SSD_LIBRARY selects another in-tree build of the library to load (the tests use
+# it for libssd_testhooks.so); by default the shipped libssd.so
+lib_path = os.environ.get("SSD_LIBRARY") or os.path.join(PKG, "libssd.so")
 
 SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_CUDA, SSD_ERR_TIMEOUT = range(5)
 SSD_F32, SSD_BF16 = 0, 1

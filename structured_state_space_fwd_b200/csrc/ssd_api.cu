@@ -85,47 +85,84 @@ Sizes sizes_of(const ssd::Dims& d) {
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Which kernels ssd_fwd runs. SSD_PATH=steps forces the four separate steps,
-// SSD_PATH=simt the CUDA-core kernels only (for testing the paths against
-// each other); by default the fused tensor-core kernel runs where supported.
-enum class Path { Fused, Steps, Simt };
+// Which kernels ssd_fwd runs. SSD_PATH (the library's one debug variable) forces a path for
+// testing the paths against each other: "fused", "segmented", "steps" or "simt";
+// a path the shape cannot take falls back to the next one down that list.
+enum class Path { Fused, Segmented, Steps, Simt };
 
-// The fused kernel hands each head's state from tile to tile through a chain
-// across CTAs, so a sequence's tiles are processed one after another. With few
-// independent chains (batch rows x head blocks) and long sequences that chain,
-// not the work, sets the time, and the four separate steps (whose chunk states
-// are computed for all chunks in parallel) are faster: measured on B200 at
-// 32K tokens x 32 heads, fused 454 vs steps 567 us with 32 chains of 64 tiles,
-// fused 866 vs steps 571 us with 16 chains of 128 tiles.
-bool chain_bound(const ssd::Dims& d) {
-    const int64_t kh = ssd::pick_kheads(d.H / d.G);
-    const int64_t chains = d.b * (d.H / kh);
-    const int64_t tiles = (d.T + 127) / 128;
-    return chains < 24 && tiles >= 32;
+const char* path_override() { return getenv("SSD_PATH"); }
+
+// The single-pass tensor-core kernel serves bf16 with head dim 64 and a state
+// dim that is a multiple of 16 up to 256.
+bool fused_ok(const ssd::Dims& d) {
+    return d.dtype == SSD_BF16 && d.P == 64 && ssd::fused_state_capacity(d.N) != 0 &&
+           d.T <= 0x7fffffffLL && ssd::tma_available();
+}
+
+// The single-pass kernel hands each head's state from tile to tile through a
+// chain across CTAs. With few independent chains (batch rows x heads) over many
+// tiles that hand-off, not the work, sets the time; then the sequence is cut
+// into segments whose entering states are computed first (segment states, a
+// scan over them), and the segments run as separate, shorter chains.
+constexpr int64_t kSegmentBelowRowHeads = 300;   // b * H under which long sequences are cut
+constexpr int64_t kSegmentMinTiles = 8;
+constexpr int64_t kTargetChains = 296;           // chains wanted when cutting (2 per SM)
+
+bool prefer_segments(const ssd::Dims& d) {
+    const int64_t ntiles = (d.T + 127) / 128;
+    return ntiles >= kSegmentMinTiles && d.b * d.H < kSegmentBelowRowHeads;
 }
 
 Path pick_path(const ssd::Dims& d) {
-    const char* e = getenv("SSD_PATH");
+    const char* e = path_override();
+    const bool fz = fused_ok(d);
     const bool tc = ssd::tc_supported(d);
     if (e && strcmp(e, "simt") == 0) return Path::Simt;
     if (e && strcmp(e, "steps") == 0) return tc ? Path::Steps : Path::Simt;
-    if (e && strcmp(e, "fused") == 0) return tc ? Path::Fused : Path::Simt;
-    if (!tc) return Path::Simt;
-    return chain_bound(d) ? Path::Steps : Path::Fused;
+    if (e && strcmp(e, "fused") == 0) return fz ? Path::Fused : (tc ? Path::Steps : Path::Simt);
+    if (e && strcmp(e, "segmented") == 0)
+        return fz && d.T > 128 ? Path::Segmented : (fz ? Path::Fused : (tc ? Path::Steps : Path::Simt));
+    if (fz) return prefer_segments(d) ? Path::Segmented : Path::Fused;
+    return tc ? Path::Steps : Path::Simt;
 }
 
 bool steps_use_tc(const ssd::Dims& d) {
-    const char* e = getenv("SSD_PATH");
+    const char* e = path_override();
     return !(e && strcmp(e, "simt") == 0) && ssd::tc_supported(d);
 }
 
+// How the single-pass kernel covers the sequence: heads per unit, tiles per
+// segment, segments (1: one chain over the whole sequence).
+struct SegPlan {
+    int kh, seg_tiles, nseg;
+};
+SegPlan seg_plan(const ssd::Dims& d, Path path) {
+    SegPlan sp;
+    const int ns = ssd::fused_state_capacity(d.N);
+    sp.kh = ssd::fused_kheads(d.H, d.G, ns);
+    const int64_t ntiles = d.T > 0 ? (d.T + 127) / 128 : 1;
+    sp.seg_tiles = (int)std::min<int64_t>(ntiles, 0x7fffffff);
+    sp.nseg = 1;
+    if (path != Path::Segmented || ntiles < 2) return sp;
+    const int64_t chains = std::max<int64_t>(1, d.b * (d.H / sp.kh));
+    int64_t nseg = std::max<int64_t>(2, (kTargetChains + chains - 1) / chains);
+    nseg = std::min(nseg, ntiles);
+    int64_t K = (ntiles + nseg - 1) / nseg;
+    K = std::min<int64_t>(K, ssd::segment_max_tiles());
+    sp.seg_tiles = (int)K;
+    sp.nseg = (int)((ntiles + K - 1) / K);
+    return sp;
+}
+
 // Workspace of ssd_fwd, regions 256-byte aligned:
-//   fused path:  [sync ints: ticket, error, flags[b*H] | chain state [b,H,P,N]]
-//   step paths:  [cs | chunk states S | entry states h_c]
+//   fused / segmented: [sync ints: ticket, error, flags[b*nseg*H] | chain state [b,H,P,N]
+//                       | segment states [b,nseg,H,P,N] | segment decays [b,nseg,H]]
+//   step paths:        [cs | chunk states S | entry states h_c]
 struct FwdWorkspace {
     Path path;
-    size_t off_cs, off_S, off_entry;   // step paths
-    size_t off_sync, off_chain;        // fused path
+    SegPlan sp;
+    size_t off_cs, off_S, off_entry;        // step paths
+    size_t off_sync, off_chain, off_seg, off_decay;  // single-pass paths
     size_t total;
 };
 
@@ -133,10 +170,14 @@ FwdWorkspace fwd_workspace(const ssd::Dims& d) {
     const Sizes z = sizes_of(d);
     FwdWorkspace w = {};
     w.path = pick_path(d);
-    if (w.path == Path::Fused) {
+    if (w.path == Path::Fused || w.path == Path::Segmented) {
+        w.sp = seg_plan(d, w.path);
+        const size_t nseg = (size_t)w.sp.nseg;
         w.off_sync = 0;
-        w.off_chain = align_up(sizeof(int) * (size_t)(2 + d.b * d.H), 256);
-        w.total = w.off_chain + align_up(z.st, 256);
+        w.off_chain = align_up(sizeof(int) * ssd::fused_sync_ints(d, w.sp.nseg), 256);
+        w.off_seg = w.off_chain + align_up(z.st, 256);
+        w.off_decay = w.off_seg + (nseg > 1 ? align_up(z.st * nseg, 256) : 0);
+        w.total = w.off_decay + (nseg > 1 ? align_up((size_t)(d.b * d.H) * nseg * 4, 256) : 0);
     } else {
         w.off_cs = 0;
         w.off_S = align_up(z.cs, 256);
@@ -187,6 +228,16 @@ ssd_status_t check_fwd_args(const ssd_shape_t* shape, const void* x, const float
     return SSD_OK;
 }
 
+// test builds: SSD_TEST_STALL_CHAIN=1 makes every chain hand-off wait run out
+int test_stall() {
+#ifdef SSD_TEST_HOOKS
+    const char* v = getenv("SSD_TEST_STALL_CHAIN");
+    return (v && v[0] == '1') ? 1 : 0;
+#else
+    return 0;
+#endif
+}
+
 ssd_status_t run_fwd(const ssd::Dims& d, const void* x, const float* dt, const float* A,
                      const void* B, const void* C, const float* D, const float* init, void* y,
                      float* final_states, void* workspace, cudaStream_t stream) {
@@ -194,17 +245,49 @@ ssd_status_t run_fwd(const ssd::Dims& d, const void* x, const float* dt, const f
     if (d.T == 0) return cuda_status("final states", ssd::launch_copy_or_zero_states(d, init, final_states, stream));
     const FwdWorkspace w = fwd_workspace(d);
     char* ws = (char*)workspace;
-    if (w.path == Path::Fused) {
-        float* chain = final_states ? final_states : (float*)(ws + w.off_chain);
-        return cuda_status("fused forward",
-                           ssd::launch_fused_tc(d, x, dt, A, B, C, D, init, y, chain,
-                                                (int*)(ws + w.off_sync), stream));
+    ssd_status_t st;
+    if (w.path == Path::Fused || w.path == Path::Segmented) {
+        CUtensorMap maps[4];
+        if (!ssd::make_tc_maps(d, x, B, C, y, maps)) {
+            ssd::set_error_detail("tensor map encoding failed");
+            return SSD_ERR_CUDA;
+        }
+        int* sync = (int*)(ws + w.off_sync);
+        if ((st = cuda_status("sync area", cudaMemsetAsync(sync, 0, sizeof(int) * ssd::fused_sync_ints(d, w.sp.nseg),
+                                                           stream))) != SSD_OK)
+            return st;
+        float* segbuf = w.sp.nseg > 1 ? (float*)(ws + w.off_seg) : nullptr;
+        if (w.sp.nseg > 1) {
+            float* decay = (float*)(ws + w.off_decay);
+            if ((st = cuda_status("segment states",
+                                  ssd::launch_segment_states(d, maps, dt, A, segbuf, decay, sync + 1, w.sp.seg_tiles,
+                                                             w.sp.nseg, w.sp.nseg, w.sp.nseg - 1,
+                                                             ssd::pick_kheads(d.H / d.G), stream))) != SSD_OK)
+                return st;
+            if ((st = cuda_status("segment scan", ssd::launch_segment_scan(d, init, segbuf, decay, w.sp.nseg, w.sp.nseg,
+                                                                           w.sp.nseg - 1, nullptr, stream))) != SSD_OK)
+                return st;
+        }
+        ssd::FusedLaunch a = {};
+        a.d = d;
+        a.maps = maps;
+        a.dt = dt;
+        a.A = A;
+        a.D = D;
+        a.init = init;
+        a.finalbuf = final_states ? final_states : (float*)(ws + w.off_chain);
+        a.segbuf = segbuf;
+        a.sync_ints = sync;
+        a.kheads = w.sp.kh;
+        a.seg_tiles = w.sp.seg_tiles;
+        a.nseg = w.sp.nseg;
+        a.stall = test_stall();
+        return cuda_status("fused forward", ssd::launch_fused(a, stream));
     }
     float* cs = (float*)(ws + w.off_cs);
     float* S = (float*)(ws + w.off_S);
     float* entry = (float*)(ws + w.off_entry);
     const bool tc = w.path == Path::Steps;
-    ssd_status_t st;
     if ((st = cuda_status("chunk cumsum", ssd::launch_chunk_cumsum(d, dt, A, cs, stream))) != SSD_OK)
         return st;
     if ((st = cuda_status("chunk state",
@@ -223,7 +306,8 @@ ssd_status_t run_fwd(const ssd::Dims& d, const void* x, const float* dt, const f
 // used this workspace: waits for `s`, then maps a nonzero word to SSD_ERR_TIMEOUT.
 ssd_status_t read_device_status(const ssd::Dims& d, const void* workspace, cudaStream_t s) {
     const FwdWorkspace w = fwd_workspace(d);
-    if (w.path != Path::Fused || w.total == 0 || d.b == 0 || d.T == 0) return SSD_OK;
+    if ((w.path != Path::Fused && w.path != Path::Segmented) || w.total == 0 || d.b == 0 || d.T == 0)
+        return SSD_OK;
     int word = 0;
     ssd_status_t st;
     const int* dev = (const int*)((const char*)workspace + w.off_sync) + 1;
@@ -316,8 +400,8 @@ ssd_status_t ssd_fwd_plan(const ssd_shape_t* shape, const char** path, int* kern
     if (st != SSD_OK) return st;
     const ssd::Dims d = ssd::make_dims(*shape);
     const Path p = pick_path(d);
-    *path = p == Path::Fused ? "fused" : (p == Path::Steps ? "steps" : "simt");
-    *kernels = (d.b == 0) ? 0 : (d.T == 0 ? 1 : (p == Path::Fused ? 1 : 4));
+    *path = p == Path::Fused ? "fused" : p == Path::Segmented ? "segmented" : p == Path::Steps ? "steps" : "simt";
+    *kernels = (d.b == 0) ? 0 : (d.T == 0 ? 1 : (p == Path::Fused ? 1 : p == Path::Segmented ? 3 : 4));
     return SSD_OK;
 }
 

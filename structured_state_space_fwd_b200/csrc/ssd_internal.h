@@ -35,24 +35,54 @@ cudaError_t launch_chunk_scan_simt(const Dims& d, const void* x, const float* dt
                                    const float* entry, void* y, cudaStream_t st);
 // Tensor-core path (sm_100a tcgen05): bf16, head dim 64, state dim 128, chunk 128/256.
 bool tc_supported(const Dims& d);
+// cuTensorMapEncodeTiled is reachable through the runtime's driver entry points.
+bool tma_available();
 cudaError_t launch_chunk_state_tc(const Dims& d, const void* x, const float* dt, const void* B,
                                   const float* cs, float* states, cudaStream_t st);
 cudaError_t launch_chunk_scan_tc(const Dims& d, const void* x, const float* dt, const void* B,
                                  const void* C, const float* D, const float* cs,
                                  const float* entry, void* y, cudaStream_t st);
-// Whole forward in one kernel; sync_ints holds 2 + b*H ints, chain b*H*P*N floats.
-cudaError_t launch_fused_tc(const Dims& d, const void* x, const float* dt, const float* A,
-                            const void* B, const void* C, const float* D, const float* init,
-                            void* y, float* chain, int* sync_ints, cudaStream_t st);
-
 int pick_kheads(int64_t heads_per_group);
 // TMA maps of x, B, C (bf16, 4-D, 64 x 1 x 128 x 1 boxes) and y (64 x 1 x 32 x 1 boxes),
 // 128-byte swizzle.
 bool make_tc_maps(const Dims& d, const void* x, const void* B, const void* C, const void* y,
                   CUtensorMap* maps);
-cudaError_t launch_fused_ws(const Dims& d, const CUtensorMap* maps, const void* x, const float* dt,
-                            const float* A, const float* D, const float* init, void* y,
-                            float* chain, int* sync_ints, int kheads, cudaStream_t st);
+
+// Single-pass forward (ssd_fused.cu): bf16, head dim 64, state dim a multiple of 16
+// up to 256. State capacity of the kernel variant for N (128 or 256; 0: unsupported).
+int fused_state_capacity(int64_t N);
+int fused_kheads(int64_t H, int64_t G, int ns);
+// ints of the kernel's sync area: ticket, error word, one flag per (b, segment, head)
+size_t fused_sync_ints(const Dims& d, int nseg);
+struct FusedLaunch {
+    Dims d;
+    const CUtensorMap* maps;   // x, B, C, y
+    const float* dt;
+    const float* A;
+    const float* D;
+    const float* init;         // [b,H,P,N] or null
+    float* finalbuf;           // [b,H,P,N]: the last segment's chain, final states on return
+    float* segbuf;             // [b,nseg,H,P,N] states entering segments 1.. (nseg > 1)
+    int* sync_ints;            // fused_sync_ints ints, zeroed by the launch
+    int kheads, seg_tiles, nseg;
+    int stall;                 // test builds: make chain waits run out
+};
+cudaError_t launch_fused(const FusedLaunch& a, cudaStream_t st);
+
+// Segment states (ssd_segment.cu): for each segment s < nseg_out of seg_tiles tiles,
+// the state it reaches from zero, written to segbuf slot s + 1 ([b,nslot,H,P,N]), and
+// its decay 2^(sum dt A log2 e) to decay[b,nseg,H] at s. The scan over segments then
+// turns slot s (1 <= s <= nseg_out) into the state entering segment s (init entering
+// segment 0) and, when `final_out` is given, writes the state after segment
+// nseg_out - 1 there. Bounded waits that give up set *error.
+int segment_max_tiles();
+cudaError_t launch_segment_states(const Dims& d, const CUtensorMap* maps, const float* dt,
+                                  const float* A, float* segbuf, float* decay, int* error,
+                                  int seg_tiles, int nseg, int nslot, int nseg_out, int kheads,
+                                  cudaStream_t st);
+cudaError_t launch_segment_scan(const Dims& d, const float* init, float* segbuf, const float* decay,
+                                int nseg, int nslot, int nseg_out, float* final_out,
+                                cudaStream_t st);
 
 // Recurrent form for a few tokens per sequence, state [b,H,P,N] updated in place.
 struct StepLayout {

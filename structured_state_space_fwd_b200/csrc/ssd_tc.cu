@@ -1,15 +1,10 @@
 // Tensor-core (tcgen05 / TMEM / TMA) kernels of the SSD forward for sm_100a.
 //
-// One kernel template covers three steps of the block-decomposition algorithm
+// One kernel template covers two steps of the block-decomposition algorithm
 // ("Transformers are SSMs: Generalized Models and Efficient Algorithms Through
-// Structured State Space Duality", Knowl 2):
+// Structured State Space Duality", Knowl 2) as separately callable steps:
 //   kModeState  step 2, chunk states S_c = B_c^T (decayed X_c)
 //   kModeScan   step 4, Y_c = (L o C B^T) dt X + decayed C h_c + D X, h_c given
-//   kModeFused  steps 1-4 in one pass: the state entering chunk c is taken
-//               from the CTA that processed chunk c-1 of the same heads and the
-//               state leaving chunk c is handed on (Knowl 2's sequential loop
-//               over chunks, done as a chain across CTAs through one
-//               L2-resident [b, H, P, N] buffer).
 //
 // Work unit: (chunk c, batch row b, block of `kheads` heads of one group). The
 // chunk's B and C tiles and its C B^T blocks (computed once on the tensor
@@ -74,34 +69,20 @@ constexpr uint32_t kTmemCols = 512;
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-enum Mode { kModeState = 0, kModeScan = 1, kModeFused = 2 };
+enum Mode { kModeState = 0, kModeScan = 1 };
 
 struct TcParams {
     const __nv_bfloat16* x;
     const float* dt;
-    const float* A;
     const float* D;
     const float* cs;          // step inputs [b,H,nc,Q] (state / scan modes)
-    const float* init;        // fused: initial states or null
     const float* entry;       // scan: states entering each chunk [b,nc,H,P,N]
     float* states_out;        // state mode: chunk states [b,nc,H,P,N]
-    float* chain;             // fused: [b,H,P,N] running state, final state at the end
     __nv_bfloat16* y;
-    int* flags;               // fused: [b*H] number of chunks whose state is published
-    int* ticket;              // fused: next unit to take
-    int* error;               // fused: set when a bounded wait gives up
+    int* error;               // set when a bounded wait gives up (may be null)
     int64_t T, H, G, nc;
     int Q, kheads, batch;
 };
-
-__device__ __forceinline__ int ld_acquire(const int* p) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_release(int* p, int v) {
-    asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -133,7 +114,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* bar_mma = bar_bc + 2;
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bar_bc + 4);
     int* s_unit = reinterpret_cast<int*>(s_tmem + 1);
-    int* s_ok = s_unit + 1;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     (void)lane;
@@ -145,7 +125,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tm_x);
         prefetch_tmap(&tm_B);
         if (kMode != kModeState) prefetch_tmap(&tm_C);
-        *s_unit = (kMode == kModeFused) ? atomicAdd(prm.ticket, 1) : (int)blockIdx.x;
+        *s_unit = (int)blockIdx.x;
     }
     if (warp == 0) tmem_alloc(s_tmem, kTmemCols);
     tc_fence_before();
@@ -208,7 +188,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     for (int kh = 0; kh < kh_n; ++kh) {
         const int h = hb * kh_n + kh;
-        const float A_h = prm.A[h];
         const float D_h = prm.D ? prm.D[h] : 0.f;
         const int64_t PN = (int64_t)kP * kN;
         float hreg[kP];  // thread n holds h[p][n] for p = 0..63
@@ -217,33 +196,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (kMode == kModeState) {
 #pragma unroll
             for (int p = 0; p < kP; ++p) hreg[p] = 0.f;
-        } else if (kMode == kModeScan) {
+        } else {
             const float* src = prm.entry + (((int64_t)bi * nc + c) * H + h) * PN + tid;
 #pragma unroll
             for (int p = 0; p < kP; ++p) hreg[p] = __ldg(src + (int64_t)p * kN);
-        } else {
-            if (c == 0) {
-                const float* src = prm.init ? prm.init + ((int64_t)bi * H + h) * PN + tid : nullptr;
-#pragma unroll
-                for (int p = 0; p < kP; ++p) hreg[p] = src ? __ldg(src + (int64_t)p * kN) : 0.f;
-            } else {
-                if (tid == 0) {
-                    const int* f = prm.flags + (int64_t)bi * H + h;
-                    int ok = 0;
-                    for (uint32_t it = 0; it < (1u << 25); ++it) {
-                        if (ld_acquire(f) >= c) { ok = 1; break; }
-                        __nanosleep(64);
-                    }
-                    if (!ok) atomicExch(prm.error, 1);
-                    *s_ok = ok;
-                }
-                __syncthreads();
-                __threadfence();
-                const float* src = prm.chain + ((int64_t)bi * H + h) * PN + tid;
-                const float bad = *s_ok ? 0.f : __int_as_float(0x7fc00000);
-#pragma unroll
-                for (int p = 0; p < kP; ++p) hreg[p] = __ldcg(src + (int64_t)p * kN) + bad;
-            }
         }
 
         for (int s = 0; s < nsub; ++s) {
@@ -260,24 +216,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // ---- cumulative sum of dt*A over the tile (log2 units), inclusive
             float dtv = 0.f, v;
-            if (kMode == kModeFused) {
-                if (tid < len) dtv = prm.dt[((int64_t)bi * T + t0 + tid) * H + h];
-                v = dtv * A_h * kLog2e;
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const float o = __shfl_up_sync(0xffffffffu, v, off);
-                    if ((tid & 31) >= off) v += o;
-                }
-                if ((tid & 31) == 31) s_wsum[warp] = v;
-                __syncthreads();
-                for (int w = 0; w < warp; ++w) v += s_wsum[w];
-            } else {
-                // cs of the step interface: chunk-relative natural-log sums; rebase to the tile
-                const float* csc = prm.cs + (((int64_t)bi * H + h) * nc + c) * Q + s * kTile;
-                const float base = s > 0 ? csc[-1] : 0.f;
-                if (tid < len) dtv = prm.dt[((int64_t)bi * T + t0 + tid) * H + h];
-                v = (csc[min(tid, len - 1)] - base) * kLog2e;
-            }
+            // cs of the step interface: chunk-relative natural-log sums; rebase to the tile
+            const float* csc = prm.cs + (((int64_t)bi * H + h) * nc + c) * Q + s * kTile;
+            const float base = s > 0 ? csc[-1] : 0.f;
+            if (tid < len) dtv = prm.dt[((int64_t)bi * T + t0 + tid) * H + h];
+            v = (csc[min(tid, len - 1)] - base) * kLog2e;
             s_cs[tid] = v;
             s_dt[tid] = dtv;
             __syncthreads();
@@ -437,13 +380,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             float* dst = prm.states_out + (((int64_t)bi * nc + c) * H + h) * PN + tid;
 #pragma unroll
             for (int p = 0; p < kP; ++p) dst[(int64_t)p * kN] = hreg[p];
-        } else if (kMode == kModeFused) {
-            float* dst = prm.chain + ((int64_t)bi * H + h) * PN + tid;
-#pragma unroll
-            for (int p = 0; p < kP; ++p) __stcg(dst + (int64_t)p * kN, hreg[p]);
-            __threadfence();
-            __syncthreads();
-            if (tid == 0) st_release(prm.flags + (int64_t)bi * H + h, c + 1);
         }
     }
 
@@ -528,6 +464,8 @@ cudaError_t launch_tc(const Dims& d, TcParams prm, const void* x, const void* B,
 
 }  // namespace
 
+bool tma_available() { return encode_fn() != nullptr; }
+
 bool tc_supported(const Dims& d) {
     return d.dtype == SSD_BF16 && d.P == kP && d.N == kN && (d.Q == 128 || d.Q == 256) &&
            d.T <= 0x7fffffffLL && d.b <= 0x7fffffffLL && d.nc * d.b * d.H < 0x7fffffffLL &&
@@ -555,34 +493,6 @@ cudaError_t launch_chunk_scan_tc(const Dims& d, const void* x, const float* dt, 
     prm.entry = entry;
     prm.y = (__nv_bfloat16*)y;
     return launch_tc<kModeScan>(d, prm, x, B, C, st);
-}
-
-cudaError_t launch_fused_tc(const Dims& d, const void* x, const float* dt, const float* A,
-                            const void* B, const void* C, const float* D, const float* init,
-                            void* y, float* chain, int* sync_ints, cudaStream_t st) {
-    // sync_ints: [0] ticket, [1] error, [2 ..] flags[b*H]; zeroed here.
-    cudaError_t e = cudaMemsetAsync(sync_ints, 0, sizeof(int) * (size_t)(2 + d.b * d.H), st);
-    if (e != cudaSuccess) return e;
-    const char* v = getenv("SSD_FUSED");
-    if (!(v && strcmp(v, "v0") == 0)) {
-        // default: the warp-specialized persistent kernel (ssd_fused.cu)
-        CUtensorMap maps[4];
-        if (!make_tc_maps(d, x, B, C, y, maps)) return cudaErrorInvalidValue;
-        return launch_fused_ws(d, maps, x, dt, A, D, init, y, chain, sync_ints,
-                               pick_kheads(d.H / d.G), st);
-    }
-    TcParams prm = {};
-    prm.x = (const __nv_bfloat16*)x;
-    prm.dt = dt;
-    prm.A = A;
-    prm.D = D;
-    prm.init = init;
-    prm.chain = chain;
-    prm.y = (__nv_bfloat16*)y;
-    prm.ticket = sync_ints;
-    prm.error = sync_ints + 1;
-    prm.flags = sync_ints + 2;
-    return launch_tc<kModeFused>(d, prm, x, B, C, st);
 }
 
 }  // namespace ssd

@@ -2,8 +2,9 @@
 
 Metric: max|y - y_ref| / max|y_ref| over the compared elements, the same for
 final states. Bars: 5e-3 for bf16 storage (fp32 accumulation), 1e-5 for the
-fp32 path. Small cases compare every element; full-size workloads compare
-whole (batch, head) sequences the oracle computes one by one.
+fp32 path. Every test compares every element of y and of the final states with
+the oracle's recurrence (the definition of the layer), full-size workloads
+included.
 """
 import numpy as np
 import pytest
@@ -16,6 +17,7 @@ from ssd_inputs import make_inputs
 pytestmark = pytest.mark.gpu
 
 TOL = {"f32": 1e-5, "bf16": 5e-3}
+TENSOR_PATHS = ["fused", "segmented", "steps"]
 
 
 @pytest.fixture(scope="module")
@@ -24,6 +26,16 @@ def ssd(cuda_device):
     build.build()
     import structured_state_space_fwd_b200 as m
     return m
+
+
+@pytest.fixture
+def path_env(monkeypatch):
+    def set_path(p):
+        if p is None:
+            monkeypatch.delenv("SSD_PATH", raising=False)
+        else:
+            monkeypatch.setenv("SSD_PATH", p)
+    return set_path
 
 
 def to_dev(inp):
@@ -38,12 +50,19 @@ def run(ssd, inp, Q, final=True):
     return out
 
 
-def check_full(ssd, inp, Q, dtype, tol=None):
+def plan_of(ssd, inp, Q):
+    return ssd.ssd_fwd_plan(ssd.make_shape(inp["x"], inp["B"], Q))[0]
+
+
+def check_full(ssd, inp, Q, dtype, tol=None, ref=None):
     tol = tol or TOL[dtype]
     y, fin = run(ssd, inp, Q)
-    y_ref, f_ref, _ = oracle.recurrence(**inp)
-    ey = oracle.rel_err(y.float().cpu(), y_ref)
-    ef = oracle.rel_err(fin.cpu(), f_ref)
+    y_ref, f_ref, _ = ref if ref is not None else oracle.recurrence(**inp)
+    yc = y.float().cpu()
+    fc = fin.cpu()
+    assert torch.isfinite(yc).all() and torch.isfinite(fc).all()
+    ey = oracle.rel_err(yc, y_ref)
+    ef = oracle.rel_err(fc, f_ref)
     assert ey <= tol, f"y rel err {ey:.3e} > {tol}"
     assert ef <= tol, f"final rel err {ef:.3e} > {tol}"
     return ey, ef
@@ -162,8 +181,10 @@ def test_continuation_on_gpu(ssd):
     assert oracle.rel_err(f2.cpu(), f.cpu()) <= 1e-5
 
 
-def test_deterministic(ssd):
-    inp = make_inputs(batch=2, seqlen=512, nheads=4, headdim=64, ngroups=1, dstate=128,
+@pytest.mark.parametrize("path", TENSOR_PATHS)
+def test_deterministic(ssd, path_env, path):
+    path_env(path)
+    inp = make_inputs(batch=2, seqlen=1500, nheads=8, headdim=64, ngroups=1, dstate=128,
                       dtype="bf16", initial_states=True, seed=1)
     y1, f1 = run(ssd, inp, 256)
     y2, f2 = run(ssd, inp, 256)
@@ -183,60 +204,13 @@ def test_host_buffer_entry_point(ssd):
     assert torch.equal(y, yd.cpu()) and torch.equal(fin, fd.cpu())
 
 
-# ---------------------------------------------------------------- full size
-def sampled_check(ssd, w, pairs, seed=0):
-    inp = W.workload_inputs(w, seed=seed)
-    y, fin = run(ssd, inp, w.chunk_size)
-    y_ref, f_ref, _ = oracle.recurrence(**inp, bh_list=pairs)
-    yc = y.float().cpu().numpy()
-    fc = fin.cpu().numpy()
-    ys = np.stack([yc[b, :, h] for b, h in pairs])
-    yr = np.stack([y_ref[b, :, h] for b, h in pairs])
-    fs = np.stack([fc[b, h] for b, h in pairs])
-    fr = np.stack([f_ref[b, h] for b, h in pairs])
-    ey, ef = oracle.rel_err(ys, yr), oracle.rel_err(fs, fr)
-    assert np.isfinite(yc).all() and np.isfinite(fc).all()
-    assert ey <= TOL[w.dtype], f"{w.name}: y rel err {ey:.3e}"
-    assert ef <= TOL[w.dtype], f"{w.name}: final rel err {ef:.3e}"
-    return ey, ef
-
-
-def corners(b, H):
-    return sorted({(0, 0), (b - 1, H - 1), (b // 2, H // 2), (0, H - 1), (b - 1, 0)})
-
-
-def test_full_mamba2_layer(ssd):
-    w = W.MAMBA2_27B_LAYER
-    sampled_check(ssd, w, corners(w.batch, w.nheads) + [(3, 41)])
-
-
-@pytest.mark.parametrize("w", W.seqlen_sweep(), ids=lambda w: w.name)
-def test_full_seqlen_sweep(ssd, w):
-    sampled_check(ssd, w, corners(w.batch, w.nheads)[:3])
-
-
-@pytest.mark.parametrize("w", W.dstate_sweep(), ids=lambda w: w.name)
-def test_full_dstate_sweep(ssd, w):
-    sampled_check(ssd, w, corners(w.batch, w.nheads)[:3])
-
-
-def test_full_long_context(ssd):
-    w = W.LONG_CONTEXT
-    sampled_check(ssd, w, [(0, 0), (0, 5), (0, 18), (0, 31)])
-
-
-# ---------------------------------------------------------------- tensor-core path
-# bf16, head dim 64, state dim 128, chunk 128 or 256 run on the tcgen05 kernels:
-# the fused kernel (SSD_PATH=fused forces it; by default it is chosen unless the
-# shape has few long chains), the separate tensor-core steps with SSD_PATH=steps.
-@pytest.fixture
-def path_env(monkeypatch):
-    def set_path(p):
-        monkeypatch.setenv("SSD_PATH", p)
-    return set_path
-
-
-@pytest.mark.parametrize("path", ["fused", "steps"])
+# ---------------------------------------------------------------- tensor-core paths
+# bf16 with head dim 64 and a state dim that is a multiple of 16 up to 256 runs on
+# the tcgen05 single-pass kernel: one chain over the sequence ("fused") or the
+# sequence cut into segments whose entering states are computed first
+# ("segmented"); SSD_PATH forces either, and "steps" the four separate steps
+# (tensor cores for state dim 128).
+@pytest.mark.parametrize("path", TENSOR_PATHS)
 @pytest.mark.parametrize("Q", [128, 256])
 @pytest.mark.parametrize("T", [1, 100, 256, 700, 1300])
 def test_tensor_path_ragged(ssd, path_env, path, Q, T):
@@ -246,8 +220,8 @@ def test_tensor_path_ragged(ssd, path_env, path, Q, T):
     check_full(ssd, inp, Q, "bf16")
 
 
-@pytest.mark.parametrize("path", ["fused", "steps"])
-@pytest.mark.parametrize("H,G", [(1, 1), (3, 1), (6, 3), (5, 5), (12, 1)])
+@pytest.mark.parametrize("path", TENSOR_PATHS)
+@pytest.mark.parametrize("H,G", [(1, 1), (3, 1), (6, 3), (5, 5), (12, 1), (16, 2)])
 def test_tensor_path_head_blocks(ssd, path_env, path, H, G):
     path_env(path)
     inp = make_inputs(batch=3, seqlen=520, nheads=H, headdim=64, ngroups=G, dstate=128,
@@ -255,19 +229,73 @@ def test_tensor_path_head_blocks(ssd, path_env, path, H, G):
     check_full(ssd, inp, 256, "bf16")
 
 
-@pytest.mark.parametrize("path", ["fused", "steps"])
+@pytest.mark.parametrize("path", ["fused", "segmented"])
+@pytest.mark.parametrize("N", [16, 32, 64, 80, 128, 176, 256])
+@pytest.mark.parametrize("H,G", [(4, 1), (8, 2), (16, 1)])
+def test_tensor_path_state_sizes(ssd, path_env, path, N, H, G):
+    # every state size on tensor cores: one, two or four 64-wide column blocks of
+    # B and C, partial blocks (80, 176), and the 256-wide kernel variant
+    path_env(path)
+    inp = make_inputs(batch=2, seqlen=900, nheads=H, headdim=64, ngroups=G, dstate=N,
+                      dtype="bf16", initial_states=True, seed=N + H)
+    assert plan_of(ssd, inp, 256) == path
+    check_full(ssd, inp, 256, "bf16")
+
+
+@pytest.mark.parametrize("path", TENSOR_PATHS)
 @pytest.mark.parametrize("scale", [8.0, 64.0])
 def test_tensor_path_strong_decay(ssd, path_env, path, scale):
-    # Every other head decays `scale` times faster, so that one 32-token block spans
-    # far more than 2^64 of decay: the masked diagonal block then takes its
-    # exponents element by element instead of in factored form. The other heads
-    # keep the mild decay of the standard draw.
+    # Every other head decays `scale` times faster, so that a unit's heads decay by
+    # far more than 2^96 over one 128-token tile: such units take the unfactored
+    # masked product (exponent per element) and a separate state-term product.
     path_env(path)
     inp = make_inputs(batch=2, seqlen=700, nheads=8, headdim=64, ngroups=2, dstate=128,
                       dtype="bf16", initial_states=True, seed=int(scale))
     A = inp["A"].clone()
     A[::2] *= scale
     inp["A"] = A
+    check_full(ssd, inp, 256, "bf16")
+
+
+@pytest.mark.parametrize("path", ["fused", "segmented"])
+@pytest.mark.parametrize("N", [64, 256])
+def test_tensor_path_mixed_decay_units(ssd, path_env, path, N):
+    # units of both forms interleaved in one launch: head blocks with mild decay
+    # next to head blocks whose decay over a tile exceeds 2^96
+    path_env(path)
+    inp = make_inputs(batch=2, seqlen=1100, nheads=16, headdim=64, ngroups=1, dstate=N,
+                      dtype="bf16", initial_states=True, seed=77 + N)
+    A = inp["A"].clone()
+    A[4:8] = -40.0
+    A[12:14] = -25.0
+    inp["A"] = A
+    check_full(ssd, inp, 256, "bf16")
+
+
+@pytest.mark.parametrize("path", TENSOR_PATHS + ["simt"])
+def test_zero_decay_is_causal_linear_attention(ssd, path_env, path):
+    # A = 0: every a_t = 1, the mask is the all-ones lower triangle and the layer is
+    # causal linear attention y_j = sum_{i<=j} (C_j . B_i) dt_i x_i + D x_j
+    # ("Mamba-2 and State Space Duality", the dual form with L = 1). The oracle's
+    # reference here is its independent triple loop for that case.
+    path_env(path)
+    inp = make_inputs(batch=2, seqlen=384, nheads=4, headdim=64, ngroups=1, dstate=64,
+                      dtype="bf16", seed=123)
+    inp["A"] = torch.zeros_like(inp["A"])
+    x, dt, B, C, D = (oracle._f64(inp[k]) for k in ("x", "dt", "B", "C", "D"))
+    G = np.einsum("btgn,bsgn->bgts", C, B)                    # C_j . B_i
+    M = np.tril(np.ones((x.shape[1], x.shape[1])))
+    y_ref = np.einsum("bgts,ts,bsh,bshp->bthp", G, M, dt, x) + D[None, None, :, None] * x
+    f_ref = np.einsum("bsh,bshp,bsgn->bhpn", dt, x, B)
+    check_full(ssd, inp, 128, "bf16", ref=(y_ref, f_ref, None))
+
+
+def test_segmented_several_tiles_per_segment(ssd, path_env):
+    # 200 tiles per sequence and 4 chains: segments of 3 tiles, 67 segments per
+    # chain, the last one short, entering states from the segment scan
+    path_env("segmented")
+    inp = make_inputs(batch=2, seqlen=128 * 200 - 37, nheads=8, headdim=64, ngroups=2, dstate=128,
+                      dtype="bf16", initial_states=True, seed=808)
     check_full(ssd, inp, 256, "bf16")
 
 
@@ -290,33 +318,28 @@ def test_tensor_steps_against_oracle(ssd, path_env):
     assert oracle.rel_err(y.float().cpu(), y_ref) <= 5e-3
 
 
-def test_path_choice(ssd, monkeypatch):
-    # fused kernel unless the shape has few independent chains of many tiles
-    monkeypatch.delenv("SSD_PATH", raising=False)
-    def plan(w):
-        return ssd.ssd_fwd_plan(ssd.ShapeT(w.batch, w.seqlen, w.nheads, w.headdim, w.ngroups,
-                                           w.dstate, w.chunk_size, ssd.SSD_BF16, 0))[0]
-    assert plan(W.MAMBA2_27B_LAYER) == "fused"
-    assert plan(W.seqlen_sweep()[4]) == "fused"     # 32 chains of 64 tiles
-    assert plan(W.seqlen_sweep()[5]) == "steps"     # 16 chains of 128 tiles
-    assert plan(W.LONG_CONTEXT) == "steps"          # 8 chains of 512 tiles
+def _plan(ssd, w):
+    return ssd.ssd_fwd_plan(ssd.ShapeT(w.batch, w.seqlen, w.nheads, w.headdim, w.ngroups,
+                                       w.dstate, w.chunk_size, ssd.SSD_BF16, 0))[0]
 
 
-def test_phase_sequential_fused_kernel(ssd, path_env, monkeypatch):
-    # The phase-sequential predecessor of the fused kernel (SSD_FUSED=v0), kept as
-    # an independent second single-pass implementation, against the oracle.
-    path_env("fused")
-    monkeypatch.setenv("SSD_FUSED", "v0")
-    inp = make_inputs(batch=2, seqlen=700, nheads=8, headdim=64, ngroups=2, dstate=128,
-                      dtype="bf16", initial_states=True, seed=41)
-    check_full(ssd, inp, 256, "bf16")
+def test_path_choice(ssd, path_env):
+    # every bf16 workload runs on the tensor-core single-pass kernel: one chain over
+    # the sequence when there are enough (batch row, head) chains to keep the GPU
+    # busy, segments otherwise
+    path_env(None)
+    assert _plan(ssd, W.MAMBA2_27B_LAYER) == "fused"
+    for w in W.seqlen_sweep() + W.dstate_sweep() + [W.LONG_CONTEXT]:
+        assert _plan(ssd, w) in ("fused", "segmented"), w.name
+    assert _plan(ssd, W.seqlen_sweep()[5]) == "segmented"
+    assert _plan(ssd, W.LONG_CONTEXT) == "segmented"
 
 
 def test_paths_agree(ssd, path_env):
     inp = make_inputs(batch=2, seqlen=900, nheads=4, headdim=64, ngroups=1, dstate=128,
                       dtype="bf16", initial_states=True, seed=33)
     outs = {}
-    for p in ("fused", "steps", "simt"):
+    for p in ("fused", "segmented", "steps", "simt"):
         path_env(p)
         outs[p] = run(ssd, inp, 256)
     y_ref, f_ref, _ = oracle.recurrence(**inp)
@@ -325,27 +348,44 @@ def test_paths_agree(ssd, path_env):
         assert oracle.rel_err(f.cpu(), f_ref) <= 5e-3, p
 
 
-# ---------------------------------------------------------------- fused kernel, whole tensors
-# The fused kernel against the four-step tensor-core path (itself checked against the
-# oracle above) on EVERY element of full-size workloads, and bitwise repeatability
-# across runs: a race between the kernel's warp roles shows up in either check.
-def _paths_full(ssd, path_env, w, seed=0, reps=3):
-    inp = W.workload_inputs(w, seed=seed)
-    path_env("steps")
-    y_ref, f_ref = run(ssd, inp, w.chunk_size)
-    path_env("fused")
+# ---------------------------------------------------------------- full size
+# Every element of y and of the final states against the oracle, on each workload
+# at its full size, in the path ssd_fwd picks for it (the one the benchmark times),
+# and bitwise repeatability across runs (a race between warp roles shows up there).
+def full_check(ssd, path_env, w, reps=2, path=None):
+    path_env(path)
+    inp = W.workload_inputs(w)
+    ref = oracle.recurrence(**inp)
     outs = [run(ssd, inp, w.chunk_size) for _ in range(reps)]
-    ref_max = y_ref.float().abs().max().item()
     for y, f in outs:
-        ey = (y.float() - y_ref.float()).abs().max().item() / ref_max
-        ef = ((f - f_ref).abs().max() / f_ref.abs().max()).item()
-        assert ey <= 5e-3, f"{w.name}: fused vs steps y rel err {ey:.3e}"
-        assert ef <= 5e-3, f"{w.name}: fused vs steps final rel err {ef:.3e}"
+        yc, fc = y.float().cpu(), f.cpu()
+        assert torch.isfinite(yc).all() and torch.isfinite(fc).all()
+        ey, ef = oracle.rel_err(yc, ref[0]), oracle.rel_err(fc, ref[1])
+        assert ey <= TOL[w.dtype], f"{w.name}: y rel err {ey:.3e}"
+        assert ef <= TOL[w.dtype], f"{w.name}: final rel err {ef:.3e}"
     for y, f in outs[1:]:
         assert torch.equal(y, outs[0][0]) and torch.equal(f, outs[0][1]), f"{w.name}: not repeatable"
 
 
-@pytest.mark.parametrize("w", [W.MAMBA2_27B_LAYER, W.seqlen_sweep()[4], W.LONG_CONTEXT],
-                         ids=lambda w: w.name)
-def test_fused_matches_steps_on_every_element(ssd, path_env, w):
-    _paths_full(ssd, path_env, w)
+def test_full_mamba2_layer(ssd, path_env):
+    full_check(ssd, path_env, W.MAMBA2_27B_LAYER, reps=3)
+
+
+@pytest.mark.parametrize("w", W.seqlen_sweep(), ids=lambda w: w.name)
+def test_full_seqlen_sweep(ssd, path_env, w):
+    full_check(ssd, path_env, w)
+
+
+@pytest.mark.parametrize("w", W.dstate_sweep(), ids=lambda w: w.name)
+def test_full_dstate_sweep(ssd, path_env, w):
+    full_check(ssd, path_env, w)
+
+
+def test_full_long_context(ssd, path_env):
+    full_check(ssd, path_env, W.LONG_CONTEXT)
+
+
+@pytest.mark.parametrize("path", ["fused", "segmented"])
+def test_full_mamba2_layer_other_path(ssd, path_env, path):
+    # the 2.7B layer in the path ssd_fwd does not pick for it, every element too
+    full_check(ssd, path_env, W.MAMBA2_27B_LAYER, reps=1, path=path)
