@@ -99,18 +99,24 @@ bool fused_ok(const ssd::Dims& d) {
            d.T <= 0x7fffffffLL && ssd::tma_available();
 }
 
-// The single-pass kernel hands each head's state from tile to tile through a
-// chain across CTAs. With few independent chains (batch rows x heads) over many
-// tiles that hand-off, not the work, sets the time; then the sequence is cut
-// into segments whose entering states are computed first (segment states, a
-// scan over them), and the segments run as separate, shorter chains.
-constexpr int64_t kSegmentBelowRowHeads = 300;   // b * H under which long sequences are cut
+// The single-pass kernel carries each (batch row, head pair) chain's state
+// through a segment of tiles inside one CTA, and from segment to segment through
+// a buffer and a flag. A chain's segments therefore run one after another; with
+// few chains (batch rows x head pairs) and many tiles that sets the time, and the
+// states entering all segments are computed first instead (segment states, a
+// scan over them), so that every segment can run at once.
+constexpr int64_t kChainedMinChains = 112;       // fewer chains than this: compute entering states first
 constexpr int64_t kSegmentMinTiles = 8;
-constexpr int64_t kTargetChains = 296;           // chains wanted when cutting (2 per SM)
+constexpr int64_t kTargetUnits = 4 * 148;        // units wanted: about four waves of CTAs
+
+int64_t fused_chains(const ssd::Dims& d) {
+    const int ns = ssd::fused_state_capacity(d.N);
+    return d.b * (d.H / ssd::fused_kheads(d.H, d.G, ns));
+}
 
 bool prefer_segments(const ssd::Dims& d) {
     const int64_t ntiles = (d.T + 127) / 128;
-    return ntiles >= kSegmentMinTiles && d.b * d.H < kSegmentBelowRowHeads;
+    return ntiles >= kSegmentMinTiles && fused_chains(d) < kChainedMinChains;
 }
 
 Path pick_path(const ssd::Dims& d) {
@@ -132,21 +138,22 @@ bool steps_use_tc(const ssd::Dims& d) {
 }
 
 // How the single-pass kernel covers the sequence: heads per unit, tiles per
-// segment, segments (1: one chain over the whole sequence).
+// segment (unit), segments; chained = entering states come from the previous
+// segment's unit, otherwise from the segment-state pass and scan.
 struct SegPlan {
     int kh, seg_tiles, nseg;
+    bool chained;
 };
 SegPlan seg_plan(const ssd::Dims& d, Path path) {
     SegPlan sp;
     const int ns = ssd::fused_state_capacity(d.N);
     sp.kh = ssd::fused_kheads(d.H, d.G, ns);
+    sp.chained = path != Path::Segmented;
     const int64_t ntiles = d.T > 0 ? (d.T + 127) / 128 : 1;
-    sp.seg_tiles = (int)std::min<int64_t>(ntiles, 0x7fffffff);
-    sp.nseg = 1;
-    if (path != Path::Segmented || ntiles < 2) return sp;
     const int64_t chains = std::max<int64_t>(1, d.b * (d.H / sp.kh));
-    int64_t nseg = std::max<int64_t>(2, (kTargetChains + chains - 1) / chains);
-    nseg = std::min(nseg, ntiles);
+    int64_t nseg = (kTargetUnits + chains - 1) / chains;
+    if (path == Path::Segmented) nseg = std::max<int64_t>(2, nseg);
+    nseg = std::max<int64_t>(1, std::min(nseg, ntiles));
     int64_t K = (ntiles + nseg - 1) / nseg;
     K = std::min<int64_t>(K, ssd::segment_max_tiles());
     sp.seg_tiles = (int)K;
@@ -155,8 +162,8 @@ SegPlan seg_plan(const ssd::Dims& d, Path path) {
 }
 
 // Workspace of ssd_fwd, regions 256-byte aligned:
-//   fused / segmented: [sync ints: ticket, error, flags[b*nseg*H] | chain state [b,H,P,N]
-//                       | segment states [b,nseg,H,P,N] | segment decays [b,nseg,H]]
+//   fused / segmented: [sync ints: ticket, error, flags[b*nseg*H] | segment states
+//                       [b,nseg,H,P,N] (nseg > 1) | segment decays [b,nseg,H] (segmented)]
 //   step paths:        [cs | chunk states S | entry states h_c]
 struct FwdWorkspace {
     Path path;
@@ -175,9 +182,9 @@ FwdWorkspace fwd_workspace(const ssd::Dims& d) {
         const size_t nseg = (size_t)w.sp.nseg;
         w.off_sync = 0;
         w.off_chain = align_up(sizeof(int) * ssd::fused_sync_ints(d, w.sp.nseg), 256);
-        w.off_seg = w.off_chain + align_up(z.st, 256);
+        w.off_seg = w.off_chain;
         w.off_decay = w.off_seg + (nseg > 1 ? align_up(z.st * nseg, 256) : 0);
-        w.total = w.off_decay + (nseg > 1 ? align_up((size_t)(d.b * d.H) * nseg * 4, 256) : 0);
+        w.total = w.off_decay + (nseg > 1 && !w.sp.chained ? align_up((size_t)(d.b * d.H) * nseg * 4, 256) : 0);
     } else {
         w.off_cs = 0;
         w.off_S = align_up(z.cs, 256);
@@ -257,7 +264,7 @@ ssd_status_t run_fwd(const ssd::Dims& d, const void* x, const float* dt, const f
                                                            stream))) != SSD_OK)
             return st;
         float* segbuf = w.sp.nseg > 1 ? (float*)(ws + w.off_seg) : nullptr;
-        if (w.sp.nseg > 1) {
+        if (w.sp.nseg > 1 && !w.sp.chained) {
             float* decay = (float*)(ws + w.off_decay);
             if ((st = cuda_status("segment states",
                                   ssd::launch_segment_states(d, maps, dt, A, segbuf, decay, sync + 1, w.sp.seg_tiles,
@@ -275,12 +282,13 @@ ssd_status_t run_fwd(const ssd::Dims& d, const void* x, const float* dt, const f
         a.A = A;
         a.D = D;
         a.init = init;
-        a.finalbuf = final_states ? final_states : (float*)(ws + w.off_chain);
+        a.finalbuf = final_states;
         a.segbuf = segbuf;
         a.sync_ints = sync;
         a.kheads = w.sp.kh;
         a.seg_tiles = w.sp.seg_tiles;
         a.nseg = w.sp.nseg;
+        a.chained = w.sp.chained ? 1 : 0;
         a.stall = test_stall();
         return cuda_status("fused forward", ssd::launch_fused(a, stream));
     }

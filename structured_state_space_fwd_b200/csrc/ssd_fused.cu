@@ -1,52 +1,49 @@
 // Warp-specialized, persistent single-pass SSD forward for sm_100a.
 //
-// "Transformers are SSMs" (Knowl 1, 2, 3, 7) with the chunk equal to one
-// 128-token tile: per tile the diagonal block in the quadratic masked form,
-// everything before the tile through the state entering it. With cs the
-// inclusive cumulative sum of dt*A inside the tile (log2 units), L = cs of the
-// tile's last token, w_i = 2^(L - cs_i) dt_i and q_j = 2^(cs_j - L), the
-// tile's outputs and leaving state are
+// "Transformers are SSMs" (Knowl 1, 2, 3, 7) in 128-token tiles: per tile the
+// diagonal block in the quadratic masked form, everything before the tile
+// through the state entering it. With cs the inclusive cumulative sum of dt*A
+// inside the tile (log2 units), L = cs of the tile's last token,
+// w_i = 2^(L - cs_i) dt_i and q_j = 2^(cs_j - L), a tile's outputs and the
+// state leaving it are
 //
 //   y_j  = q_j [ (tril(C B^T) (w o x))_j + C_j . (2^L h) + D x_j / q_j ]
 //   h'   = 2^L h + B^T (w o x)
 //
 // (the 1-semiseparable mask of Knowl 3 factored through the tile's last token).
 // The three terms in brackets accumulate in ONE tensor-memory accumulator Y'':
-// the skip term is stored into it first, then the masked product and the
-// state term are added by the tensor cores, so the epilogue is one scaling.
-// The tile-local products S = B^T (w o x) and tril(C B^T)(w o x) do not depend
-// on the state entering the tile; only the element-wise h' = 2^L h + S and
-// the product C (2^L h)^T wait for it. A unit whose heads decay by more than
-// 2^96 over the tile takes the unfactored form instead: per head
-// P = (C B^T) o exp(segsum) o dt (exponent per element), Y = P x + D x, and
-// R = C h^T into a separate accumulator, y = Y + 2^cs R.
+// the skip term is stored into it first, then the masked product and the state
+// term are added by the tensor cores, so the epilogue is one scaling. A tile
+// whose heads decay by more than 2^96 over it takes the unfactored form:
+// per head P = (C B^T) o exp(segsum) o dt (exponent per element), Y = P x + D x,
+// R = C h^T in a separate accumulator, y = Y + 2^cs R.
 //
-// Roles (16 warps):
-//   warp 0      TMA producer; takes units from a global ticket and hands their
-//               ids to every role through a small ring
+// Work unit: a SEGMENT of up to `seg_tiles` consecutive tiles of one batch row
+// and one pair of heads of a group (Knowl 7: the pair shares B and C). The CTA
+// that takes a unit walks its tiles in order and carries the pair's state in
+// registers from tile to tile (Knowl 2's state passing, inside the unit); only
+// the state entering the unit and the state leaving it touch global memory.
+// Every product of a tile is one MMA group of N = 128 (the two heads' 64
+// columns side by side). The state entering segment s > 0 is written by the
+// unit of segment s - 1 (units are handed out by an atomic ticket in
+// segment-major order, so that unit was taken earlier by a running CTA, and a
+// flag says when its state is out), or, for sequences with few (batch row,
+// pair) chains, computed beforehand by the segment-state pass and the scan over
+// segments (ssd_segment.cu), so that all segments run at once.
+//
+// Roles (20 warps):
+//   warp 0      TMA producer; takes units from the ticket and hands their ids to
+//               every role through a small ring
 //   warp 1      TMEM owner and MMA issuer (one thread)
-//   warp 2      per item: dt loads, cumulative sum, the chain flag of the
-//               state entering the tile (acquire)
-//   warp 3      chain publisher: releases the flag of each head's leaving state
-//   warps 4-7   mask group (thread = token row): tril(C B^T) into TMEM once per
-//               unit, per item the skip-term preload and w o x in place
-//   warps 8-11  chain group (thread = state row): per item the leaving state
-//               onto the chain and the bf16 state operand of C h^T
-//   warps 12-15 epilogue group (thread = token row): per item y = q Y'' staged
-//               in shared memory, one TMA store per warp
-// The chain and epilogue groups run their own loops: a head's state update does
-// not wait for the previous item's output, only for the operand buffer it reuses
-// (two buffers, each also the staging of one item's y).
-//
-// Work: a unit is (tile t, batch row b, block of k heads of one group), units
-// in tile-major order, handed out by an atomic ticket so that a unit's
-// predecessor on its chain (same b and heads, tile t-1) was always taken
-// earlier by a CTA that is running. An item is (unit, head). The state of
-// (b, h) after tile t goes to tile t+1 through one L2-resident buffer and a
-// release/acquire flag. Optionally the sequence is cut into segments of
-// `seg_tiles` tiles whose entering states were computed beforehand (segment
-// states and a scan over them, ssd_segment.cu); then each segment is a chain
-// of its own and many short chains run side by side.
+//   warp 2      per tile and head: dt loads, cumulative sum; per unit the flag of
+//               the state entering it (acquire)
+//   warp 3      per unit: makes the leaving state visible and releases its flag
+//   warps 4-7   mask group (thread = token row): per tile tril(C B^T) into TMEM,
+//               the skip-term preload and w o x in place of the x tiles
+//   warps 8-15  chain group (thread = state row, half of the head dim): carries
+//               the state, per tile the bf16 operand of C (2^L h)^T
+//   warps 16-19 epilogue group (thread = token row): per tile and head
+//               y = q Y'', staged in shared memory, one TMA store per warp
 //
 // Every wait is bounded; a wait that gives up sets the error word and makes
 // every role leave its loop, after which the CTA drains its MMAs and exits.
@@ -67,58 +64,56 @@ using namespace sm100;
 constexpr int kTile = 128;
 constexpr int kP = 64;
 constexpr int kThreads = 640;
-constexpr int kCsSlots = 2;
-constexpr int kYSlots = 3;
+constexpr int kCsSlots = 4;       // per tile and head
+constexpr int kYSlots = 2;        // Y'' accumulators, one tile of the pair each
 constexpr int kURing = 4;
-constexpr int kPubStages = 4;
 
 constexpr uint32_t kAtom = kTile * 128;    // 16 KB: 128 rows of 128 bytes (64 bf16)
-// per item: cs[128], dt[128], then L (cs of the last token), D_h, unit mode
+// per tile and head: cs[128], dt[128], then L (cs of the last token), D_h, tile mode
 constexpr uint32_t kCsSlotBytes = 2 * kTile * 4 + 64;
 constexpr int kCsL = 2 * kTile, kCsD = 2 * kTile + 1, kCsMode = 2 * kTile + 2;
+// per Y'' accumulator: each head's row factor (q_j, or 2^cs_j), per head 2^L, the mode
+constexpr uint32_t kYInfoBytes = 2 * kTile * 4 + 16;
+constexpr int kYiEL = 2 * kTile, kYiMode = 2 * kTile + 2;
 
-// TMEM columns: G = C B^T (fp32), P (bf16 pairs, the A operand of the masked
-// product), S slots, three Y'' accumulators
+// TMEM columns: G = C B^T (fp32), overwritten in place by P' = tril(G) (bf16
+// pairs, columns 0..63) for factored tiles; the S slot (the pair's two 64-column
+// states, or one 256-row state as two halves; for an unfactored tile first its
+// per-head P, later its C h^T); two Y'' accumulators of a pair each.
 constexpr uint32_t kColG = 0;
-constexpr uint32_t kColP = 128;
-constexpr uint32_t kColS = 192;
-constexpr uint32_t kColY = 320;
+constexpr uint32_t kColP = 0;
+constexpr uint32_t kColS = 128;
+constexpr uint32_t kColY = 256;
 
 constexpr float kLog2e = 1.4426950408889634f;
-// Widest decay over one tile (log2 units) for which a unit takes the factored
+// Widest decay over one tile (log2 units) for which a tile takes the factored
 // form: 2^(L - cs) dt (bf16 operand) and 2^(L - cs) (skip-term divisor) then stay
 // inside the normal fp32 / bf16 exponent range with a wide margin.
 constexpr float kSharedMaskRangeLog2 = 96.f;
 
-// Shared-memory layout for state capacity NS (128 or 256 state elements).
-// per Y'' accumulator: the epilogue's row factor (q_j, or 2^cs_j), then 2^L, unit mode
-constexpr uint32_t kYInfoBytes = kTile * 4 + 16;
-
-// B and C tiles live in a ring of tile buffers, taken in the order B_0, C_0, B_1,
-// C_1, ...: a unit's B is released once its S products are done, its C once its
-// state products are, so three buffers let the next unit's tiles load early.
+// Shared-memory layout for state capacity NS (128 or 256 state elements). B and C
+// tiles live in a ring of tile buffers taken in the order B_0, C_0, B_1, C_1, ...:
+// a tile's B is released once its S product is done, its C once its state
+// product is.
 template <int NS>
 struct Cfg {
     static constexpr int kAtoms = NS / 64;                  // 64-wide column atoms of B or C
-    static constexpr uint32_t kBCTile = kAtoms * kAtom;     // B (or C) tile of one unit
+    static constexpr uint32_t kBCTile = kAtoms * kAtom;     // B (or C) tile
     static constexpr int kBufs = NS == 128 ? 3 : 2;         // tile buffers
-    static constexpr int kXSlots = NS == 128 ? 4 : 3;
-    static constexpr int kSSlots = NS == 128 ? 2 : 1;
-    static constexpr int kMHalves = NS / 128;               // 128-row halves of the state
-    static constexpr int kHYSlots = NS == 128 ? 2 : 1;      // state operand buffers
-    static constexpr uint32_t kHYBytes = NS * 128;          // NS rows of 64 bf16
-    // y staging: its own 4 KB per epilogue warp, or (NS = 256) the operand buffer
-    static constexpr bool kOwnStaging = NS == 128;
+    static constexpr int kMH = NS / 128;                    // 128-row halves of the state
+    static constexpr int kNP = NS == 128 ? 2 : 1;           // heads per unit at most
+    static constexpr int kXSlots = 2;                       // x slots, one tile of the pair each
+    static constexpr uint32_t kXBytes = kNP * kAtom;
+    static constexpr uint32_t kHBytes = 2 * kAtom;          // state operand: 2 atoms
     static constexpr uint32_t kOffBC = 0;
     static constexpr uint32_t kOffX = kOffBC + kBufs * kBCTile;
-    static constexpr uint32_t kOffHY = kOffX + kXSlots * kAtom;
-    static constexpr uint32_t kOffStage = kOffHY + kHYSlots * kHYBytes;
-    static constexpr uint32_t kOffCs = kOffStage + (kOwnStaging ? kAtom : 0);
+    static constexpr uint32_t kOffH = kOffX + kXSlots * kXBytes;
+    static constexpr uint32_t kOffStage = kOffH + kHBytes;  // 4 KB per epilogue warp
+    static constexpr uint32_t kOffCs = kOffStage + kAtom;
     static constexpr uint32_t kOffYInfo = kOffCs + kCsSlots * kCsSlotBytes;
     static constexpr uint32_t kOffBar = kOffYInfo + kYSlots * kYInfoBytes;
     static constexpr uint32_t kSmem = kOffBar + 1024;
     static_assert(kSmem <= 232448, "shared memory budget");
-    static_assert(kColY + kYSlots * 64 <= 512, "tensor memory budget");
 };
 
 struct Params {
@@ -126,38 +121,41 @@ struct Params {
     const float* A;
     const float* D;
     const float* init;    // [b,H,P,N] or null (zeros)
-    float* finalbuf;      // chain buffer of the last segment: final states or workspace
+    float* finalbuf;      // [b,H,P,N] final states, or null (not written)
     float* segbuf;        // [b,nseg,H,P,N]: slot s >= 1 holds the state entering segment s
     int* ticket;
     int* error;
-    int* flags;           // [b*nseg*H] tiles of the segment whose leaving state is out
+    int* flags;           // [b*nseg*nhb] state entering the segment written (chained)
     int64_t T;
     int H, G, N, kheads, batch, nunits, ntiles, seg_tiles, nseg;
+    int chained;          // entering states come from the previous segment's unit
     int stall;            // test builds only: chain flags awaited at a value never reached
 };
 
 struct Bars {
     uint64_t u_full[kURing], u_empty[kURing];
     uint64_t tb_full[3], tb_empty[3];
-    uint64_t x_full[4], x_empty[4];
-    uint64_t wx_full[4];          // item's operands ready (w o x, or P and raw x); mode in xmode
-    uint64_t wx2_full;            // unfactored item: x scaled in place after Y = P x
-    uint64_t g_full, g_empty, p_full, p_empty, xr_done;
+    uint64_t x_full[2], x_empty[2];
+    uint64_t wx_full[2];          // tile's operands ready (w o x, or per-head P and raw x); mode in xmode
+    uint64_t wx2_full;            // unfactored tile: x scaled in place after Y = P x
+    uint64_t xr_done;             // unfactored tile: Y = P x has read the raw tiles
+    uint64_t g_full, g_empty_mma, g_empty_mask, p_full;
     uint64_t cs_full[kCsSlots], cs_empty[kCsSlots];
-    uint64_t s_full[2], s_empty[2];
+    uint64_t s_full, s_empty;
     uint64_t y_full[kYSlots], y_empty[kYSlots], yi_full[kYSlots];
-    uint64_t h_full[2], hy_free[2];
-    uint64_t pub_full[kPubStages], pub_empty[kPubStages];
+    uint64_t h_full, h_free;
+    uint64_t pub_full[2], pub_empty[2];   // per unit: leaving state stored / flag released
     uint64_t fin;
     int uid[kURing];
-    int xmode[4];
+    int xmode[2];
     uint32_t tmem;
     int abort;
 };
 static_assert(sizeof(Bars) <= 1024, "barrier block");
 
-// arrivals on u_empty: MMA thread, cumsum warp, publisher, mask, chain and epilogue groups
-constexpr uint32_t kUnitReaders = 1 + 32 + 1 + 128 + 256 + 128;
+// arrivals on u_empty: x loader, MMA thread, cumsum warp, publisher, mask, chain and
+// epilogue groups
+constexpr uint32_t kUnitReaders = 1 + 1 + 32 + 1 + 128 + 256 + 128;
 
 __device__ __forceinline__ int ld_acquire(const int* p) {
     int v;
@@ -167,6 +165,9 @@ __device__ __forceinline__ int ld_acquire(const int* p) {
 __device__ __forceinline__ void st_release(int* p, int v) {
     asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+// Orders every memory access this thread has made or observed (the chain group's
+// state stores, seen through an mbarrier) before its later accesses, GPU-wide.
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&h);
@@ -252,8 +253,8 @@ __device__ __forceinline__ bool wait_bar_all(uint64_t* bar, uint32_t parity, Bar
 }
 
 struct Unit {
-    int t, kk, s, b, hb;   // tile, tile within its segment, segment, batch row, head block
-    int64_t t0;            // first token of the tile
+    int s, b, hb;          // segment, batch row, head block (pair)
+    int t_begin, t_end;    // its tiles
 };
 __device__ __forceinline__ Unit decode(const Params& p, int u) {
     const int nhb = p.H / p.kheads;
@@ -261,28 +262,26 @@ __device__ __forceinline__ Unit decode(const Params& p, int u) {
     r.hb = u % nhb;
     int q = u / nhb;
     r.b = q % p.batch;
-    q /= p.batch;
-    r.s = q % p.nseg;
-    r.kk = q / p.nseg;
-    r.t = r.s * p.seg_tiles + r.kk;
-    r.t0 = (int64_t)r.t * kTile;
+    r.s = q / p.batch;
+    r.t_begin = r.s * p.seg_tiles;
+    r.t_end = min(p.ntiles, r.t_begin + p.seg_tiles);
     return r;
 }
-__device__ __forceinline__ int64_t chain_index(const Params& p, const Unit& U, int h) {
-    return ((int64_t)U.b * p.nseg + U.s) * p.H + h;
+__device__ __forceinline__ int64_t flag_index(const Params& p, int b, int s, int hb) {
+    return ((int64_t)b * p.nseg + s) * (p.H / p.kheads) + hb;
 }
-// buffer that carries (b, h)'s state from tile to tile inside segment s
-__device__ __forceinline__ float* chain_buf(const Params& p, const Unit& U, int h) {
-    const int64_t PN = (int64_t)kP * p.N;
-    if (U.s == p.nseg - 1) return p.finalbuf + ((int64_t)U.b * p.H + h) * PN;
-    return p.segbuf + chain_index(p, U, h) * PN;
-}
-// state entering the unit's tile for head h (null: zeros)
+// state entering the unit for head h (null: zeros)
 __device__ __forceinline__ const float* entry_src(const Params& p, const Unit& U, int h) {
     const int64_t PN = (int64_t)kP * p.N;
-    if (U.kk != 0) return chain_buf(p, U, h);
     if (U.s == 0) return p.init ? p.init + ((int64_t)U.b * p.H + h) * PN : nullptr;
-    return p.segbuf + chain_index(p, U, h) * PN;
+    return p.segbuf + (((int64_t)U.b * p.nseg + U.s) * p.H + h) * PN;
+}
+// where the state leaving the unit goes for head h (null: nowhere)
+__device__ __forceinline__ float* exit_dst(const Params& p, const Unit& U, int h) {
+    const int64_t PN = (int64_t)kP * p.N;
+    if (U.s == p.nseg - 1) return p.finalbuf ? p.finalbuf + ((int64_t)U.b * p.H + h) * PN : nullptr;
+    if (!p.chained) return nullptr;
+    return p.segbuf + (((int64_t)U.b * p.nseg + U.s + 1) * p.H + h) * PN;
 }
 
 // Byte offset of row `row`, 16-byte chunk `c` in a 128-byte-swizzled tile.
@@ -311,6 +310,18 @@ __device__ __forceinline__ void mma_state_dim_n(int ks, uint32_t d, uint64_t dA,
         default: mma_state_dim<16, kBRows>(d, dA, dB, idesc, acc0); break;
     }
 }
+// 8 steps of K = 16 over the tile's tokens: A from shared memory (B^T, N-contiguous)
+// or from tensor memory (P), B the x tiles of the pair (N-contiguous).
+__device__ __forceinline__ void mma_tokens_smem(uint32_t d, uint64_t dA, uint64_t dB, uint32_t idesc) {
+#pragma unroll
+    for (int kk = 0; kk < kTile / 16; ++kk)
+        mma_bf16(d, dA + (uint64_t)(kk * 128), dB + (uint64_t)(kk * 128), idesc, kk > 0 ? 1u : 0u);
+}
+__device__ __forceinline__ void mma_tokens_tmem(uint32_t d, uint32_t a, uint64_t dB, uint32_t idesc) {
+#pragma unroll
+    for (int kk = 0; kk < kTile / 16; ++kk)
+        mma_bf16_tmem_a(d, a + 8 * kk, dB + (uint64_t)(kk * 128), idesc, 1u);
+}
 
 template <int NS>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -334,38 +345,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bs->tb_empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&bs->s_full[i], 1);
-            mbar_init(&bs->s_empty[i], 256);
-        }
-        for (int i = 0; i < 4; ++i) {
             mbar_init(&bs->x_full[i], 1);
             mbar_init(&bs->x_empty[i], 1);
             mbar_init(&bs->wx_full[i], 128);
+            mbar_init(&bs->pub_full[i], 256);
+            mbar_init(&bs->pub_empty[i], 1);
         }
         mbar_init(&bs->wx2_full, 128);
-        mbar_init(&bs->g_full, 1);
-        mbar_init(&bs->g_empty, 128);
-        mbar_init(&bs->p_full, 128);
-        mbar_init(&bs->p_empty, 1);
         mbar_init(&bs->xr_done, 1);
+        mbar_init(&bs->g_full, 1);
+        mbar_init(&bs->g_empty_mma, 1);
+        mbar_init(&bs->g_empty_mask, 128);
+        mbar_init(&bs->p_full, 128);
         for (int i = 0; i < kCsSlots; ++i) {
             mbar_init(&bs->cs_full[i], 32);
             mbar_init(&bs->cs_empty[i], 128);
         }
+        mbar_init(&bs->s_full, 1);
+        mbar_init(&bs->s_empty, 256);
         for (int i = 0; i < kYSlots; ++i) {
             mbar_init(&bs->y_full[i], 1);
             mbar_init(&bs->y_empty[i], 128);
             mbar_init(&bs->yi_full[i], 128);
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&bs->h_full[i], 256);
-            // freed by the state product's commit, or by the epilogue warps' y stores
-            mbar_init(&bs->hy_free[i], K::kOwnStaging ? 1 : 4);
-        }
-        for (int i = 0; i < kPubStages; ++i) {
-            mbar_init(&bs->pub_full[i], 256);
-            mbar_init(&bs->pub_empty[i], 1);
-        }
+        mbar_init(&bs->h_full, 256);
+        mbar_init(&bs->h_free, 1);
         mbar_init(&bs->fin, 1);
         bs->abort = 0;
         fence_barrier_init();
@@ -382,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // (error already set) but still release TMEM below
     const bool misaligned = (smem_u32(smem) & 1023u) != 0;
     const uint32_t tmem = bs->tmem;
-    const int kh = prm.kheads;
+    const int np = prm.kheads;             // heads per unit (1 or 2)
     const int64_t T = prm.T;
     const int H = prm.H;
     // K steps of the products over the state dim: a power of two covering N (the B
@@ -395,13 +399,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         // nothing
     } else if (warp == 0) {
         // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            int m = 0, n = 0, mb = 0;    // units taken, x tiles and tile buffers loaded
+        // Lane 0 takes units and loads B and C; lane 1 loads the x tiles, so that they
+        // do not queue behind tile buffers still in use.
+        if (lane == 1) {
+            int n = 0;
+            for (int m = 0;; ++m) {
+                const int ur = m % kURing;
+                if (!wait_bar_idle(&bs->u_full[ur], (m / kURing) & 1, bs, err)) goto xdrain;
+                const int u = bs->uid[ur];
+                mbar_arrive(&bs->u_empty[ur]);
+                if (u < 0) break;
+                const Unit U = decode(prm, u);
+                for (int t = U.t_begin; t < U.t_end; ++t, ++n) {
+                    const int xs = n % K::kXSlots;
+                    if (!wait_bar_idle(&bs->x_empty[xs], ((n / K::kXSlots) & 1) ^ 1, bs, err)) goto xdrain;
+                    mbar_arrive_expect_tx(&bs->x_full[xs], np * kAtom);
+                    for (int e = 0; e < np; ++e)
+                        tma_load_4d(smem + K::kOffX + xs * K::kXBytes + e * kAtom, &tm_x, &bs->x_full[xs], 0,
+                                    U.hb * np + e, t * kTile, U.b);
+                }
+            }
+        xdrain:
+            for (int i = 0; i < K::kXSlots && i < n; ++i)
+                mbar_wait(&bs->x_full[(n - 1 - i) % K::kXSlots], ((n - 1 - i) / K::kXSlots) & 1, 1u << 22);
+        } else if (lane == 0) {
+            int m = 0, mb = 0;    // units taken, tile buffers loaded
             for (;; ++m) {
                 int u;
                 do {
                     u = atomicAdd(prm.ticket, 1);
-                } while (u < prm.nunits && decode(prm, u).t >= prm.ntiles);
+                } while (u < prm.nunits && decode(prm, u).t_begin >= prm.ntiles);
                 if (u >= prm.nunits) u = -1;
                 const int ur = m % kURing;
                 if (!wait_bar_idle(&bs->u_empty[ur], ((m / kURing) & 1) ^ 1, bs, err)) goto pdrain;
@@ -409,60 +436,51 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(&bs->u_full[ur]);
                 if (u < 0) break;
                 const Unit U = decode(prm, u);
-                const int g = U.hb * kh / (H / prm.G);
-                for (int bc = 0; bc < 2; ++bc, ++mb) {    // B, then C
-                    const int tb = mb % K::kBufs;
-                    if (!wait_bar_idle(&bs->tb_empty[tb], ((mb / K::kBufs) & 1) ^ 1, bs, err)) goto pdrain;
-                    mbar_arrive_expect_tx(&bs->tb_full[tb], natoms * kAtom);
-                    for (int a = 0; a < natoms; ++a)
-                        tma_load_4d(smem + K::kOffBC + tb * K::kBCTile + a * kAtom, bc ? &tm_C : &tm_B,
-                                    &bs->tb_full[tb], a * 64, g, (int)U.t0, U.b);
-                }
-                for (int k = 0; k < kh; ++k, ++n) {
-                    const int xs = n % K::kXSlots;
-                    if (!wait_bar_idle(&bs->x_empty[xs], ((n / K::kXSlots) & 1) ^ 1, bs, err)) goto pdrain;
-                    mbar_arrive_expect_tx(&bs->x_full[xs], kAtom);
-                    tma_load_4d(smem + K::kOffX + xs * kAtom, &tm_x, &bs->x_full[xs], 0, U.hb * kh + k,
-                                (int)U.t0, U.b);
+                const int g = U.hb * np / (H / prm.G);
+                for (int t = U.t_begin; t < U.t_end; ++t) {
+                    for (int bc = 0; bc < 2; ++bc, ++mb) {    // B, then C
+                        const int tb = mb % K::kBufs;
+                        if (!wait_bar_idle(&bs->tb_empty[tb], ((mb / K::kBufs) & 1) ^ 1, bs, err)) goto pdrain;
+                        mbar_arrive_expect_tx(&bs->tb_full[tb], natoms * kAtom);
+                        for (int a = 0; a < natoms; ++a)
+                            tma_load_4d(smem + K::kOffBC + tb * K::kBCTile + a * kAtom, bc ? &tm_C : &tm_B,
+                                        &bs->tb_full[tb], a * 64, g, t * kTile, U.b);
+                    }
                 }
             }
         pdrain:
             // No TMA load may still be writing shared memory when the CTA exits: wait for
-            // the last load issued into each slot (already complete unless a role aborted).
-            for (int i = 0; i < K::kXSlots && i < n; ++i)
-                mbar_wait(&bs->x_full[(n - 1 - i) % K::kXSlots], ((n - 1 - i) / K::kXSlots) & 1, 1u << 22);
+            // the last load issued into each buffer (already complete unless a role aborted).
             for (int i = 0; i < K::kBufs && i < mb; ++i)
                 mbar_wait(&bs->tb_full[(mb - 1 - i) % K::kBufs], ((mb - 1 - i) / K::kBufs) & 1, 1u << 22);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        // Per item i: S_i and the masked product (neither waits for the chain), then
-        // the previous item's state product C h^T, whose operand the chain group
-        // writes once that head's entering state is known.
+        // Per tile i: G = C B^T, S_i and the masked product (neither waits for the
+        // state), then the tile's state product C h^T once the chain group has
+        // written its operand (a register update of the carried state).
         if (lane == 0) {
             constexpr uint32_t idG = idesc_bf16(128, 128, 0, 0);   // C (K-major) x B (K-major)
-            constexpr uint32_t idS = idesc_bf16(128, kP, 1, 1);    // B^T (N-contiguous) x (w o x)
-            constexpr uint32_t idY = idesc_bf16(128, kP, 0, 1);    // P or C (K-major) x (w o x) or h
+            const uint32_t idS = np == 2 ? idesc_bf16(128, 128, 1, 1) : idesc_bf16(128, 64, 1, 1);
+            const uint32_t idY = np == 2 ? idesc_bf16(128, 128, 0, 1) : idesc_bf16(128, 64, 0, 1);
+            constexpr uint32_t idY1 = idesc_bf16(128, 64, 0, 1);   // one head (unfactored masked product)
+            const uint64_t dH = sw128_desc(smem_u32(smem + K::kOffH), kAtom, 1024);
             struct Pend {
-                int item, ys, ss, cb;   // cb: tile buffer of the unit's C
-                bool shared, last;
+                int item, ys, cb;   // cb: tile buffer of the tile's C
+                bool shared;
             };
-            Pend pv{};
-            bool have = false;
-            int psh = 0, nsh = 0;
-            // C (2^L h)^T onto Y'' (factored units) or C h^T into the item's S slot
+            int psh = 0, nsh = 0, gm = 0, gk = 0;
+            bool prev_shared = true;
+            // C (2^L h)^T onto Y'' (factored) or C h^T into the S slot (unfactored)
             auto issue_r = [&](const Pend& q) -> bool {
-                const int hs = q.item % K::kHYSlots;
-                if (!wait_bar(&bs->h_full[hs], (q.item / K::kHYSlots) & 1, bs, err)) return false;
+                if (!wait_bar(&bs->h_full, q.item & 1, bs, err)) return false;
                 tc_fence_after();
-                const uint64_t dH = sw128_desc(smem_u32(smem + K::kOffHY + hs * K::kHYBytes), kAtom, 1024);
-                const uint32_t cB = smem_u32(smem + K::kOffBC + q.cb * K::kBCTile);
-                const uint64_t dC = sw128_desc(cB, 16, 1024);
-                const uint32_t d = q.shared ? tmem + kColY + 64 * q.ys : tmem + kColS + 64 * q.ss;
+                const uint64_t dC = sw128_desc(smem_u32(smem + K::kOffBC + q.cb * K::kBCTile), 16, 1024);
+                const uint32_t d = q.shared ? tmem + kColY + 128 * q.ys : tmem + kColS;
                 mma_state_dim_n<true>(ksN, d, dC, dH, idY, q.shared ? 1u : 0u);
                 mma_commit(&bs->y_full[q.ys]);
-                if (K::kOwnStaging) mma_commit(&bs->hy_free[hs]);
-                if (q.last) mma_commit(&bs->tb_empty[q.cb]);
+                mma_commit(&bs->h_free);
+                mma_commit(&bs->tb_empty[q.cb]);
                 return true;
             };
             int m = 0, i = 0;
@@ -472,85 +490,67 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int u = bs->uid[ur];
                 mbar_arrive(&bs->u_empty[ur]);
                 if (u < 0) break;
-                const int tbB = (2 * m) % K::kBufs, tbC = (2 * m + 1) % K::kBufs;
-                const uint32_t bcB = smem_u32(smem + K::kOffBC + tbB * K::kBCTile);
-                const uint32_t bcC = smem_u32(smem + K::kOffBC + tbC * K::kBCTile);
-                // G = C B^T of the tile, shared by the unit's heads
-                if (!wait_bar(&bs->tb_full[tbB], ((2 * m) / K::kBufs) & 1, bs, err)) goto drain;
-                if (!wait_bar(&bs->tb_full[tbC], ((2 * m + 1) / K::kBufs) & 1, bs, err)) goto drain;
-                if (!wait_bar(&bs->g_empty, (m & 1) ^ 1, bs, err)) goto drain;
-                tc_fence_after();
-                {
-                    mma_state_dim_n<false>(ksN, tmem + kColG, sw128_desc(bcC, 16, 1024), sw128_desc(bcB, 16, 1024),
-                                           idG, 0u);
-                }
-                mma_commit(&bs->g_full);
-                const uint64_t dSA = sw128_desc(bcB, kAtom, 1024);
-                for (int k = 0; k < kh; ++k, ++i) {
-                    const int xs = i % K::kXSlots, ys = i % kYSlots, ss = i % K::kSSlots;
+                const Unit U = decode(prm, u);
+                for (int t = U.t_begin; t < U.t_end; ++t, ++i) {
+                    const int xs = i % K::kXSlots, ys = i % kYSlots;
+                    const int tbB = (2 * i) % K::kBufs, tbC = (2 * i + 1) % K::kBufs;
+                    const uint32_t bcB = smem_u32(smem + K::kOffBC + tbB * K::kBCTile);
+                    const uint32_t bcC = smem_u32(smem + K::kOffBC + tbC * K::kBCTile);
+                    if (!wait_bar(&bs->tb_full[tbB], ((2 * i) / K::kBufs) & 1, bs, err)) goto drain;
+                    if (!wait_bar(&bs->tb_full[tbC], ((2 * i + 1) / K::kBufs) & 1, bs, err)) goto drain;
+                    // G = C B^T into the G/P' columns, free once the previous tile's masked
+                    // product (factored) or its per-head masks (unfactored) are done
+                    if (i > 0) {
+                        if (prev_shared) {
+                            if (!wait_bar(&bs->g_empty_mma, gm & 1, bs, err)) goto drain;
+                            ++gm;
+                        } else {
+                            if (!wait_bar(&bs->g_empty_mask, gk & 1, bs, err)) goto drain;
+                            ++gk;
+                        }
+                    }
+                    tc_fence_after();
+                    mma_state_dim_n<false>(ksN, tmem + kColG, sw128_desc(bcC, 16, 1024), sw128_desc(bcB, 16, 1024), idG, 0u);
+                    mma_commit(&bs->g_full);
+                    const uint64_t dSA = sw128_desc(bcB, kAtom, 1024);
                     if (!wait_bar(&bs->wx_full[xs], (i / K::kXSlots) & 1, bs, err)) goto drain;
                     const bool shared = *(volatile int*)&bs->xmode[xs] != 0;
-                    // a pending unfactored item's C h^T goes into its S slot before this
-                    // item's S may reuse that slot
-                    if (have && !pv.shared) {
-                        if (!issue_r(pv)) goto drain;
-                        have = false;
-                    }
-                    const uint64_t dX = sw128_desc(smem_u32(smem + K::kOffX + xs * kAtom), kAtom, 1024);
-                    auto issue_s = [&]() -> bool {
-                        if (!wait_bar(&bs->s_empty[ss], ((i / K::kSSlots) & 1) ^ 1, bs, err)) return false;
-                        tc_fence_after();
-                        for (int mh = 0; mh < K::kMHalves; ++mh)
-                            for (int kk = 0; kk < kTile / 16; ++kk)
-                                mma_bf16(tmem + kColS + 64 * ss + 64 * mh,
-                                         dSA + (uint64_t)((2 * mh * kAtom) >> 4) + (uint64_t)(kk * 128),
-                                         dX + (uint64_t)(kk * 128), idS, kk > 0);
-                        mma_commit(&bs->s_full[ss]);
-                        return true;
-                    };
+                    const uint64_t dX = sw128_desc(smem_u32(smem + K::kOffX + xs * K::kXBytes), kAtom, 1024);
                     if (shared) {
+                        if (!wait_bar(&bs->s_empty, (i & 1) ^ 1, bs, err)) goto drain;
                         tc_fence_after();
-                        if (!issue_s()) goto drain;
-                        if (k == 0) {
-                            if (!wait_bar(&bs->p_full, psh & 1, bs, err)) goto drain;
-                            ++psh;
-                            tc_fence_after();
-                        }
-                        for (int kk = 0; kk < kTile / 16; ++kk)
-                            mma_bf16_tmem_a(tmem + kColY + 64 * ys, tmem + kColP + 8 * kk,
-                                            dX + (uint64_t)(kk * 128), idY, 1u);
+#pragma unroll
+                        for (int mh = 0; mh < K::kMH; ++mh)
+                            mma_tokens_smem(tmem + kColS + 64 * mh, dSA + (uint64_t)((2 * mh * kAtom) >> 4), dX, idS);
+                        mma_commit(&bs->s_full);
+                        if (!wait_bar(&bs->p_full, psh & 1, bs, err)) goto drain;
+                        ++psh;
+                        tc_fence_after();
+                        mma_tokens_tmem(tmem + kColY + 128 * ys, tmem + kColP, dX, idY);
                         mma_commit(&bs->x_empty[xs]);
-                        if (k == kh - 1) mma_commit(&bs->p_empty);
+                        mma_commit(&bs->g_empty_mma);
                     } else {
-                        // Y = P x with the raw tile, then S once the tile is scaled in place
+                        // per head Y = P x with the raw tile (P in the S slot), then S once
+                        // the tile is scaled in place
                         tc_fence_after();
-                        for (int kk = 0; kk < kTile / 16; ++kk)
-                            mma_bf16_tmem_a(tmem + kColY + 64 * ys, tmem + kColP + 8 * kk,
-                                            dX + (uint64_t)(kk * 128), idY, 1u);
+                        for (int e = 0; e < np; ++e)
+                            mma_tokens_tmem(tmem + kColY + 128 * ys + 64 * e, tmem + kColS + 64 * e,
+                                            dX + (uint64_t)((e * kAtom) >> 4), idY1);
                         mma_commit(&bs->xr_done);
-                        mma_commit(&bs->p_empty);
                         if (!wait_bar(&bs->wx2_full, nsh & 1, bs, err)) goto drain;
                         ++nsh;
-                        if (!issue_s()) goto drain;
+                        tc_fence_after();
+#pragma unroll
+                        for (int mh = 0; mh < K::kMH; ++mh)
+                            mma_tokens_smem(tmem + kColS + 64 * mh, dSA + (uint64_t)((2 * mh * kAtom) >> 4), dX, idS);
+                        mma_commit(&bs->s_full);
                         mma_commit(&bs->x_empty[xs]);
                     }
-                    if (have) {
-                        if (!issue_r(pv)) goto drain;
-                        have = false;
-                    }
-                    // the unit's B has served its last S product
-                    if (k == kh - 1) mma_commit(&bs->tb_empty[tbB]);
-                    pv = Pend{i, ys, ss, tbC, shared, k == kh - 1};
-                    have = true;
-                    // with two tile buffers the next unit's C reuses this unit's: its last
-                    // state product goes out first
-                    if (K::kBufs == 2 && k == kh - 1) {
-                        if (!issue_r(pv)) goto drain;
-                        have = false;
-                    }
+                    prev_shared = shared;
+                    mma_commit(&bs->tb_empty[tbB]);    // this tile's B has served its S
+                    if (!issue_r(Pend{i, ys, tbC, shared})) goto drain;
                 }
             }
-            if (have && !issue_r(pv)) goto drain;
         drain:
             // every MMA issued so far is complete before TMEM is released
             mma_commit(&bs->fin);
@@ -558,23 +558,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 2) {
         // ------------------------------------------------------------ cumsum warp
-        // Per unit, the dt of all its heads is loaded at once, and lane k polls head
-        // k's chain flag, so no item waits a full memory round trip of its own.
-        constexpr int kMaxKh = NS == 256 ? 8 : 4;
-        float dtv[kMaxKh][4];
-        auto load_dt = [&](const Unit& U, float (&v)[kMaxKh][4]) {
-            const int len = (int)min((int64_t)kTile, T - U.t0);
-#pragma unroll
-            for (int k = 0; k < kMaxKh; ++k)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int t = lane * 4 + e;
-                    v[k][e] = (k < kh && t < len)
-                                  ? __ldg(prm.dt + ((int64_t)U.b * T + U.t0 + t) * H + U.hb * kh + k)
-                                  : 0.f;
-                }
-        };
-        int m = 0, i = 0;
+        // Per unit: the flag of the state entering it (written by the previous
+        // segment's unit). Per tile: the dt of the pair's heads, the tile's form
+        // (factored unless a head decays by more than 2^96 over it), and per head
+        // the cumulative sum of dt A (log2 units) into a slot for the mask group.
+        int m = 0, hi = 0;
         for (;; ++m) {
             const int ur = m % kURing;
             if (!__all_sync(0xffffffffu, wait_bar_idle(&bs->u_full[ur], (m / kURing) & 1, bs, err)))
@@ -583,189 +571,165 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&bs->u_empty[ur]);
             if (u < 0) break;
             const Unit U = decode(prm, u);
-            load_dt(U, dtv);
-            // Does every head of the unit decay by at most kSharedMaskRangeLog2 over this
-            // tile? Then the unit takes the factored form.
-            float worst = 0.f;
-#pragma unroll
-            for (int k = 0; k < kMaxKh; ++k) {
-                if (k >= kh) break;
-                float sdt = dtv[k][0] + dtv[k][1] + dtv[k][2] + dtv[k][3];
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) sdt += __shfl_xor_sync(0xffffffffu, sdt, off);
-                worst = fmaxf(worst, sdt * fabsf(__ldg(prm.A + U.hb * kh + k)) * kLog2e);
-            }
-            const float mode = worst <= kSharedMaskRangeLog2 ? 1.f : 0.f;
-            // lane k < kh watches the chain flag of head k (the state entering this tile
-            // comes from the previous tile of the same segment)
-            const bool watch = U.kk > 0 && lane < kh;
-            const int* myflag = prm.flags + chain_index(prm, U, U.hb * kh + (lane < kh ? lane : 0));
-            const int want = U.kk + (prm.stall ? (1 << 30) : 0);
-            bool seen = !watch;
-            const uint64_t tw = global_ns();
-#pragma unroll
-            for (int k = 0; k < kMaxKh; ++k) {
-                if (k >= kh) break;
-                const int h = U.hb * kh + k;
-                const float a2 = __ldg(prm.A + h) * kLog2e;
-                const float d_h = prm.D ? __ldg(prm.D + h) : 0.f;
-                const int c = i % kCsSlots;
-                if (!__all_sync(0xffffffffu,
-                                wait_bar_idle(&bs->cs_empty[c], ((i / kCsSlots) & 1) ^ 1, bs, err)))
-                    goto done;
-                // acquire head k's flag before the consumers may read its state
-                for (uint32_t it = 0;; ++it) {
-                    if (!seen) seen = ld_acquire(myflag) >= want;
-                    if (__shfl_sync(0xffffffffu, seen ? 1 : 0, k)) break;
-                    int bad = 0;
-                    if ((it & 15) == 15) {
-                        bad = *(volatile int*)&bs->abort ? 2 : (global_ns() - tw > kWaitLimitNs ? 1 : 0);
-                        bad = __shfl_sync(0xffffffffu, bad, 0);
-                    }
-                    if (bad) {
-                        if (bad == 1 && lane == 0) {
-                            *(volatile int*)&bs->abort = 1;
-                            atomicExch(err, 1);
-                        }
-                        goto done;
-                    }
-                    if (it >= 2) __nanosleep(64);
-                }
-                float run = 0.f, v[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    run += dtv[k][e] * a2;
-                    v[e] = run;
-                }
-                float incl = run;
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const float o = __shfl_up_sync(0xffffffffu, incl, off);
-                    if (lane >= off) incl += o;
-                }
-                const float excl = incl - run;
-                const float last = __shfl_sync(0xffffffffu, incl, 31);
-                float* cs = reinterpret_cast<float*>(smem + K::kOffCs + c * kCsSlotBytes);
-                reinterpret_cast<float4*>(cs)[lane] =
-                    make_float4(excl + v[0], excl + v[1], excl + v[2], excl + v[3]);
-                reinterpret_cast<float4*>(cs + kTile)[lane] =
-                    make_float4(dtv[k][0], dtv[k][1], dtv[k][2], dtv[k][3]);
+            if (prm.chained && U.s > 0) {
+                int bad = 0;
                 if (lane == 0) {
-                    cs[kCsL] = last;
-                    cs[kCsD] = d_h;
-                    cs[kCsMode] = mode;
+                    const int* f = prm.flags + flag_index(prm, U.b, U.s, U.hb);
+                    const int want = 1 + (prm.stall ? (1 << 30) : 0);
+                    bool ok = false;
+                    const uint64_t t0 = global_ns();
+                    for (uint32_t it = 0;; ++it) {
+                        if (ld_acquire(f) >= want) {
+                            ok = true;
+                            break;
+                        }
+                        if (it >= 2) __nanosleep(128);
+                        if ((it & 15) == 15 &&
+                            (*(volatile int*)&bs->abort || global_ns() - t0 > kWaitLimitNs))
+                            break;
+                    }
+                    if (!ok) {
+                        *(volatile int*)&bs->abort = 1;
+                        atomicExch(err, 1);
+                        bad = 1;
+                    }
                 }
-                __syncwarp();
-                mbar_arrive(&bs->cs_full[c]);
-                ++i;
+                if (__any_sync(0xffffffffu, bad)) goto done;
+            }
+            for (int t = U.t_begin; t < U.t_end; ++t) {
+                const int64_t t0 = (int64_t)t * kTile;
+                const int len = (int)min((int64_t)kTile, T - t0);
+                float dtv[2][4];
+#pragma unroll
+                for (int e = 0; e < 2; ++e)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int tt = lane * 4 + q;
+                        dtv[e][q] = (e < np && tt < len) ? __ldg(prm.dt + ((int64_t)U.b * T + t0 + tt) * H + U.hb * np + e)
+                                                         : 0.f;
+                    }
+                float worst = 0.f;
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    if (e >= np) break;
+                    float sdt = dtv[e][0] + dtv[e][1] + dtv[e][2] + dtv[e][3];
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) sdt += __shfl_xor_sync(0xffffffffu, sdt, off);
+                    worst = fmaxf(worst, sdt * fabsf(__ldg(prm.A + U.hb * np + e)) * kLog2e);
+                }
+                const float mode = worst <= kSharedMaskRangeLog2 ? 1.f : 0.f;
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    if (e >= np) break;
+                    const int h = U.hb * np + e;
+                    const float a2 = __ldg(prm.A + h) * kLog2e;
+                    const float d_h = prm.D ? __ldg(prm.D + h) : 0.f;
+                    const int c = hi % kCsSlots;
+                    if (!__all_sync(0xffffffffu,
+                                    wait_bar_idle(&bs->cs_empty[c], ((hi / kCsSlots) & 1) ^ 1, bs, err)))
+                        goto done;
+                    float run = 0.f, v[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        run += dtv[e][q] * a2;
+                        v[q] = run;
+                    }
+                    float incl = run;
+#pragma unroll
+                    for (int off = 1; off < 32; off <<= 1) {
+                        const float o = __shfl_up_sync(0xffffffffu, incl, off);
+                        if (lane >= off) incl += o;
+                    }
+                    const float excl = incl - run;
+                    const float last = __shfl_sync(0xffffffffu, incl, 31);
+                    float* cs = reinterpret_cast<float*>(smem + K::kOffCs + c * kCsSlotBytes);
+                    reinterpret_cast<float4*>(cs)[lane] = make_float4(excl + v[0], excl + v[1], excl + v[2], excl + v[3]);
+                    reinterpret_cast<float4*>(cs + kTile)[lane] = make_float4(dtv[e][0], dtv[e][1], dtv[e][2], dtv[e][3]);
+                    if (lane == 0) {
+                        cs[kCsL] = last;
+                        cs[kCsD] = d_h;
+                        cs[kCsMode] = mode;
+                    }
+                    __syncwarp();
+                    mbar_arrive(&bs->cs_full[c]);
+                    ++hi;
+                }
             }
         }
     } else if (warp == 3) {
-        // ------------------------------------------------------------ chain publisher
-        // The state group stores a head's leaving state and arrives on pub_full; this lane
-        // then makes those stores visible GPU-wide (one fence, cumulative over the stores
-        // ordered before the barrier) and releases the chain flag.
+        // ------------------------------------------------------------ publisher
+        // Per unit: once the chain group has stored the state leaving it, one fence
+        // makes those stores visible GPU-wide and the flag of the next segment's unit
+        // is released.
         if (lane == 0) {
-            int m = 0, np = 0;
-            for (;; ++m) {
+            for (int m = 0;; ++m) {
                 const int ur = m % kURing;
                 if (!wait_bar_idle(&bs->u_full[ur], (m / kURing) & 1, bs, err)) goto done;
                 const int u = bs->uid[ur];
                 mbar_arrive(&bs->u_empty[ur]);
                 if (u < 0) break;
                 const Unit U = decode(prm, u);
-                for (int k = 0; k < kh; ++k, ++np) {
-                    const int ps = np % kPubStages;
-                    if (!wait_bar_idle(&bs->pub_full[ps], (np / kPubStages) & 1, bs, err)) goto done;
-                    __threadfence();
-                    st_release(prm.flags + chain_index(prm, U, U.hb * kh + k), U.kk + 1);
-                    mbar_arrive(&bs->pub_empty[ps]);
+                if (!wait_bar_idle(&bs->pub_full[m & 1], (m >> 1) & 1, bs, err)) goto done;
+                if (prm.chained && U.s < prm.nseg - 1) {
+                    fence_acq_rel_gpu();
+                    st_release(prm.flags + flag_index(prm, U.b, U.s + 1, U.hb), 1);
                 }
+                mbar_arrive(&bs->pub_empty[m & 1]);
             }
         }
     } else if (warp >= 4 && warp < 8) {
         // ------------------------------------------------------------ mask group
-        // Thread j owns token row j of the tile (its TMEM lane). Per unit: the masked
-        // product's A operand, tril(G) for a factored unit. Per item: the skip term
-        // D x_j / q_j (or D x_j) stored into the item's Y'' accumulator, and w o x in
-        // place of the x tile (the B operand of S and of the factored masked product).
-        // An unfactored item first gets its own P = G o exp(cs_j - cs_i) dt_i and is
-        // multiplied with the raw x tile before x is scaled in place.
+        // Thread j owns token row j of the tile (its TMEM lane). Per tile and head:
+        // the skip term D x_j / q_j (or D x_j) stored into the tile's Y'' accumulator
+        // and w o x in place of the x tile (the B operand of S and of the factored
+        // masked product); then P' = tril(C B^T) in place over G. An unfactored tile
+        // first gets each head's P = G o exp(cs_j - cs_i) dt_i in the S slot and is
+        // multiplied with the raw x tiles before they are scaled in place.
         const int wq = warp - 4;
         const int j = tid - 128;
         const int jj = j & 31;
         const uint32_t lb = (uint32_t)(wq * 32) << 16;
-        int m = 0, i = 0, pph = 0, nsh = 0;
+        int m = 0, i = 0, hi = 0, nsh = 0;
         for (;; ++m) {
             const int ur = m % kURing;
             if (!wait_bar_all(&bs->u_full[ur], (m / kURing) & 1, bs, err)) goto done;
             const int u = bs->uid[ur];
             mbar_arrive(&bs->u_empty[ur]);
             if (u < 0) break;
-            if (!wait_bar_all(&bs->cs_full[i % kCsSlots], (i / kCsSlots) & 1, bs, err)) goto done;
-            const bool shared = cs_base[(i % kCsSlots) * (kCsSlotBytes / 4) + kCsMode] != 0.f;
-            if (!wait_bar_all(&bs->g_full, m & 1, bs, err)) goto done;
-            if (shared) {
-                if (!wait_bar_all(&bs->p_empty, (pph & 1) ^ 1, bs, err)) goto done;
-                tc_fence_after();
-                __syncwarp();
-#pragma unroll 1
-                for (int blk = 0; blk < 4; ++blk) {
-                    uint32_t pk[16];
-                    if (blk > wq) {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) pk[e] = 0u;
-                    } else {
-                        float gv[32];
-                        tmem_ld32(tmem + lb + kColG + 32 * blk, gv);
-                        tmem_ld_wait_regs(gv);
-                        if (blk < wq) {
-#pragma unroll
-                            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(gv[2 * e], gv[2 * e + 1]);
-                        } else {
-#pragma unroll
-                            for (int e = 0; e < 16; ++e)   // causal mask: column i kept while i <= row
-                                pk[e] = pack_bf16(2 * e <= jj ? gv[2 * e] : 0.f,
-                                                  2 * e + 1 <= jj ? gv[2 * e + 1] : 0.f);
-                        }
-                    }
-                    tmem_st16(tmem + lb + kColP + 16 * blk, pk);
-                }
-                tmem_st_wait();
-                tc_fence_before();
-                mbar_arrive(&bs->p_full);
-                ++pph;
-                mbar_arrive(&bs->g_empty);
-            } else {
-                tc_fence_after();
-            }
-            for (int k = 0; k < kh; ++k, ++i) {
-                const int c = i % kCsSlots, xs = i % K::kXSlots, ys = i % kYSlots;
-                if (!wait_bar_all(&bs->cs_full[c], (i / kCsSlots) & 1, bs, err)) goto done;
+            const Unit U = decode(prm, u);
+            for (int t = U.t_begin; t < U.t_end; ++t, ++i) {
+                const int xs = i % K::kXSlots, ys = i % kYSlots;
+                if (!wait_bar_all(&bs->cs_full[hi % kCsSlots], (hi / kCsSlots) & 1, bs, err)) goto done;
+                const bool shared = cs_base[(hi % kCsSlots) * (kCsSlotBytes / 4) + kCsMode] != 0.f;
                 if (!wait_bar_all(&bs->x_full[xs], (i / K::kXSlots) & 1, bs, err)) goto done;
                 if (!wait_bar_all(&bs->y_empty[ys], ((i / kYSlots) & 1) ^ 1, bs, err)) goto done;
-                const float* cs = cs_base + c * (kCsSlotBytes / 4);
-                const float L = cs[kCsL], csj = cs[j];
-                const float up = ex2(L - csj);                  // 2^(L - cs_j) <= 1
-                const float w = up * cs[kTile + j];             // w_j = 2^(L - cs_j) dt_j
-                const float dq = cs[kCsD] * (shared ? up : 1.f);  // D / q_j, or D
-                // what the chain and epilogue groups need of this item, kept with its Y''
-                {
-                    float* yi = reinterpret_cast<float*>(smem + K::kOffYInfo + ys * kYInfoBytes);
-                    yi[j] = shared ? ex2(csj - L) : ex2(csj);   // q_j, or 2^cs_j
-                    if (j == 0) {
-                        yi[kTile] = ex2(L);
-                        yi[kTile + 1] = shared ? 1.f : 0.f;
-                    }
-                    mbar_arrive(&bs->yi_full[ys]);
+                if (!shared) {
+                    // the per-head masks need G and go into the S slot (free once the
+                    // previous tile's S, or C h^T, has been read)
+                    if (!wait_bar_all(&bs->g_full, i & 1, bs, err)) goto done;
+                    if (!wait_bar_all(&bs->s_empty, (i & 1) ^ 1, bs, err)) goto done;
                 }
-                uint8_t* sx = smem + K::kOffX + xs * kAtom;
-                uint4 xv[8];
-#pragma unroll
-                for (int c8 = 0; c8 < 8; ++c8) xv[c8] = *reinterpret_cast<const uint4*>(sx + swz(j, c8));
-                // skip term into the Y'' accumulator (drained by the epilogue of item i - 3)
+                float* yi = reinterpret_cast<float*>(smem + K::kOffYInfo + ys * kYInfoBytes);
+                uint8_t* sxp = smem + K::kOffX + xs * K::kXBytes;
                 tc_fence_after();
-                {
+                __syncwarp();
+                float wv[2];
+                for (int e = 0; e < np; ++e) {
+                    const int c = (hi + e) % kCsSlots;
+                    if (!wait_bar_all(&bs->cs_full[c], ((hi + e) / kCsSlots) & 1, bs, err)) goto done;
+                    const float* cs = cs_base + c * (kCsSlotBytes / 4);
+                    const float L = cs[kCsL], csj = cs[j];
+                    const float up = ex2(L - csj);                  // 2^(L - cs_j) <= 1
+                    wv[e] = up * cs[kTile + j];                     // w_j = 2^(L - cs_j) dt_j
+                    const float dq = cs[kCsD] * (shared ? up : 1.f);  // D / q_j, or D
+                    // what the chain and epilogue groups need, kept with the tile's Y''
+                    yi[e * kTile + j] = shared ? ex2(csj - L) : ex2(csj);   // q_j, or 2^cs_j
+                    if (j == 0) yi[kYiEL + e] = ex2(L);
+                    uint8_t* sx = sxp + e * kAtom;
+                    uint4 xv[8];
+#pragma unroll
+                    for (int c8 = 0; c8 < 8; ++c8) xv[c8] = *reinterpret_cast<const uint4*>(sx + swz(j, c8));
+                    // skip term into head e's 64 columns of the tile's Y''
                     const float2 d2 = make_float2(dq, dq);
 #pragma unroll
                     for (int h4 = 0; h4 < 4; ++h4) {
@@ -775,101 +739,130 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const uint32_t xw[4] = {xv[2 * h4 + cc].x, xv[2 * h4 + cc].y, xv[2 * h4 + cc].z,
                                                     xv[2 * h4 + cc].w};
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const float2 v = mul2(d2, unpack_bf16(xw[e]));
-                                pre[8 * cc + 2 * e] = __float_as_uint(v.x);
-                                pre[8 * cc + 2 * e + 1] = __float_as_uint(v.y);
+                            for (int e2 = 0; e2 < 4; ++e2) {
+                                const float2 v = mul2(d2, unpack_bf16(xw[e2]));
+                                pre[8 * cc + 2 * e2] = __float_as_uint(v.x);
+                                pre[8 * cc + 2 * e2 + 1] = __float_as_uint(v.y);
                             }
                         }
-                        tmem_st16(tmem + lb + kColY + 64 * ys + 16 * h4, pre);
+                        tmem_st16(tmem + lb + kColY + 128 * ys + 64 * e + 16 * h4, pre);
                     }
-                    tmem_st_wait();
-                }
-                // w o x over the raw row (re-read: the unfactored path holds no copy)
-                auto scale_in_place = [&]() {
-                    const float2 w2 = make_float2(w, w);
+                    if (shared) {
+                        const float2 w2 = make_float2(wv[e], wv[e]);
 #pragma unroll
-                    for (int c8 = 0; c8 < 8; ++c8) {
-                        const uint4 xr = *reinterpret_cast<const uint4*>(sx + swz(j, c8));
-                        *reinterpret_cast<uint4*>(sx + swz(j, c8)) =
-                            make_uint4(pack_bf16(mul2(w2, unpack_bf16(xr.x))), pack_bf16(mul2(w2, unpack_bf16(xr.y))),
-                                       pack_bf16(mul2(w2, unpack_bf16(xr.z))), pack_bf16(mul2(w2, unpack_bf16(xr.w))));
+                        for (int c8 = 0; c8 < 8; ++c8)
+                            *reinterpret_cast<uint4*>(sx + swz(j, c8)) =
+                                make_uint4(pack_bf16(mul2(w2, unpack_bf16(xv[c8].x))),
+                                           pack_bf16(mul2(w2, unpack_bf16(xv[c8].y))),
+                                           pack_bf16(mul2(w2, unpack_bf16(xv[c8].z))),
+                                           pack_bf16(mul2(w2, unpack_bf16(xv[c8].w))));
+                    } else {
+                        // head e's P = G o exp(cs_j - cs_i) dt_i (exact exponent per element)
+                        const float* dts = cs + kTile;
+#pragma unroll 1
+                        for (int blk = 0; blk < 4; ++blk) {
+                            uint32_t pk[16];
+                            if (blk > wq) {
+#pragma unroll
+                                for (int q2 = 0; q2 < 16; ++q2) pk[q2] = 0u;
+                            } else {
+                                float gv[32];
+                                tmem_ld32(tmem + lb + kColG + 32 * blk, gv);
+                                tmem_ld_wait_regs(gv);
+#pragma unroll
+                                for (int q2 = 0; q2 < 16; ++q2) {
+                                    const int i0 = 32 * blk + 2 * q2;
+                                    const float p0 = i0 <= j ? gv[2 * q2] * ex2(csj - cs[i0]) * dts[i0] : 0.f;
+                                    const float p1 =
+                                        i0 + 1 <= j ? gv[2 * q2 + 1] * ex2(csj - cs[i0 + 1]) * dts[i0 + 1] : 0.f;
+                                    pk[q2] = pack_bf16(p0, p1);
+                                }
+                            }
+                            tmem_st16(tmem + lb + kColS + 64 * e + 16 * blk, pk);
+                        }
                     }
-                    fence_proxy_async_smem();
-                };
+                }
+                if (j == 0) yi[kYiMode] = shared ? 1.f : 0.f;
+                tmem_st_wait();
+                mbar_arrive(&bs->yi_full[ys]);
                 if (shared) {
-                    scale_in_place();
+                    fence_proxy_async_smem();
                     if (j == 0) bs->xmode[xs] = 1;
                     tc_fence_before();
                     mbar_arrive(&bs->wx_full[xs]);
-                } else {
-                    // this head's P = G o exp(cs_j - cs_i) dt_i (exact exponent per element)
-                    if (!wait_bar_all(&bs->p_empty, (pph & 1) ^ 1, bs, err)) goto done;
+                    // P' = tril(G) in bf16 over G's first 64 columns: block blk reads G
+                    // columns 32 blk.. and writes P' columns 16 blk.., both already read
+                    if (!wait_bar_all(&bs->g_full, i & 1, bs, err)) goto done;
                     tc_fence_after();
                     __syncwarp();
-                    const float* dts = cs + kTile;
 #pragma unroll 1
                     for (int blk = 0; blk < 4; ++blk) {
                         uint32_t pk[16];
                         if (blk > wq) {
 #pragma unroll
-                            for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                            for (int q2 = 0; q2 < 16; ++q2) pk[q2] = 0u;
                         } else {
                             float gv[32];
                             tmem_ld32(tmem + lb + kColG + 32 * blk, gv);
                             tmem_ld_wait_regs(gv);
+                            if (blk < wq) {
 #pragma unroll
-                            for (int e = 0; e < 16; ++e) {
-                                const int i0 = 32 * blk + 2 * e;
-                                const float p0 = i0 <= j ? gv[2 * e] * ex2(csj - cs[i0]) * dts[i0] : 0.f;
-                                const float p1 =
-                                    i0 + 1 <= j ? gv[2 * e + 1] * ex2(csj - cs[i0 + 1]) * dts[i0 + 1] : 0.f;
-                                pk[e] = pack_bf16(p0, p1);
+                                for (int q2 = 0; q2 < 16; ++q2) pk[q2] = pack_bf16(gv[2 * q2], gv[2 * q2 + 1]);
+                            } else {
+#pragma unroll
+                                for (int q2 = 0; q2 < 16; ++q2)   // causal mask: column i kept while i <= row
+                                    pk[q2] = pack_bf16(2 * q2 <= jj ? gv[2 * q2] : 0.f,
+                                                       2 * q2 + 1 <= jj ? gv[2 * q2 + 1] : 0.f);
                             }
                         }
                         tmem_st16(tmem + lb + kColP + 16 * blk, pk);
                     }
                     tmem_st_wait();
-                    ++pph;
+                    tc_fence_before();
+                    mbar_arrive(&bs->p_full);
+                } else {
                     if (j == 0) bs->xmode[xs] = 0;
                     tc_fence_before();
                     mbar_arrive(&bs->wx_full[xs]);
-                    if (k == kh - 1) mbar_arrive(&bs->g_empty);
-                    // the product with the raw x tile has read it: now scale it in place
+                    mbar_arrive(&bs->g_empty_mask);     // G has served the masks
+                    // the products with the raw x tiles have read them: now scale in place
                     if (!wait_bar_all(&bs->xr_done, nsh & 1, bs, err)) goto done;
                     ++nsh;
-                    scale_in_place();
+                    for (int e = 0; e < np; ++e) {
+                        uint8_t* sx = sxp + e * kAtom;
+                        const float2 w2 = make_float2(wv[e], wv[e]);
+#pragma unroll
+                        for (int c8 = 0; c8 < 8; ++c8) {
+                            const uint4 xr = *reinterpret_cast<const uint4*>(sx + swz(j, c8));
+                            *reinterpret_cast<uint4*>(sx + swz(j, c8)) =
+                                make_uint4(pack_bf16(mul2(w2, unpack_bf16(xr.x))), pack_bf16(mul2(w2, unpack_bf16(xr.y))),
+                                           pack_bf16(mul2(w2, unpack_bf16(xr.z))), pack_bf16(mul2(w2, unpack_bf16(xr.w))));
+                        }
+                    }
+                    fence_proxy_async_smem();
                     mbar_arrive(&bs->wx2_full);
                 }
-                mbar_arrive(&bs->cs_empty[c]);
+                for (int e = 0; e < np; ++e) mbar_arrive(&bs->cs_empty[(hi + e) % kCsSlots]);
+                hi += np;
             }
         }
     } else if (warp >= 8 && warp < 16) {
         // ------------------------------------------------------------ chain group
-        // Thread (q, lane) of warp 8 + 4 ph + q owns TMEM lane r = 32q + lane, i.e. state
-        // row r (and r + 128), head-dim columns 32ph..32ph+31. Per item: the leaving
-        // state 2^L h + S onto the chain, and the operand of C h^T (bf16 2^L h, or h)
-        // into the item's operand buffer. The next item's entering state is loaded
-        // while this one is finished.
+        // Thread (q, lane) of warp 8 + 4 ph + q owns TMEM lane r = 32q + lane and head-dim
+        // columns 32ph..32ph+31. The pair's state is V pieces of 32 values per thread,
+        // carried in registers through the unit's tiles: piece v is head v of the pair
+        // (state 128), or state rows r + 128 v of the one head (state 256); its S sits
+        // at TMEM columns 64 v, its operand in atom v. Per tile: the operand of
+        // C h^T (bf16 2^L h, or h), then h <- 2^L h + S. At the unit's end the state
+        // goes to the next segment (or the final states).
+        constexpr int V = K::kNP * K::kMH;   // 2
         const int q = warp & 3;
         const int ph = (warp - 8) >> 2;
         const int r = q * 32 + lane;
         const uint32_t lb = (uint32_t)(q * 32) << 16;
         const int N = prm.N;
-        constexpr bool kPrefetch = K::kMHalves == 1;
-        float hv[32];
-        bool have_h = false;          // hv holds the next item's entering state (row r)
-        auto load_rows = [&](const float* src, int n, float (&v)[32]) {
-            if (src && n < N) {
-                const float* s0 = src + (int64_t)(32 * ph) * N + n;
-#pragma unroll
-                for (int p = 0; p < 32; ++p) v[p] = __ldcg(s0 + (int64_t)p * N);
-            } else {
-#pragma unroll
-                for (int p = 0; p < 32; ++p) v[p] = 0.f;
-            }
-        };
-        int np = 0;
+        const int nv = np * K::kMH;
+        float hv[V][32];
         int m = 0, i = 0;
         for (;; ++m) {
             const int ur = m % kURing;
@@ -878,72 +871,82 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&bs->u_empty[ur]);
             if (u < 0) break;
             const Unit U = decode(prm, u);
-            for (int k = 0; k < kh; ++k, ++i) {
-                const int ys = i % kYSlots, ss = i % K::kSSlots, hs = i % K::kHYSlots;
-                const int h = U.hb * kh + k;
+            for (int t = U.t_begin; t < U.t_end; ++t, ++i) {
+                const int ys = i % kYSlots;
                 if (!wait_bar_all(&bs->yi_full[ys], (i / kYSlots) & 1, bs, err)) goto done;
                 const float* yi = reinterpret_cast<const float*>(smem + K::kOffYInfo + ys * kYInfoBytes);
-                const float eL = yi[kTile];
-                const bool shared = yi[kTile + 1] != 0.f;
-                const float sc = shared ? eL : 1.f;   // the operand: 2^L h, or h
-                const float* src = entry_src(prm, U, h);
-                float* dst = chain_buf(prm, U, h);
-                if (kPrefetch && !have_h) load_rows(src, r, hv);
-                have_h = false;
-                if (!wait_bar_all(&bs->hy_free[hs], ((i / K::kHYSlots) & 1) ^ 1, bs, err)) goto done;
-                if (!wait_bar_all(&bs->s_full[ss], (i / K::kSSlots) & 1, bs, err)) goto done;
-                if (!wait_bar_all(&bs->pub_empty[np % kPubStages], ((np / kPubStages) & 1) ^ 1, bs, err))
-                    goto done;
-                tc_fence_after();
-                uint8_t* hy = smem + K::kOffHY + hs * K::kHYBytes;
-#pragma unroll 1
-                for (int mh = 0; mh < K::kMHalves; ++mh) {
-                    const int n = r + 128 * mh;
-                    if (!kPrefetch) load_rows(src, n, hv);
+                const bool shared = yi[kYiMode] != 0.f;
+                if (t == U.t_begin) {
+                    // the state entering the unit (its flag was acquired before the tile's
+                    // Y'' info was published)
 #pragma unroll
-                    for (int pc = 0; pc < 2; ++pc) {   // 16 head-dim columns at a time
-                        float sv[16];
-                        tmem_ld16(tmem + lb + kColS + 64 * ss + 64 * mh + 32 * ph + 16 * pc, sv);
-                        tmem_ld_wait_regs(sv);
-                        if (n < N) {
-                            float* d = dst + (int64_t)(32 * ph + 16 * pc) * N + n;
+                    for (int v = 0; v < V; ++v) {
+                        const int e = v / K::kMH, mh = v % K::kMH;
+                        const int n = r + 128 * mh;
+                        const float* src = v < nv ? entry_src(prm, U, U.hb * np + e) : nullptr;
+                        if (src && n < N) {
+                            const float* s0 = src + (int64_t)(32 * ph) * N + n;
 #pragma unroll
-                            for (int e = 0; e < 16; ++e) __stcg(d + (int64_t)e * N, fmaf(eL, hv[16 * pc + e], sv[e]));
+                            for (int p2 = 0; p2 < 32; ++p2) hv[v][p2] = __ldcg(s0 + (int64_t)p2 * N);
+                        } else {
+#pragma unroll
+                            for (int p2 = 0; p2 < 32; ++p2) hv[v][p2] = 0.f;
                         }
-                        uint32_t op[8];
+                    }
+                }
+                if (!wait_bar_all(&bs->h_free, (i & 1) ^ 1, bs, err)) goto done;
+                if (!wait_bar_all(&bs->s_full, i & 1, bs, err)) goto done;
+                tc_fence_after();
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            op[e] = pack_bf16(sc * hv[16 * pc + 2 * e], sc * hv[16 * pc + 2 * e + 1]);
-                        *reinterpret_cast<uint4*>(hy + swz(n, 4 * ph + 2 * pc)) = make_uint4(op[0], op[1], op[2], op[3]);
-                        *reinterpret_cast<uint4*>(hy + swz(n, 4 * ph + 2 * pc + 1)) =
-                            make_uint4(op[4], op[5], op[6], op[7]);
+                for (int v = 0; v < V; ++v) {
+                    if (v >= nv) break;
+                    const float eL = yi[kYiEL + v / K::kMH];
+                    const float sc = shared ? eL : 1.f;   // the operand: 2^L h, or h
+                    uint8_t* ha = smem + K::kOffH + v * kAtom;
+#pragma unroll
+                    for (int pc = 0; pc < 4; ++pc) {   // 8 head-dim columns at a time
+                        float sv[8];
+                        tmem_ld8(tmem + lb + kColS + 64 * v + 32 * ph + 8 * pc, sv);
+                        tmem_ld_wait_regs(sv);
+                        uint32_t op[4];
+#pragma unroll
+                        for (int e2 = 0; e2 < 4; ++e2)
+                            op[e2] = pack_bf16(sc * hv[v][8 * pc + 2 * e2], sc * hv[v][8 * pc + 2 * e2 + 1]);
+                        *reinterpret_cast<uint4*>(ha + swz(r, 4 * ph + pc)) = make_uint4(op[0], op[1], op[2], op[3]);
+#pragma unroll
+                        for (int e2 = 0; e2 < 8; ++e2) hv[v][8 * pc + e2] = fmaf(eL, hv[v][8 * pc + e2], sv[e2]);
                     }
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
-                mbar_arrive(&bs->h_full[hs]);
-                if (shared) mbar_arrive(&bs->s_empty[ss]);
-                mbar_arrive(&bs->pub_full[np % kPubStages]);
-                ++np;
-                // the next item of this unit: its entering state (its chain flag was
-                // acquired before its Y'' info was published)
-                if (kPrefetch && k + 1 < kh) {
-                    const int yn = (i + 1) % kYSlots;
-                    if (!wait_bar_all(&bs->yi_full[yn], ((i + 1) / kYSlots) & 1, bs, err)) goto done;
-                    load_rows(entry_src(prm, U, h + 1), r, hv);
-                    have_h = true;
+                if (shared) mbar_arrive(&bs->s_empty);
+                mbar_arrive(&bs->h_full);
+            }
+            // the state leaving the unit
+            if (!wait_bar_all(&bs->pub_empty[m & 1], ((m >> 1) & 1) ^ 1, bs, err)) goto done;
+#pragma unroll
+            for (int v = 0; v < V; ++v) {
+                if (v >= nv) break;
+                const int e = v / K::kMH, mh = v % K::kMH;
+                const int n = r + 128 * mh;
+                float* dst = exit_dst(prm, U, U.hb * np + e);
+                if (dst && n < N) {
+                    float* d0 = dst + (int64_t)(32 * ph) * N + n;
+#pragma unroll
+                    for (int p2 = 0; p2 < 32; ++p2) __stcg(d0 + (int64_t)p2 * N, hv[v][p2]);
                 }
             }
+            mbar_arrive(&bs->pub_full[m & 1]);
         }
     } else if (warp >= 16) {
         // ------------------------------------------------------------ epilogue group
-        // Thread (q, lane) of warp 16 + q owns token row r = 32q + lane (TMEM lane) and
-        // all 64 head-dim columns: y = q_r Y'' (or Y'' + 2^cs_r R) staged in the warp's
-        // own 4 KB (or, for the 256-wide state, over the item's operand buffer once the
-        // state product has read it), then one TMA store of the warp's 32 rows.
+        // Thread (q, lane) of warp 16 + q owns token row r = 32q + lane (TMEM lane): per
+        // tile and head y = q_r Y'' (or Y'' + 2^cs_r R) over all 64 columns, staged in
+        // the warp's own 4 KB, then one TMA store of the warp's 32 rows.
         const int q = warp - 16;
         const int r = q * 32 + lane;
         const uint32_t lb = (uint32_t)(q * 32) << 16;
+        uint8_t* stg = smem + K::kOffStage;
         int m = 0, i = 0;
         for (;; ++m) {
             const int ur = m % kURing;
@@ -952,56 +955,51 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&bs->u_empty[ur]);
             if (u < 0) break;
             const Unit U = decode(prm, u);
-            for (int k = 0; k < kh; ++k, ++i) {
-                const int ys = i % kYSlots, ss = i % K::kSSlots, hs = i % K::kHYSlots;
+            for (int t = U.t_begin; t < U.t_end; ++t, ++i) {
+                const int ys = i % kYSlots;
+                const int64_t t0 = (int64_t)t * kTile;
                 if (!wait_bar_all(&bs->y_full[ys], (i / kYSlots) & 1, bs, err)) goto done;
                 tc_fence_after();
                 const float* yi = reinterpret_cast<const float*>(smem + K::kOffYInfo + ys * kYInfoBytes);
-                const float f = yi[r];
-                const bool shared = yi[kTile + 1] != 0.f;
-                const float2 f2 = make_float2(f, f);
-                uint8_t* hy = K::kOwnStaging ? smem + K::kOffStage : smem + K::kOffHY + hs * K::kHYBytes;
-                if (K::kOwnStaging) {
+                const bool shared = yi[kYiMode] != 0.f;
+                for (int e = 0; e < np; ++e) {
+                    const float f = yi[e * kTile + r];
+                    const float2 f2 = make_float2(f, f);
                     // the warp's previous store has read its staging rows
                     if (lane == 0) bulk_wait_group_read0();
                     __syncwarp();
-                }
 #pragma unroll 1
-                for (int pc = 0; pc < 4; ++pc) {
-                    float yv[16], rv[16];
-                    tmem_ld16(tmem + lb + kColY + 64 * ys + 16 * pc, yv);
-                    if (shared) {
-                        tmem_ld_wait_regs(yv);
-                    } else {
-                        tmem_ld16(tmem + lb + kColS + 64 * ss + 16 * pc, rv);
-                        tmem_ld_wait_regs(yv, rv);
-                    }
-#pragma unroll
-                    for (int cc = 0; cc < 2; ++cc) {
-                        uint32_t o[4];
-#pragma unroll
-                        for (int e2 = 0; e2 < 4; ++e2) {
-                            const int x0 = 8 * cc + 2 * e2;
-                            const float2 yy = make_float2(yv[x0], yv[x0 + 1]);
-                            o[e2] = pack_bf16(shared ? mul2(f2, yy) : fma2(f2, make_float2(rv[x0], rv[x0 + 1]), yy));
+                    for (int pc = 0; pc < 4; ++pc) {
+                        float yv[16], rv[16];
+                        tmem_ld16(tmem + lb + kColY + 128 * ys + 64 * e + 16 * pc, yv);
+                        if (shared) {
+                            tmem_ld_wait_regs(yv);
+                        } else {
+                            tmem_ld16(tmem + lb + kColS + 64 * e + 16 * pc, rv);
+                            tmem_ld_wait_regs(yv, rv);
                         }
-                        *reinterpret_cast<uint4*>(hy + swz(r, 2 * pc + cc)) = make_uint4(o[0], o[1], o[2], o[3]);
+#pragma unroll
+                        for (int cc = 0; cc < 2; ++cc) {
+                            uint32_t o[4];
+#pragma unroll
+                            for (int e2 = 0; e2 < 4; ++e2) {
+                                const int x0 = 8 * cc + 2 * e2;
+                                const float2 yy = make_float2(yv[x0], yv[x0 + 1]);
+                                o[e2] = pack_bf16(shared ? mul2(f2, yy) : fma2(f2, make_float2(rv[x0], rv[x0 + 1]), yy));
+                            }
+                            *reinterpret_cast<uint4*>(stg + swz(r, 2 * pc + cc)) = make_uint4(o[0], o[1], o[2], o[3]);
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0 && t0 + 32 * q < T) {   // rows past T are clipped by the store
+                        tma_store_4d(&tm_y, stg + q * (kAtom / 4), 0, U.hb * np + e, (int)(t0 + 32 * q), U.b);
+                        bulk_commit_group();
                     }
                 }
                 tc_fence_before();
                 mbar_arrive(&bs->y_empty[ys]);
-                if (!shared) mbar_arrive_cnt(&bs->s_empty[ss], 2);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    if (U.t0 + 32 * q < T) {   // rows past T are clipped by the store
-                        tma_store_4d(&tm_y, hy + q * (kAtom / 4), 0, U.hb * kh + k, (int)(U.t0 + 32 * q), U.b);
-                        bulk_commit_group();
-                        if (!K::kOwnStaging) bulk_wait_group_read0();
-                    }
-                    if (!K::kOwnStaging) mbar_arrive(&bs->hy_free[hs]);
-                }
-                __syncwarp();
+                if (!shared) mbar_arrive_cnt(&bs->s_empty, 2);
             }
         }
     }
@@ -1042,21 +1040,17 @@ int fused_state_capacity(int64_t N) {
 }
 
 int fused_kheads(int64_t H, int64_t G, int ns) {
-    const int64_t hpg = H / G;
-    const int want = ns == 256 ? 8 : 4;
-    for (int k = want; k > 1; --k)
-        if (hpg % k == 0) return k;
-    return 1;
+    return (ns == 128 && (H / G) % 2 == 0) ? 2 : 1;
 }
 
 size_t fused_sync_ints(const Dims& d, int nseg) { return 2 + (size_t)(d.b * nseg * d.H); }
 
 cudaError_t launch_fused(const FusedLaunch& a, cudaStream_t st) {
     const Dims& d = a.d;
-    cudaError_t e = cudaMemsetAsync(a.sync_ints, 0, sizeof(int) * fused_sync_ints(d, a.nseg), st);
-    if (e != cudaSuccess) return e;
     const int ns = fused_state_capacity(d.N);
-    if (ns == 0 || a.nseg < 1 || a.seg_tiles < 1) return cudaErrorInvalidValue;
+    if (ns == 0 || a.nseg < 1 || a.seg_tiles < 1 || a.kheads < 1 || a.kheads > 2 || d.H % a.kheads != 0 ||
+        (ns == 256 && a.kheads != 1))
+        return cudaErrorInvalidValue;
     Params prm = {};
     prm.dt = a.dt;
     prm.A = a.A;
@@ -1074,13 +1068,14 @@ cudaError_t launch_fused(const FusedLaunch& a, cudaStream_t st) {
     prm.kheads = a.kheads;
     prm.batch = (int)d.b;
     const int64_t ntiles = (d.T + kTile - 1) / kTile;
-    const int64_t nunits = (int64_t)a.seg_tiles * a.nseg * d.b * (d.H / a.kheads);
+    const int64_t nunits = (int64_t)a.nseg * d.b * (d.H / a.kheads);
     if (nunits > INT32_MAX / 2 || d.T > INT32_MAX || (int64_t)a.seg_tiles * a.nseg < ntiles)
         return cudaErrorInvalidValue;
     prm.nunits = (int)nunits;
     prm.ntiles = (int)ntiles;
     prm.seg_tiles = a.seg_tiles;
     prm.nseg = a.nseg;
+    prm.chained = a.chained;
     prm.stall = a.stall;
     return ns == 128 ? launch_ns<128>(a, prm, st) : launch_ns<256>(a, prm, st);
 }

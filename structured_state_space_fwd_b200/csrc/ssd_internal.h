@@ -61,10 +61,11 @@ struct FusedLaunch {
     const float* A;
     const float* D;
     const float* init;         // [b,H,P,N] or null
-    float* finalbuf;           // [b,H,P,N]: the last segment's chain, final states on return
+    float* finalbuf;           // [b,H,P,N] final states, or null
     float* segbuf;             // [b,nseg,H,P,N] states entering segments 1.. (nseg > 1)
-    int* sync_ints;            // fused_sync_ints ints, zeroed by the launch
+    int* sync_ints;            // fused_sync_ints ints, zeroed by the caller
     int kheads, seg_tiles, nseg;
+    int chained;               // segment s > 0 takes its entering state from segment s - 1's unit
     int stall;                 // test builds: make chain waits run out
 };
 cudaError_t launch_fused(const FusedLaunch& a, cudaStream_t st);
