@@ -130,9 +130,9 @@ SSD_API ssd_status_t ssd_fwd(const ssd_shape_t* shape,
  *   (ssd_fwd_workspace_size) exceeds 64 MiB is rejected with
  *   SSD_ERR_UNSUPPORTED before anything is enqueued; ssd_last_error_detail()
  *   then says so. The library allocates nothing on this path.
- *   The first call on a device looks up that device's scratch address
- *   (cudaGetSymbolAddress, with the device current); make that first call
- *   before any stream capture. All calls on a device share the one array and
+ *   Every call looks up the current device's copy of the array
+ *   (cudaGetSymbolAddress), so a context recreated after cudaDeviceReset is
+ *   served too. All calls on a device share the one array and
  *   it keeps the last call's contents, which no call relies on; calls that can
  *   overlap on the GPU (different streams, or different host threads without
  *   ordering) race on it and must be serialized by the caller.
@@ -166,9 +166,12 @@ SSD_API ssd_status_t ssd_fwd_host_workspace_size(const ssd_shape_t* shape, size_
  * workspace, runs ssd_fwd there, copies y (and final_states when non-NULL)
  * back, and returns when everything is done, so the host outputs are ready on
  * return. The batch is processed in up to 8 slices of rows: the forward of a
- * slice runs on `stream` while two streams the call creates (and destroys
- * before returning) copy the next slice in and the previous one out; the
- * copies start after the work already queued on `stream`. Host buffers should be page-locked for full
+ * slice runs on `stream` while two copy streams copy the next slice in and
+ * the previous one out; the copies start after the work already queued on
+ * `stream`. The copy streams and their events come from a per-device pool
+ * that the library keeps until the process exits: the first call creates a
+ * set, later calls reuse it (concurrent calls each take their own set), so a
+ * steady stream of calls creates no CUDA objects. Host buffers should be page-locked for full
  * copy bandwidth; pageable memory works but is slower. The device workspace
  * must hold ssd_fwd_host_workspace_size() bytes. Returns SSD_ERR_TIMEOUT (as
  * ssd_fwd_check) when the fused kernel's bounded waits gave up.
@@ -179,6 +182,53 @@ SSD_API ssd_status_t ssd_fwd_host(const ssd_shape_t* shape,
                           const float* initial_states,
                           void* y, float* final_states,
                           void* device_workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Packed variable-length documents (Knowl 8, variable-length processing:
+ * sequences of different lengths are concatenated into one flat sequence with
+ * no padding, and the transition a_t is 0 at each document's first token, so
+ * the state restarts at every boundary). Equivalent to one ssd_fwd per
+ * document on its slice of the pack, computed in one pass over the pack.
+ *   shape              batch = 1; seqlen = T, the packed length; the other
+ *                      fields as for ssd_fwd (chunk_size not used). Supported:
+ *                      dtype SSD_BF16, headdim 64, dstate a multiple of 16 up
+ *                      to 256 (else SSD_ERR_UNSUPPORTED, nothing enqueued).
+ *   x, dt, B, C, y     the pack, laid out as ssd_fwd's tensors with b = 1.
+ *   A, D               as for ssd_fwd.
+ *   cu_seqlens         DEVICE int32 [n_docs + 1]: document k is tokens
+ *                      cu_seqlens[k] .. cu_seqlens[k+1] - 1; the list must
+ *                      run from 0 to T, non-decreasing (empty documents are
+ *                      allowed). It is read on the device: a malformed list is
+ *                      clamped into [0, T] (nothing outside the pack is read or
+ *                      written) and reported by ssd_fwd_varlen_check as
+ *                      SSD_ERR_INVALID_ARG.
+ *   n_docs             >= 0 (0 only with T = 0: nothing to do).
+ *   initial_states     [n_docs, H, P, N] fp32 or NULL (zeros).
+ *   final_states       [n_docs, H, P, N] fp32 or NULL (not written); an empty
+ *                      document's final state is its initial state.
+ *   workspace          ssd_fwd_varlen_workspace_size() bytes, 16-byte aligned;
+ *                      holds the call's status words and the document order.
+ * Two kernel launches: the documents are ranked by length (identity order
+ * beyond 8192 documents) and checked, then the single-pass kernel runs one
+ * unit per (document, head block), the longest documents first; a document's
+ * tiles start at its first token, its tokens past the end get dt = 0 and rows
+ * of the next document are never written.
+ */
+SSD_API ssd_status_t ssd_fwd_varlen_workspace_size(const ssd_shape_t* shape, int64_t n_docs,
+                                                   size_t* bytes);
+SSD_API ssd_status_t ssd_fwd_varlen(const ssd_shape_t* shape,
+                                    const void* x, const float* dt, const float* A,
+                                    const void* B, const void* C, const float* D,
+                                    const int32_t* cu_seqlens, int64_t n_docs,
+                                    const float* initial_states,
+                                    void* y, float* final_states,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+/* Status of the last ssd_fwd_varlen on `workspace` (waits for `stream`):
+ * SSD_ERR_INVALID_ARG for a malformed cu_seqlens, SSD_ERR_TIMEOUT when a
+ * bounded wait inside the kernel gave up, else SSD_OK. */
+SSD_API ssd_status_t ssd_fwd_varlen_check(const ssd_shape_t* shape, int64_t n_docs,
+                                          const void* workspace, size_t workspace_bytes,
+                                          void* stream);
 
 /*
  * Recurrent (linear) form for the decoding mode of the layer (Knowl 1, linear

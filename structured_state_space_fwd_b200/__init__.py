@@ -24,7 +24,8 @@ from ._lib import (SSD_BF16, SSD_F32, SSDError, ShapeT, check, lib, lib_path,  #
 
 __all__ = ["ssd_fwd", "ssd_fwd_host", "ssd_fwd_workspace_size", "ssd_fwd_plan", "ssd_fwd_check",
            "ssd_step", "ssd_fwd_cp", "ssd_cp_begin", "ssd_cp_end", "ssd_cp_record_floats",
-           "ssd_gated_rmsnorm", "ssd_fwd_varlen", "ssd_chunk_cumsum",
+           "ssd_gated_rmsnorm", "ssd_fwd_varlen", "ssd_fwd_varlen_workspace_size",
+           "ssd_fwd_varlen_check", "ssd_chunk_cumsum",
            "ssd_chunk_state", "ssd_state_passing", "ssd_chunk_scan", "SSDError", "make_shape",
            "lib_path"]
 
@@ -103,47 +104,72 @@ def ssd_fwd(x, dt, A, B, C, D=None, chunk_size: int = 256, initial_states=None,
     return (y, final_states) if return_final_states else y
 
 
+def check_cu_seqlens(cu_seqlens, T: int) -> list[int]:
+    """A host-side offset list as ints, or ValueError unless it runs from 0 to T, non-decreasing."""
+    cu = [int(v) for v in (cu_seqlens.tolist() if hasattr(cu_seqlens, "tolist") else cu_seqlens)]
+    if len(cu) < 2 or cu[0] != 0 or cu[-1] != T or any(b < a for a, b in zip(cu, cu[1:])):
+        raise ValueError("cu_seqlens must run from 0 to T, non-decreasing")
+    return cu
+
+
+def ssd_fwd_varlen_workspace_size(shape: ShapeT, n_docs: int) -> int:
+    n = ctypes.c_size_t(0)
+    check(lib().ssd_fwd_varlen_workspace_size(ctypes.byref(shape), ctypes.c_int64(n_docs), ctypes.byref(n)),
+          "ssd_fwd_varlen_workspace_size")
+    return int(n.value)
+
+
 def ssd_fwd_varlen(x, dt, A, B, C, D=None, cu_seqlens=None, chunk_size: int = 256,
                    initial_states=None, return_final_states: bool = False, y=None,
-                   final_states=None, stream=None):
+                   final_states=None, workspace=None, stream=None):
     """Packed variable-length documents (Knowl 8): batch row 0 of x [1, T, H, P]
     holds documents at tokens cu_seqlens[k] .. cu_seqlens[k+1]-1, each an
     independent sequence (a_t = 0 at its first token). Returns y, or
     (y, final_states [n_docs, H, P, N]); initial_states [n_docs, H, P, N] or None.
 
-    A document is a contiguous slice of every packed tensor, so each runs as one
-    ssd_fwd call on views of the caller's buffers (one workspace, reused in stream
-    order); nothing is copied and every step runs in the library's kernels.
+    cu_seqlens: a device int32 tensor [n_docs + 1] (passed as is), or a host list /
+    tensor (copied to the device). One ssd_fwd_varlen call: every document runs in
+    the single-pass kernel's one launch.
     """
-    # device, dtype and alignment are ssd_fwd's checks, per document
-    _need(x, "x", device=False)
+    _need(x, "x")
     if x.shape[0] != 1:
         raise ValueError("packed documents need batch 1 (x [1, T, H, P])")
-    cu = [int(v) for v in (cu_seqlens.tolist() if hasattr(cu_seqlens, "tolist") else cu_seqlens)]
-    T = x.shape[1]
-    if len(cu) < 2 or cu[0] != 0 or cu[-1] != T or any(b < a for a, b in zip(cu, cu[1:])):
-        raise ValueError("cu_seqlens must run from 0 to T, non-decreasing")
-    ndoc = len(cu) - 1
+    if isinstance(cu_seqlens, torch.Tensor) and cu_seqlens.is_cuda:
+        if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_contiguous() or cu_seqlens.dim() != 1:
+            raise ValueError("device cu_seqlens must be a contiguous 1-D int32 tensor")
+        if cu_seqlens.numel() < 1:
+            raise ValueError("cu_seqlens needs at least one entry")
+        cu_dev = cu_seqlens   # checked on the device; see ssd_fwd_varlen_check
+    else:
+        cu_dev = torch.tensor(check_cu_seqlens(cu_seqlens, x.shape[1]), dtype=torch.int32).to(x.device)
+    ndoc = cu_dev.numel() - 1
     H, P, N = x.shape[2], x.shape[3], B.shape[3]
+    shape = make_shape(x, B, chunk_size)
     if initial_states is not None:
-        _need(initial_states, "initial_states", torch.float32, device=False)
+        _need(initial_states, "initial_states", torch.float32)
         if tuple(initial_states.shape) != (ndoc, H, P, N):
             raise ValueError("initial_states must be [n_docs, H, P, N]")
     if y is None:
         y = torch.empty_like(x)
-    if final_states is None:
+    if final_states is None and return_final_states:
         final_states = torch.empty((ndoc, H, P, N), dtype=torch.float32, device=x.device)
-    # one workspace, large enough for every document length in the pack
-    need = max(ssd_fwd_workspace_size(make_shape(x[:, :L], B[:, :L], chunk_size))
-               for L in sorted({b - a for a, b in zip(cu, cu[1:])}))
-    ws = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
-    for k in range(ndoc):
-        a, b = cu[k], cu[k + 1]
-        ssd_fwd(x[:, a:b], dt[:, a:b], A, B[:, a:b], C[:, a:b], D, chunk_size=chunk_size,
-                initial_states=initial_states[k:k + 1] if initial_states is not None else None,
-                return_final_states=True, y=y[:, a:b], final_states=final_states[k:k + 1],
-                workspace=ws, stream=stream)
+    nbytes = ssd_fwd_varlen_workspace_size(shape, ndoc)
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=x.device)
+    check(lib().ssd_fwd_varlen(ctypes.byref(shape), _p(x), _p(dt), _p(A), _p(B), _p(C), _p(D),
+                               _p(cu_dev), ctypes.c_int64(ndoc), _p(initial_states), _p(y),
+                               _p(final_states), _p(workspace), ctypes.c_size_t(nbytes),
+                               _stream(stream)), "ssd_fwd_varlen")
     return (y, final_states) if return_final_states else y
+
+
+def ssd_fwd_varlen_check(shape: ShapeT, n_docs: int, workspace, stream=None):
+    """Status of the last ssd_fwd_varlen on `workspace` (waits for the stream): raises
+    SSDError with SSD_ERR_INVALID_ARG for malformed cu_seqlens, SSD_ERR_TIMEOUT when a
+    bounded wait gave up."""
+    nbytes = ssd_fwd_varlen_workspace_size(shape, n_docs)
+    check(lib().ssd_fwd_varlen_check(ctypes.byref(shape), ctypes.c_int64(n_docs), _p(workspace),
+                                     ctypes.c_size_t(nbytes), _stream(stream)), "ssd_fwd_varlen_check")
 
 
 def ssd_fwd_check(shape: ShapeT, workspace, stream=None):

@@ -47,6 +47,12 @@ _SIGS = {
     "ssd_fwd_host": ([ctypes.POINTER(ShapeT)] + [_VP] * 10 + [ctypes.c_size_t, _VP], ctypes.c_int),
     "ssd_fwd_no_alloc": ([ctypes.POINTER(ShapeT)] + [_VP] * 10, ctypes.c_int),
     "ssd_fwd_check": ([ctypes.POINTER(ShapeT), _VP, ctypes.c_size_t, _VP], ctypes.c_int),
+    "ssd_fwd_varlen_workspace_size": ([ctypes.POINTER(ShapeT), ctypes.c_int64,
+                                       ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
+    "ssd_fwd_varlen": ([ctypes.POINTER(ShapeT)] + [_VP] * 7 + [ctypes.c_int64] + [_VP] * 4
+                       + [ctypes.c_size_t, _VP], ctypes.c_int),
+    "ssd_fwd_varlen_check": ([ctypes.POINTER(ShapeT), ctypes.c_int64, _VP, ctypes.c_size_t, _VP],
+                             ctypes.c_int),
     "ssd_step": ([ctypes.POINTER(ShapeT)] + [_VP] * 9, ctypes.c_int),
     "ssd_cp_record_floats": ([ctypes.POINTER(ShapeT), ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
     "ssd_cp_workspace_size": ([ctypes.POINTER(ShapeT), ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),

@@ -9,6 +9,8 @@
 #include <cstdlib>
 #include <cstring>
 #include <initializer_list>
+#include <mutex>
+#include <vector>
 
 #include "ssd.h"
 #include "ssd_internal.h"
@@ -105,9 +107,16 @@ bool fused_ok(const ssd::Dims& d) {
 // few chains (batch rows x head pairs) and many tiles that sets the time, and the
 // states entering all segments are computed first instead (segment states, a
 // scan over them), so that every segment can run at once.
-constexpr int64_t kChainedMinChains = 112;       // fewer chains than this: compute entering states first
+#ifndef SSD_CHAINED_MIN_CHAINS
+#define SSD_CHAINED_MIN_CHAINS 112
+#endif
+#ifndef SSD_TARGET_UNITS
+#define SSD_TARGET_UNITS (4 * 148)
+#endif
+constexpr int64_t kChainedMinChains = SSD_CHAINED_MIN_CHAINS;  // fewer chains: compute entering states first
 constexpr int64_t kSegmentMinTiles = 8;
-constexpr int64_t kTargetUnits = 4 * 148;        // units wanted: about four waves of CTAs
+constexpr int64_t kTargetUnits = SSD_TARGET_UNITS;             // units wanted: about four waves of CTAs
+constexpr int64_t kSmCount = 148;
 
 int64_t fused_chains(const ssd::Dims& d) {
     const int ns = ssd::fused_state_capacity(d.N);
@@ -151,7 +160,10 @@ SegPlan seg_plan(const ssd::Dims& d, Path path) {
     sp.chained = path != Path::Segmented;
     const int64_t ntiles = d.T > 0 ? (d.T + 127) / 128 : 1;
     const int64_t chains = std::max<int64_t>(1, d.b * (d.H / sp.kh));
+    // Chained segments of one chain run one after another, so with no more
+    // chains than SMs splitting them only adds hand-offs to the critical path.
     int64_t nseg = (kTargetUnits + chains - 1) / chains;
+    if (sp.chained && chains <= kSmCount) nseg = 1;
     if (path == Path::Segmented) nseg = std::max<int64_t>(2, nseg);
     nseg = std::max<int64_t>(1, std::min(nseg, ntiles));
     int64_t K = (ntiles + nseg - 1) / nseg;
@@ -290,6 +302,7 @@ ssd_status_t run_fwd(const ssd::Dims& d, const void* x, const float* dt, const f
         a.nseg = w.sp.nseg;
         a.chained = w.sp.chained ? 1 : 0;
         a.stall = test_stall();
+        a.y = y;
         return cuda_status("fused forward", ssd::launch_fused(a, stream));
     }
     float* cs = (float*)(ws + w.off_cs);
@@ -360,13 +373,14 @@ size_t cp_record_floats(const ssd::Dims& d) {
 // the forward and the copies out of different slices overlap (the two copy
 // directions use separate copy engines). Each slice has its own forward
 // workspace, so every slice's device status word survives until it is read.
+constexpr int kHostMaxSlices = 8;
 struct HostPlan {
     int64_t nslices, rows;     // slices of `rows` batch rows (the last may be shorter)
     size_t ws_slice;           // forward workspace of one full slice
 };
 HostPlan host_plan(const ssd::Dims& d) {
     HostPlan hp;
-    hp.nslices = d.b < 8 ? (d.b > 0 ? d.b : 1) : 8;
+    hp.nslices = d.b < kHostMaxSlices ? (d.b > 0 ? d.b : 1) : kHostMaxSlices;
     // slices start at row boundaries: keep the 16-byte alignment of every tensor
     if (d.b > 0) {
         const Sizes z = sizes_of(d);
@@ -379,6 +393,121 @@ HostPlan host_plan(const ssd::Dims& d) {
     ds.b = hp.rows;
     hp.ws_slice = align_up(fwd_workspace(ds).total, 256);
     return hp;
+}
+
+
+// The two copy streams and the events of one ssd_fwd_host call. Sets are kept
+// per device in a pool and reused: a call takes one (creating it only when all
+// are in use by concurrent calls) and returns it when done, so repeated calls
+// create no CUDA objects. The pool lives until the process exits.
+constexpr int kPoolDevices = 64;
+struct HostCopySet {
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    cudaEvent_t ev[2 * kHostMaxSlices] = {};
+};
+std::mutex g_pool_mutex;
+std::vector<HostCopySet*> g_pool[kPoolDevices];
+
+void destroy_copy_set(HostCopySet* c) {
+    for (cudaEvent_t e : c->ev)
+        if (e) cudaEventDestroy(e);
+    if (c->s_in) cudaStreamDestroy(c->s_in);
+    if (c->s_out) cudaStreamDestroy(c->s_out);
+    delete c;
+}
+
+// A copy set for device `dev` (the current one), or nullptr with the failing call's status in *st.
+HostCopySet* take_copy_set(int dev, ssd_status_t* st) {
+    {
+        std::lock_guard<std::mutex> lock(g_pool_mutex);
+        if (!g_pool[dev].empty()) {
+            HostCopySet* c = g_pool[dev].back();
+            g_pool[dev].pop_back();
+            return c;
+        }
+    }
+    HostCopySet* c = new HostCopySet;
+    if ((*st = cuda_status("stream create", cudaStreamCreateWithFlags(&c->s_in, cudaStreamNonBlocking))) != SSD_OK ||
+        (*st = cuda_status("stream create", cudaStreamCreateWithFlags(&c->s_out, cudaStreamNonBlocking))) != SSD_OK) {
+        destroy_copy_set(c);
+        return nullptr;
+    }
+    for (cudaEvent_t& e : c->ev)
+        if ((*st = cuda_status("event create", cudaEventCreateWithFlags(&e, cudaEventDisableTiming))) != SSD_OK) {
+            destroy_copy_set(c);
+            return nullptr;
+        }
+    return c;
+}
+
+void return_copy_set(int dev, HostCopySet* c) {
+    std::lock_guard<std::mutex> lock(g_pool_mutex);
+    g_pool[dev].push_back(c);
+}
+
+
+// Packed documents: workspace [ticket, error, malformed-offsets flag, pad | order[ndoc]]
+// on the single-pass kernel; [status words | one document's ssd_fwd workspace] for
+// the shapes it does not take, which run document by document (step paths, whose
+// workspace grows with the sequence, so the whole pack's bounds every document's).
+constexpr size_t kVarlenSyncBytes = 256;
+size_t varlen_workspace(const ssd::Dims& d, int64_t ndoc) {
+    if (fused_ok(d)) return kVarlenSyncBytes + align_up((size_t)ndoc * 4, 256);
+    return kVarlenSyncBytes + align_up(fwd_workspace(d).total, 256);
+}
+
+ssd_status_t check_varlen_shape(const ssd_shape_t* shape, int64_t ndoc) {
+    ssd_status_t st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    if (shape->batch != 1 || ndoc < 0 || (ndoc == 0 && shape->seqlen != 0)) return SSD_ERR_INVALID_ARG;
+    if (ndoc > 1 << 24) return SSD_ERR_UNSUPPORTED;
+    const ssd::Dims d = ssd::make_dims(*shape);
+    if ((double)ndoc * (double)d.H > 1.0e9) return SSD_ERR_UNSUPPORTED;
+    return SSD_OK;
+}
+
+// Packed documents on shapes the single-pass kernel does not take: the offsets are
+// read back (the call waits for `s`), checked, and each document runs as its own
+// forward on its slice of the pack, one after another on `s`.
+ssd_status_t varlen_by_document(const ssd::Dims& d, const void* x, const float* dt, const float* A,
+                                const void* B, const void* C, const float* D, const int32_t* cu,
+                                int64_t ndoc, const float* init, void* y, float* final_states,
+                                char* ws, cudaStream_t s) {
+    std::vector<int32_t> h((size_t)ndoc + 1);
+    ssd_status_t st;
+    if ((st = cuda_status("cu_seqlens read", cudaMemcpyAsync(h.data(), cu, h.size() * 4, cudaMemcpyDeviceToHost,
+                                                             s))) != SSD_OK ||
+        (st = cuda_status("stream synchronize", cudaStreamSynchronize(s))) != SSD_OK)
+        return st;
+    if (h[0] != 0 || h[(size_t)ndoc] != d.T) goto bad;
+    for (int64_t k = 0; k < ndoc; ++k)
+        if (h[k + 1] < h[k]) goto bad;
+    {
+        const size_t es = elem_size(d.dtype);
+        const size_t PN = (size_t)(d.H * d.P * d.N);
+        for (int64_t k = 0; k < ndoc; ++k) {
+            const int64_t a = h[k], len = h[k + 1] - h[k];
+            ssd::Dims dk = d;
+            dk.T = len;
+            dk.nc = (len + d.Q - 1) / d.Q;
+            const char* xk = (const char*)x + (size_t)(a * d.H * d.P) * es;
+            const char* bk = (const char*)B + (size_t)(a * d.G * d.N) * es;
+            const char* ck = (const char*)C + (size_t)(a * d.G * d.N) * es;
+            char* yk = (char*)y + (size_t)(a * d.H * d.P) * es;
+            if (len > 0 && (!aligned(xk, 16) || !aligned(bk, 16) || !aligned(ck, 16))) {
+                ssd::set_error_detail("ssd_fwd_varlen: a document's slice of x, B or C does not start on "
+                                      "16 bytes (H*P and G*N elements per token must allow it)");
+                return SSD_ERR_INVALID_ARG;
+            }
+            if ((st = run_fwd(dk, xk, dt + a * d.H, A, bk, ck, D, init ? init + k * PN : nullptr, yk,
+                              final_states ? final_states + k * PN : nullptr, ws, s)) != SSD_OK)
+                return st;
+        }
+    }
+    return SSD_OK;
+bad:
+    ssd::set_error_detail("ssd_fwd_varlen: cu_seqlens is not a non-decreasing list from 0 to seqlen");
+    return SSD_ERR_INVALID_ARG;
 }
 
 }  // namespace
@@ -484,27 +613,24 @@ ssd_status_t ssd_fwd_host(const ssd_shape_t* shape, const void* x, const float* 
     if (d.b == 0) return SSD_OK;
     // bytes of one batch row of each batch-major tensor
     const size_t rx = z.x / d.b, rdt = z.dt / d.b, rbc = z.bc / d.b, rst = z.st / d.b;
-    cudaStream_t s_in = nullptr, s_out = nullptr;
-    cudaEvent_t ev[2 * 8] = {};
-    auto cleanup = [&]() {
-        for (cudaEvent_t e : ev)
-            if (e) cudaEventDestroy(e);
-        if (s_in) cudaStreamDestroy(s_in);
-        if (s_out) cudaStreamDestroy(s_out);
-    };
+    int dev = -1;
+    if ((st = cuda_status("current device", cudaGetDevice(&dev))) != SSD_OK) return st;
+    if (dev < 0 || dev >= kPoolDevices) {
+        ssd::set_error_detail("ssd_fwd_host: device ordinal beyond the copy-stream pool");
+        return SSD_ERR_UNSUPPORTED;
+    }
+    HostCopySet* cs = take_copy_set(dev, &st);
+    if (!cs) return st;
+    cudaStream_t s_in = cs->s_in, s_out = cs->s_out;
+    cudaEvent_t* ev = cs->ev;
+    // every way out waits for the call's copies and kernels, then returns the set
     auto fail = [&](ssd_status_t r) {
         cudaStreamSynchronize(s);
-        if (s_in) cudaStreamSynchronize(s_in);
-        if (s_out) cudaStreamSynchronize(s_out);
-        cleanup();
+        cudaStreamSynchronize(s_in);
+        cudaStreamSynchronize(s_out);
+        return_copy_set(dev, cs);
         return r;
     };
-    if ((st = cuda_status("stream create", cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking))) != SSD_OK ||
-        (st = cuda_status("stream create", cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking))) != SSD_OK)
-        return fail(st);
-    for (int64_t k = 0; k < 2 * hp.nslices; ++k)
-        if ((st = cuda_status("event create", cudaEventCreateWithFlags(&ev[k], cudaEventDisableTiming))) != SSD_OK)
-            return fail(st);
     // s_in starts after whatever the caller queued on `stream` before this call
     if ((st = cuda_status("event record", cudaEventRecord(ev[0], s))) != SSD_OK ||
         (st = cuda_status("stream wait", cudaStreamWaitEvent(s_in, ev[0], 0))) != SSD_OK)
@@ -548,7 +674,7 @@ ssd_status_t ssd_fwd_host(const ssd_shape_t* shape, const void* x, const float* 
     if ((st = cuda_status("stream synchronize", cudaStreamSynchronize(s_out))) != SSD_OK ||
         (st = cuda_status("stream synchronize", cudaStreamSynchronize(s))) != SSD_OK)
         return fail(st);
-    cleanup();
+    return_copy_set(dev, cs);
     // every slice's fused kernel reports through its own status word
     for (int64_t k = 0; k < hp.nslices; ++k) {
         ssd::Dims ds = d;
@@ -566,6 +692,113 @@ ssd_status_t ssd_fwd_check(const ssd_shape_t* shape, const void* workspace, size
     const FwdWorkspace w = fwd_workspace(d);
     if (workspace_bytes < w.total || (w.total > 0 && !workspace)) return SSD_ERR_INVALID_ARG;
     return read_device_status(d, workspace, (cudaStream_t)stream);
+}
+
+ssd_status_t ssd_fwd_varlen_workspace_size(const ssd_shape_t* shape, int64_t n_docs, size_t* bytes) {
+    if (!bytes) return SSD_ERR_INVALID_ARG;
+    ssd_status_t st = check_varlen_shape(shape, n_docs);
+    if (st != SSD_OK) return st;
+    *bytes = n_docs > 0 ? varlen_workspace(ssd::make_dims(*shape), n_docs) : 0;
+    return SSD_OK;
+}
+
+ssd_status_t ssd_fwd_varlen(const ssd_shape_t* shape, const void* x, const float* dt, const float* A,
+                            const void* B, const void* C, const float* D, const int32_t* cu_seqlens,
+                            int64_t n_docs, const float* initial_states, void* y, float* final_states,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+    ssd_status_t st = check_varlen_shape(shape, n_docs);
+    if (st != SSD_OK) return st;
+    if (n_docs == 0) return SSD_OK;
+    const ssd::Dims d = ssd::make_dims(*shape);
+    const Sizes z = sizes_of(d);
+    const size_t zst = (size_t)(n_docs * d.H * d.P * d.N) * 4;    // [n_docs,H,P,N] states
+    const size_t need = varlen_workspace(d, n_docs);
+    if ((!x && z.x) || (!dt && z.dt) || !A || (!B && z.bc) || (!C && z.bc) || (!y && z.x) || !cu_seqlens ||
+        !workspace)
+        return SSD_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(y, 16) || !aligned(workspace, 16))
+        return SSD_ERR_INVALID_ARG;
+    if (!aligned(dt, 4) || !aligned(A, 4) || (D && !aligned(D, 4)) || !aligned(cu_seqlens, 4))
+        return SSD_ERR_INVALID_ARG;
+    if ((initial_states && !aligned(initial_states, 16)) || (final_states && !aligned(final_states, 16)))
+        return SSD_ERR_INVALID_ARG;
+    if (workspace_bytes < need) return SSD_ERR_INVALID_ARG;
+    const Range ins[] = {{x, z.x}, {dt, z.dt}, {A, z.hv}, {B, z.bc}, {C, z.bc}, {D, D ? z.hv : 0},
+                         {initial_states, initial_states ? zst : 0}, {cu_seqlens, (size_t)(n_docs + 1) * 4}};
+    const Range outs[] = {{y, z.x}, {final_states, final_states ? zst : 0}, {workspace, need}};
+    for (const Range& o : outs)
+        for (const Range& i : ins)
+            if (overlaps(o, i)) return SSD_ERR_INVALID_ARG;
+    for (int i = 0; i < 3; ++i)
+        for (int j = i + 1; j < 3; ++j)
+            if (overlaps(outs[i], outs[j])) return SSD_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    char* ws = (char*)workspace;
+    int* sync = (int*)ws;
+    int* order = (int*)(ws + kVarlenSyncBytes);
+    if ((st = cuda_status("sync area", cudaMemsetAsync(sync, 0, 16, s))) != SSD_OK) return st;
+    if (!fused_ok(d))
+        return varlen_by_document(d, x, dt, A, B, C, D, cu_seqlens, n_docs, initial_states, y, final_states,
+                                  ws + kVarlenSyncBytes, s);
+    if ((st = cuda_status("document order", ssd::launch_varlen_order(cu_seqlens, (int)n_docs, d.T, order,
+                                                                      sync + 2, s))) != SSD_OK)
+        return st;
+    if (d.T == 0) {   // every document is empty: final states are the initial ones
+        ssd::Dims dd = d;
+        dd.b = n_docs;
+        return cuda_status("final states", ssd::launch_copy_or_zero_states(dd, initial_states, final_states, s));
+    }
+    CUtensorMap maps[4];
+    if (!ssd::make_tc_maps(d, x, B, C, y, maps)) {
+        ssd::set_error_detail("tensor map encoding failed");
+        return SSD_ERR_CUDA;
+    }
+    ssd::FusedLaunch a = {};
+    a.d = d;
+    a.maps = maps;
+    a.dt = dt;
+    a.A = A;
+    a.D = D;
+    a.init = initial_states;
+    a.finalbuf = final_states;
+    a.segbuf = nullptr;
+    a.sync_ints = sync;
+    a.kheads = ssd::fused_kheads(d.H, d.G, ssd::fused_state_capacity(d.N));
+    a.seg_tiles = 1;
+    a.nseg = 1;
+    a.chained = 0;
+    a.stall = 0;
+    a.y = y;
+    a.cu = cu_seqlens;
+    a.order = order;
+    a.ndoc = (int)n_docs;
+    return cuda_status("fused forward (packed documents)", ssd::launch_fused(a, s));
+}
+
+ssd_status_t ssd_fwd_varlen_check(const ssd_shape_t* shape, int64_t n_docs, const void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+    ssd_status_t st = check_varlen_shape(shape, n_docs);
+    if (st != SSD_OK) return st;
+    if (n_docs == 0) return SSD_OK;
+    if (!workspace || workspace_bytes < varlen_workspace(ssd::make_dims(*shape), n_docs))
+        return SSD_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    int words[3] = {0, 0, 0};
+    if ((st = cuda_status("status read", cudaMemcpyAsync(words, workspace, sizeof(words),
+                                                         cudaMemcpyDeviceToHost, s))) != SSD_OK)
+        return st;
+    if ((st = cuda_status("stream synchronize", cudaStreamSynchronize(s))) != SSD_OK) return st;
+    if (words[2] != 0) {
+        ssd::set_error_detail("ssd_fwd_varlen: cu_seqlens is not a non-decreasing list from 0 to seqlen "
+                              "(offsets were clamped into the row; outputs are not meaningful)");
+        return SSD_ERR_INVALID_ARG;
+    }
+    if (words[1] != 0) {
+        ssd::set_error_detail(words[1] == 3 ? "fused kernel: an mbarrier wait between warp roles timed out"
+                                            : "fused kernel: device error");
+        return SSD_ERR_TIMEOUT;
+    }
+    return SSD_OK;
 }
 
 ssd_status_t ssd_step(const ssd_shape_t* shape, const void* x, const float* dt, const float* A,

@@ -126,6 +126,9 @@ struct Params {
     int* ticket;
     int* error;
     int* flags;           // [b*nseg*nhb] state entering the segment written (chained)
+    void* y;              // [b,T,H,P] bf16, for rows a tile store must not cover
+    const int* cu;        // packed documents: token offsets [ndoc+1] in batch row 0, or null
+    const int* order;     // packed documents: unit order (documents, longest first)
     int64_t T;
     int H, G, N, kheads, batch, nunits, ntiles, seg_tiles, nseg;
     int chained;          // entering states come from the previous segment's unit
@@ -255,14 +258,34 @@ __device__ __forceinline__ bool wait_bar_all(uint64_t* bar, uint32_t parity, Bar
 struct Unit {
     int s, b, hb;          // segment, batch row, head block (pair)
     int t_begin, t_end;    // its tiles
+    int doc;               // sequence index of the initial / final states (batch row, or document)
+    int tok0, len;         // the sequence's first token in its row, its length in tokens
 };
 __device__ __forceinline__ Unit decode(const Params& p, int u) {
     const int nhb = p.H / p.kheads;
     Unit r;
     r.hb = u % nhb;
     int q = u / nhb;
+    if (p.cu) {
+        // packed documents: one unit per (document, head block), the whole document;
+        // offsets are clamped to the row, so a malformed list reads and writes only
+        // inside it (the ordering kernel reports it)
+        r.doc = __ldg(p.order + q);
+        const int a = min(max(__ldg(p.cu + r.doc), 0), (int)p.T);
+        const int e = min(max(__ldg(p.cu + r.doc + 1), a), (int)p.T);
+        r.b = 0;
+        r.s = 0;
+        r.tok0 = a;
+        r.len = e - a;
+        r.t_begin = 0;
+        r.t_end = (r.len + kTile - 1) / kTile;
+        return r;
+    }
     r.b = q % p.batch;
     r.s = q / p.batch;
+    r.doc = r.b;
+    r.tok0 = 0;
+    r.len = (int)p.T;
     r.t_begin = r.s * p.seg_tiles;
     r.t_end = min(p.ntiles, r.t_begin + p.seg_tiles);
     return r;
@@ -273,13 +296,13 @@ __device__ __forceinline__ int64_t flag_index(const Params& p, int b, int s, int
 // state entering the unit for head h (null: zeros)
 __device__ __forceinline__ const float* entry_src(const Params& p, const Unit& U, int h) {
     const int64_t PN = (int64_t)kP * p.N;
-    if (U.s == 0) return p.init ? p.init + ((int64_t)U.b * p.H + h) * PN : nullptr;
+    if (U.s == 0) return p.init ? p.init + ((int64_t)U.doc * p.H + h) * PN : nullptr;
     return p.segbuf + (((int64_t)U.b * p.nseg + U.s) * p.H + h) * PN;
 }
 // where the state leaving the unit goes for head h (null: nowhere)
 __device__ __forceinline__ float* exit_dst(const Params& p, const Unit& U, int h) {
     const int64_t PN = (int64_t)kP * p.N;
-    if (U.s == p.nseg - 1) return p.finalbuf ? p.finalbuf + ((int64_t)U.b * p.H + h) * PN : nullptr;
+    if (U.s == p.nseg - 1) return p.finalbuf ? p.finalbuf + ((int64_t)U.doc * p.H + h) * PN : nullptr;
     if (!p.chained) return nullptr;
     return p.segbuf + (((int64_t)U.b * p.nseg + U.s + 1) * p.H + h) * PN;
 }
@@ -416,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive_expect_tx(&bs->x_full[xs], np * kAtom);
                     for (int e = 0; e < np; ++e)
                         tma_load_4d(smem + K::kOffX + xs * K::kXBytes + e * kAtom, &tm_x, &bs->x_full[xs], 0,
-                                    U.hb * np + e, t * kTile, U.b);
+                                    U.hb * np + e, U.tok0 + t * kTile, U.b);
                 }
             }
         xdrain:
@@ -444,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mbar_arrive_expect_tx(&bs->tb_full[tb], natoms * kAtom);
                         for (int a = 0; a < natoms; ++a)
                             tma_load_4d(smem + K::kOffBC + tb * K::kBCTile + a * kAtom, bc ? &tm_C : &tm_B,
-                                        &bs->tb_full[tb], a * 64, g, t * kTile, U.b);
+                                        &bs->tb_full[tb], a * 64, g, U.tok0 + t * kTile, U.b);
                     }
                 }
             }
@@ -598,15 +621,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             for (int t = U.t_begin; t < U.t_end; ++t) {
                 const int64_t t0 = (int64_t)t * kTile;
-                const int len = (int)min((int64_t)kTile, T - t0);
+                // tokens past the sequence's end get dt = 0: they neither move the
+                // state nor reach a stored row
+                const int len = (int)min((int64_t)kTile, (int64_t)U.len - t0);
+                const float* dtr = prm.dt + ((int64_t)U.b * T + U.tok0 + t0) * H + U.hb * np;
                 float dtv[2][4];
 #pragma unroll
                 for (int e = 0; e < 2; ++e)
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         const int tt = lane * 4 + q;
-                        dtv[e][q] = (e < np && tt < len) ? __ldg(prm.dt + ((int64_t)U.b * T + t0 + tt) * H + U.hb * np + e)
-                                                         : 0.f;
+                        dtv[e][q] = (e < np && tt < len) ? __ldg(dtr + (int64_t)tt * H + e) : 0.f;
                     }
                 float worst = 0.f;
 #pragma unroll
@@ -863,6 +888,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int N = prm.N;
         const int nv = np * K::kMH;
         float hv[V][32];
+        auto load_entry = [&](const Unit& U) {
+#pragma unroll
+            for (int v = 0; v < V; ++v) {
+                const int e = v / K::kMH, mh = v % K::kMH;
+                const int n = r + 128 * mh;
+                const float* src = v < nv ? entry_src(prm, U, U.hb * np + e) : nullptr;
+                if (src && n < N) {
+                    const float* s0 = src + (int64_t)(32 * ph) * N + n;
+#pragma unroll
+                    for (int p2 = 0; p2 < 32; ++p2) hv[v][p2] = __ldcg(s0 + (int64_t)p2 * N);
+                } else {
+#pragma unroll
+                    for (int p2 = 0; p2 < 32; ++p2) hv[v][p2] = 0.f;
+                }
+            }
+        };
         int m = 0, i = 0;
         for (;; ++m) {
             const int ur = m % kURing;
@@ -871,29 +912,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&bs->u_empty[ur]);
             if (u < 0) break;
             const Unit U = decode(prm, u);
+            // an empty document has no tiles: its final state is its initial state
+            if (U.t_begin == U.t_end) load_entry(U);
             for (int t = U.t_begin; t < U.t_end; ++t, ++i) {
                 const int ys = i % kYSlots;
                 if (!wait_bar_all(&bs->yi_full[ys], (i / kYSlots) & 1, bs, err)) goto done;
                 const float* yi = reinterpret_cast<const float*>(smem + K::kOffYInfo + ys * kYInfoBytes);
                 const bool shared = yi[kYiMode] != 0.f;
-                if (t == U.t_begin) {
-                    // the state entering the unit (its flag was acquired before the tile's
-                    // Y'' info was published)
-#pragma unroll
-                    for (int v = 0; v < V; ++v) {
-                        const int e = v / K::kMH, mh = v % K::kMH;
-                        const int n = r + 128 * mh;
-                        const float* src = v < nv ? entry_src(prm, U, U.hb * np + e) : nullptr;
-                        if (src && n < N) {
-                            const float* s0 = src + (int64_t)(32 * ph) * N + n;
-#pragma unroll
-                            for (int p2 = 0; p2 < 32; ++p2) hv[v][p2] = __ldcg(s0 + (int64_t)p2 * N);
-                        } else {
-#pragma unroll
-                            for (int p2 = 0; p2 < 32; ++p2) hv[v][p2] = 0.f;
-                        }
-                    }
-                }
+                // the state entering the unit (its flag was acquired before the tile's
+                // Y'' info was published)
+                if (t == U.t_begin) load_entry(U);
                 if (!wait_bar_all(&bs->h_free, (i & 1) ^ 1, bs, err)) goto done;
                 if (!wait_bar_all(&bs->s_full, i & 1, bs, err)) goto done;
                 tc_fence_after();
@@ -990,11 +1018,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                             *reinterpret_cast<uint4*>(stg + swz(r, 2 * pc + cc)) = make_uint4(o[0], o[1], o[2], o[3]);
                         }
                     }
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0 && t0 + 32 * q < T) {   // rows past T are clipped by the store
-                        tma_store_4d(&tm_y, stg + q * (kAtom / 4), 0, U.hb * np + e, (int)(t0 + 32 * q), U.b);
-                        bulk_commit_group();
+                    const int64_t row0 = t0 + 32 * q;   // the warp's first row in the sequence
+                    if (row0 + 32 <= U.len) {
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_4d(&tm_y, stg + q * (kAtom / 4), 0, U.hb * np + e, (int)(U.tok0 + row0), U.b);
+                            bulk_commit_group();
+                        }
+                    } else if (t0 + r < U.len) {
+                        // the sequence ends inside the warp's rows: the rows after it belong to
+                        // the next document (or lie past the row), so each thread stores its own
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(prm.y) +
+                            (((int64_t)U.b * T + U.tok0 + t0 + r) * H + U.hb * np + e) * kP);
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) dst[c] = *reinterpret_cast<const uint4*>(stg + swz(r, c));
                     }
                 }
                 tc_fence_before();
@@ -1045,6 +1083,43 @@ int fused_kheads(int64_t H, int64_t G, int ns) {
 
 size_t fused_sync_ints(const Dims& d, int nseg) { return 2 + (size_t)(d.b * nseg * d.H); }
 
+namespace {
+constexpr int kVarlenSortMax = 8192;
+
+// One thread per document: its rank among the documents ordered by decreasing
+// length (ties: lower index first) places it in `order`, so that the longest
+// documents' units are taken first and the last wave holds short ones.
+__global__ void varlen_order_kernel(const int* __restrict__ cu, int ndoc, int64_t T, int sort,
+                                    int* __restrict__ order, int* __restrict__ bad) {
+    const int k = blockIdx.x * blockDim.x + threadIdx.x;
+    if (k >= ndoc) return;
+    const int a = cu[k], e = cu[k + 1];
+    if (a > e || a < 0 || (int64_t)e > T || (k == 0 && a != 0) || (k == ndoc - 1 && (int64_t)e != T))
+        atomicExch(bad, 1);
+    if (!sort) {
+        order[k] = k;
+        return;
+    }
+    const int len = e - a;
+    int rank = 0;
+    for (int j = 0; j < ndoc; ++j) {
+        const int lj = __ldg(cu + j + 1) - __ldg(cu + j);
+        rank += (lj > len) || (lj == len && j < k);
+    }
+    order[rank] = k;
+}
+}  // namespace
+
+int varlen_sort_max() { return kVarlenSortMax; }
+
+cudaError_t launch_varlen_order(const int* cu, int ndoc, int64_t T, int* order, int* bad,
+                                cudaStream_t st) {
+    if (ndoc <= 0) return cudaSuccess;
+    varlen_order_kernel<<<(ndoc + 255) / 256, 256, 0, st>>>(cu, ndoc, T, ndoc <= kVarlenSortMax ? 1 : 0,
+                                                            order, bad);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_fused(const FusedLaunch& a, cudaStream_t st) {
     const Dims& d = a.d;
     const int ns = fused_state_capacity(d.N);
@@ -1061,15 +1136,23 @@ cudaError_t launch_fused(const FusedLaunch& a, cudaStream_t st) {
     prm.ticket = a.sync_ints;
     prm.error = a.sync_ints + 1;
     prm.flags = a.sync_ints + 2;
+    prm.y = a.y;
+    prm.cu = a.cu;
+    prm.order = a.order;
     prm.T = d.T;
     prm.H = (int)d.H;
     prm.G = (int)d.G;
     prm.N = (int)d.N;
     prm.kheads = a.kheads;
     prm.batch = (int)d.b;
-    const int64_t ntiles = (d.T + kTile - 1) / kTile;
-    const int64_t nunits = (int64_t)a.nseg * d.b * (d.H / a.kheads);
-    if (nunits > INT32_MAX / 2 || d.T > INT32_MAX || (int64_t)a.seg_tiles * a.nseg < ntiles)
+    const bool packed = a.cu != nullptr;
+    if (!a.y || (packed && (!a.order || a.ndoc < 1 || d.b != 1 || a.nseg != 1 || a.chained)))
+        return cudaErrorInvalidValue;
+    // packed documents: every document's tiles start at tile 0, and at most all T
+    // tokens form one document
+    const int64_t ntiles = (d.T + kTile - 1) / kTile + (packed ? 1 : 0);
+    const int64_t nunits = (packed ? (int64_t)a.ndoc : (int64_t)a.nseg * d.b) * (d.H / a.kheads);
+    if (nunits > INT32_MAX / 2 || d.T > INT32_MAX / 2 || (!packed && (int64_t)a.seg_tiles * a.nseg < ntiles))
         return cudaErrorInvalidValue;
     prm.nunits = (int)nunits;
     prm.ntiles = (int)ntiles;

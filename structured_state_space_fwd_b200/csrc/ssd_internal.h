@@ -67,8 +67,21 @@ struct FusedLaunch {
     int kheads, seg_tiles, nseg;
     int chained;               // segment s > 0 takes its entering state from segment s - 1's unit
     int stall;                 // test builds: make chain waits run out
+    void* y;                   // [b,T,H,P] bf16 (the map's tensor): rows of partial tiles
+    // packed documents (d.b == 1, nseg == 1): document k is tokens cu[k] .. cu[k+1]-1;
+    // init / finalbuf are [ndoc,H,P,N]; units run in `order` (varlen_order output)
+    const int* cu;
+    const int* order;
+    int ndoc;
 };
 cudaError_t launch_fused(const FusedLaunch& a, cudaStream_t st);
+
+// Packed documents: order[ndoc] = documents by decreasing length (ties by index;
+// identity order above varlen_sort_max() documents), and *bad = 1 when cu is not a
+// non-decreasing list from 0 to T.
+int varlen_sort_max();
+cudaError_t launch_varlen_order(const int* cu, int ndoc, int64_t T, int* order, int* bad,
+                                cudaStream_t st);
 
 // Segment states (ssd_segment.cu): for each segment s < nseg_out of seg_tiles tiles,
 // the state it reaches from zero, written to segbuf slot s + 1 ([b,nslot,H,P,N]), and

@@ -12,7 +12,6 @@
 #include <cuda_runtime.h>
 
 #include <cstdio>
-#include <mutex>
 
 #include "ssd.h"
 #include "ssd_internal.h"
@@ -20,42 +19,27 @@
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;  // 64 MiB
-constexpr int kMaxDevices = 64;
 
 // Device-side scratch shared by every ssd_fwd_no_alloc call on a device. In
 // host code this name is only a stand-in for the symbol, never an address a
 // kernel may be given: the device address comes from cudaGetSymbolAddress.
 static __device__ __align__(256) unsigned char g_ssd_scratch[kNoAllocScratchBytes];
 
-std::mutex g_setup_mutex;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Once per device, with that device current: look up the device address of
-// the scratch array. Returns nullptr (and a detail message) on failure.
+// The device address of the scratch array on the current device, looked up on
+// every call (a host-side symbol lookup, nothing enqueued), so that it follows
+// the current device and a context recreated after cudaDeviceReset. Returns
+// nullptr (and a detail message) on failure.
 void* scratch_for_current_device() {
-    int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_ssd_scratch);
+    if (e != cudaSuccess || !p) {
         char msg[160];
-        snprintf(msg, sizeof(msg), "ssd_fwd_no_alloc: no usable current device (%s)",
+        snprintf(msg, sizeof(msg), "ssd_fwd_no_alloc: cudaGetSymbolAddress failed: %s",
                  cudaGetErrorString(e));
         ssd::set_error_detail(msg);
         return nullptr;
     }
-    std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (!g_scratch_ptr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_ssd_scratch);
-        if (e != cudaSuccess || !p) {
-            char msg[160];
-            snprintf(msg, sizeof(msg), "ssd_fwd_no_alloc: cudaGetSymbolAddress failed: %s",
-                     cudaGetErrorString(e));
-            ssd::set_error_detail(msg);
-            return nullptr;
-        }
-        g_scratch_ptr[dev] = p;
-    }
-    return g_scratch_ptr[dev];
+    return p;
 }
 
 }  // namespace

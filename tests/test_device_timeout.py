@@ -26,12 +26,15 @@ import structured_state_space_fwd_b200 as ssd
 from structured_state_space_fwd_b200._lib import SSD_ERR_TIMEOUT, SSDError
 
 assert ssd.lib_path.endswith("libssd_testhooks.so"), ssd.lib_path
-# two 128-token tiles per sequence, so every sequence has one hand-off
-inp = make_inputs(batch=2, seqlen=256, nheads=8, headdim=64, ngroups=2, dstate=128,
+# 160 chains (head pairs of one batch row), more than the GPU has SMs, so the
+# two-tile sequence is split into two segments with one hand-off between them
+inp = make_inputs(batch=1, seqlen=256, nheads=320, headdim=64, ngroups=1, dstate=128,
                   dtype="bf16", initial_states=True, seed=5)
 d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
 shape = ssd.make_shape(d["x"], d["B"], 256)
 assert ssd.ssd_fwd_plan(shape)[0] == "fused"
+# the workspace holds a segment-state buffer only when a sequence has several segments
+assert ssd.ssd_fwd_workspace_size(shape) >= 2 * 320 * 64 * 128 * 4
 ws = torch.empty(ssd.ssd_fwd_workspace_size(shape), dtype=torch.uint8, device="cuda")
 
 os.environ["SSD_TEST_STALL_CHAIN"] = "1"

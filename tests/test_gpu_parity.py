@@ -299,6 +299,19 @@ def test_segmented_several_tiles_per_segment(ssd, path_env):
     check_full(ssd, inp, 256, "bf16")
 
 
+@pytest.mark.parametrize("N,T", [(128, 128 * 9 - 5), (64, 128 * 5 + 3), (256, 128 * 6)])
+def test_chained_segments(ssd, path_env, N, T):
+    # more chains than SMs, so each sequence is split into segments of a few
+    # tiles whose states hand off through the segment buffer and its flags
+    path_env(None)
+    inp = make_inputs(batch=2, seqlen=T, nheads=160, headdim=64, ngroups=1, dstate=N,
+                      dtype="bf16", initial_states=True, seed=909 + N)
+    shp = ssd.make_shape(inp["x"], inp["B"], 256)
+    assert ssd.ssd_fwd_plan(shp)[0] == "fused"
+    assert ssd.ssd_fwd_workspace_size(shp) >= 2 * 2 * 160 * 64 * N * 4  # segment states present
+    check_full(ssd, inp, 256, "bf16")
+
+
 def test_tensor_steps_against_oracle(ssd, path_env):
     path_env("steps")
     Q = 256
