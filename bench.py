@@ -41,7 +41,11 @@ UNIT = "Mtokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant kernel, from
 # one ncu capture of this workload (profiles/); None until captured for the current kernel
-TRAFFIC = {"fused": 326415872}
+TRAFFIC = {"fused": 368611328}
+KERNEL_NAMES = {"fused": "ssd_fused_kernel",
+                "segmented": "segment_state_kernel + segment_scan_kernel + ssd_fused_kernel",
+                "steps": "chunk_cumsum + chunk_state_tc + state_passing + chunk_scan_tc",
+                "simt": "chunk_cumsum + chunk_state + state_passing + chunk_scan"}
 
 
 # ------------------------------------------------------------------ counts
@@ -174,6 +178,89 @@ def oracle_sample(w: W.Workload, budget_s: float, inputs64=None):
     desc = (f"batch row 0, heads 0..{nh2 - 1} of {w.nheads} (T={w.seqlen}); "
             f"{nh2 * w.seqlen} token-heads = {tokens_equiv:.0f} token-equivalents per run")
     return run, tokens_equiv, desc, threads
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def oracle_single_thread(w: W.Workload, inp, budget_s: float = 3.0):
+    """The oracle's recurrence on one thread (one head of batch row 0, repeated for
+    about budget_s), in the bench unit: what one host core sustains."""
+    import oracle
+    x = np.ascontiguousarray(inp["x"][:1, :, :1].double().numpy())
+    dt = np.ascontiguousarray(inp["dt"][:1, :, :1].double().numpy())
+    A = np.ascontiguousarray(inp["A"][:1].double().numpy())
+    B = inp["B"][:1].double().numpy()
+    C = inp["C"][:1].double().numpy()
+    D = np.ascontiguousarray(inp["D"][:1].double().numpy()) if inp["D"] is not None else None
+    reps, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < budget_s:
+        oracle.recurrence(x, dt, A, B, C, D)
+        reps += 1
+    el = time.perf_counter() - t0
+    tok = w.seqlen / w.nheads * reps     # one head of T tokens = T / H token-equivalents
+    return {"value": tok / el / 1e6, "unit": UNIT, "threads": 1,
+            "sample": f"batch row 0, head 0 (T={w.seqlen}), {reps} runs in {el:.1f} s"}
+
+
+# ------------------------------------------------------------------ sweeps
+def measure_workload(ssd, dev, stream, w: W.Workload, steps, warmup, seed=0):
+    """One ssd_fwd step of workload w (final states returned), timed with CUDA events:
+    throughput, path, and the fraction of the HBM roofline the whole step reaches
+    (algorithmic bytes of the step / step time)."""
+    inp = W.workload_inputs(w, seed=seed)
+    d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+    shp = ssd.make_shape(d["x"], d["B"], w.chunk_size)
+    ws = torch.empty(max(ssd.ssd_fwd_workspace_size(shp), 1), dtype=torch.uint8, device=dev)
+    y = torch.empty_like(d["x"])
+    fin = torch.empty((w.batch, w.nheads, w.headdim, w.dstate), dtype=torch.float32, device=dev)
+
+    def step():
+        ssd.ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], chunk_size=w.chunk_size,
+                    initial_states=d["initial_states"], y=y, final_states=fin,
+                    return_final_states=True, workspace=ws, stream=stream)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ssd.ssd_fwd_check(shp, ws, stream=stream)
+    ms = e0.elapsed_time(e1) / steps
+    path, nk = ssd.ssd_fwd_plan(shp)
+    _, by = alg_counts(w, with_final=True, with_init=w.initial_states)
+    pk, pk_kind = peaks()
+    ach = by / (ms / 1e3) / 1e9
+    return {"workload": w.name, "value": w.tokens / (ms / 1e3) / 1e6, "unit": UNIT, "ms_per_step": ms,
+            "steps": steps, "warmup": warmup, "path": path, "gpu_launches_per_step": nk,
+            "roofline": {"kernel": KERNEL_NAMES[path] + " (whole step)", "bound": "hbm",
+                         "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": ach / pk["hbm_gbs"], "alg_bytes_per_step": by, "traffic": None,
+                         "peak_source": pk_kind}}
+
+
+def measure_sweeps(ssd, dev, stream, seed=0):
+    """The sequence-length sweep (32768 tokens at every T), the state-size sweep and the
+    long-context workload, each as its own row."""
+    rows = {}
+    for w in W.seqlen_sweep():
+        rows[f"seqlen_T{w.seqlen}"] = measure_workload(ssd, dev, stream, w, 20, 3, seed=seed)
+    for w in W.dstate_sweep():
+        rows[f"dstate_N{w.dstate}"] = measure_workload(ssd, dev, stream, w, 20, 3, seed=seed)
+    rows["long_context"] = measure_workload(ssd, dev, stream, W.LONG_CONTEXT, 20, 3, seed=seed)
+    return rows
 
 
 # ------------------------------------------------------------------ reference arm
@@ -605,10 +692,10 @@ def run_ours(args):
 
     # dominant kernel and its average launch duration (CUDA events on its stream)
     if path_name == "fused":
-        # one kernel per step: the fused forward; its launch duration is the
+        # one kernel per step: the single-pass forward; its launch duration is the
         # timed step (which also holds the small counter memset before it)
-        ktimes = {"ssd_fused_ws_kernel": ms_step}
-        dom = ("ssd_fused_ws_kernel", None, by)
+        ktimes = {"ssd_fused_kernel": ms_step}
+        dom = ("ssd_fused_kernel", None, by)
     else:
         plan = kernel_plan(ssd, w, d, bufs, stream)
         ktimes = {}
@@ -662,9 +749,31 @@ def run_ours(args):
         ms_e2e = max_over_ranks(a0.elapsed_time(a1), world, dev) / ke
         h2d = sum(v.numel() * v.element_size() for v in hp.values() if v is not None)
         d2h = hy.numel() * hy.element_size() + hf.numel() * hf.element_size()
+        # the same bytes copied alone (one pinned copy each way), for the copy engines' rate
+        hx = torch.empty(int(h2d), dtype=torch.uint8).pin_memory()
+        dx = torch.empty(int(h2d), dtype=torch.uint8, device=dev)
+        hyb = torch.empty(int(d2h), dtype=torch.uint8).pin_memory()
+        dyb = torch.empty(int(d2h), dtype=torch.uint8, device=dev)
+        for _ in range(2):
+            dx.copy_(hx, non_blocking=True)
+            hyb.copy_(dyb, non_blocking=True)
+        torch.cuda.synchronize()
+        c0, c1, c2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        c0.record(stream)
+        dx.copy_(hx, non_blocking=True)
+        c1.record(stream)
+        hyb.copy_(dyb, non_blocking=True)
+        c2.record(stream)
+        torch.cuda.synchronize()
+        h2d_gbs = h2d / (c0.elapsed_time(c1) / 1e3) / 1e9
+        d2h_gbs = d2h / (c1.elapsed_time(c2) / 1e3) / 1e9
+        del hx, dx, hyb, dyb
         e2e = {"value": w.tokens * world / (ms_e2e / 1e3) / 1e6, "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": ms_e2e, "api": "ssd_fwd_host (pinned host buffers)"}
+               "ms_per_step": ms_e2e, "api": "ssd_fwd_host (pinned host buffers)",
+               "copy_gbs": {"h2d_alone": h2d_gbs, "d2h_alone": d2h_gbs,
+                            "h2d_plus_d2h_over_step": (h2d + d2h) / (ms_e2e / 1e3) / 1e9},
+               "copy_bound_ms": (h2d / h2d_gbs + d2h / d2h_gbs) / 1e6}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.profile:
@@ -679,12 +788,14 @@ def run_ours(args):
             run()
         el = time.perf_counter() - t0
         cpu = {"value": tok * reps / el / 1e6, "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": f"fp64 sequential recurrence, {desc}; {reps} runs in {el:.1f} s"}
+               "sample": f"fp64 sequential recurrence, {desc}; {reps} runs in {el:.1f} s",
+               "cpu_model": cpu_model(), "single_thread": oracle_single_thread(w, inp)}
 
     decode = None
     cp = None
     gate = None
     varlen = None
+    sweeps = None
     if not args.profile:
         # secondary rows, measured after the headline: a failure here is reported in
         # its own entry and does not take the headline line down with it
@@ -702,6 +813,7 @@ def run_ours(args):
         cp = guarded(measure_cp_slice, ssd, dev, stream, 50, 5)
         gate = guarded(measure_gate, ssd, dev, stream, 100, 5, seed=rank)
         varlen = guarded(measure_varlen, ssd, dev, stream, 20, 3, seed=rank)
+        sweeps = guarded(measure_sweeps, ssd, dev, stream, seed=rank)
 
     if rank == 0:
         line = {
@@ -720,6 +832,7 @@ def run_ours(args):
             "e2e": e2e,
             "gpu_launches": kernels_per_step * args.steps,
             "clocks": clk,
+            "workload_rows": sweeps,
             "next_rows": {"decode_step": decode, "context_parallel": cp, "gate_norm": gate,
                           "packed_docs": varlen},
         }

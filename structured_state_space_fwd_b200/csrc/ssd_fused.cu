@@ -145,6 +145,7 @@ struct Bars {
     uint64_t g_full, g_empty_mma, g_empty_mask, p_full;
     uint64_t cs_full[kCsSlots], cs_empty[kCsSlots];
     uint64_t s_full, s_empty;
+    uint64_t s_read;              // unfactored tile: the chain group has read S (its slot takes C h^T next)
     uint64_t y_full[kYSlots], y_empty[kYSlots], yi_full[kYSlots];
     uint64_t h_full, h_free;
     uint64_t pub_full[2], pub_empty[2];   // per unit: leaving state stored / flag released
@@ -386,6 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(&bs->s_full, 1);
         mbar_init(&bs->s_empty, 256);
+        mbar_init(&bs->s_read, 256);
         for (int i = 0; i < kYSlots; ++i) {
             mbar_init(&bs->y_full[i], 1);
             mbar_init(&bs->y_empty[i], 128);
@@ -446,18 +448,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < K::kXSlots && i < n; ++i)
                 mbar_wait(&bs->x_full[(n - 1 - i) % K::kXSlots], ((n - 1 - i) / K::kXSlots) & 1, 1u << 22);
         } else if (lane == 0) {
-            int m = 0, mb = 0;    // units taken, tile buffers loaded
-            for (;; ++m) {
+            int mb = 0;    // tile buffers loaded
+            auto take = [&]() -> int {
                 int u;
                 do {
                     u = atomicAdd(prm.ticket, 1);
                 } while (u < prm.nunits && decode(prm, u).t_begin >= prm.ntiles);
-                if (u >= prm.nunits) u = -1;
+                return u < prm.nunits ? u : -1;
+            };
+            auto publish = [&](int m, int u) -> bool {
                 const int ur = m % kURing;
-                if (!wait_bar_idle(&bs->u_empty[ur], ((m / kURing) & 1) ^ 1, bs, err)) goto pdrain;
+                if (!wait_bar_idle(&bs->u_empty[ur], ((m / kURing) & 1) ^ 1, bs, err)) return false;
                 bs->uid[ur] = u;
                 mbar_arrive(&bs->u_full[ur]);
-                if (u < 0) break;
+                return true;
+            };
+            // Each unit's successor is taken and published before the unit's own tiles
+            // are loaded, so the other roles (the x loader first) run into it without
+            // waiting for this lane. Units are still taken in ticket order and worked in
+            // that order, so a chained unit's predecessor always has a lower ticket that
+            // some CTA is working on or has finished.
+            int u = take();
+            if (!publish(0, u)) goto pdrain;
+            for (int m = 0; u >= 0; ++m) {
+                const int un = take();
+                if (!publish(m + 1, un)) goto pdrain;
                 const Unit U = decode(prm, u);
                 const int g = U.hb * np / (H / prm.G);
                 for (int t = U.t_begin; t < U.t_end; ++t) {
@@ -470,6 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                         &bs->tb_full[tb], a * 64, g, U.tok0 + t * kTile, U.b);
                     }
                 }
+                u = un;
             }
         pdrain:
             // No TMA load may still be writing shared memory when the CTA exits: wait for
@@ -479,9 +495,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        // Per tile i: G = C B^T, S_i and the masked product (neither waits for the
-        // state), then the tile's state product C h^T once the chain group has
-        // written its operand (a register update of the carried state).
+        // Per tile i (factored): G = C B^T, S_i, the state term C (2^L h)^T once the
+        // chain group has written its operand from the state entering the tile (ready
+        // a tile ahead: it needs S_{i-1}, not S_i), then the masked product. An
+        // unfactored tile: per-head Y = P x, S_i, and C h^T into the S slot once the
+        // chain group has read S_i.
         if (lane == 0) {
             constexpr uint32_t idG = idesc_bf16(128, 128, 0, 0);   // C (K-major) x B (K-major)
             const uint32_t idS = np == 2 ? idesc_bf16(128, 128, 1, 1) : idesc_bf16(128, 64, 1, 1);
@@ -492,7 +510,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int item, ys, cb;   // cb: tile buffer of the tile's C
                 bool shared;
             };
-            int psh = 0, nsh = 0, gm = 0, gk = 0;
+            int psh = 0, nsh = 0, nrd = 0, gm = 0, gk = 0;
             bool prev_shared = true;
             // C (2^L h)^T onto Y'' (factored) or C h^T into the S slot (unfactored)
             auto issue_r = [&](const Pend& q) -> bool {
@@ -501,7 +519,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint64_t dC = sw128_desc(smem_u32(smem + K::kOffBC + q.cb * K::kBCTile), 16, 1024);
                 const uint32_t d = q.shared ? tmem + kColY + 128 * q.ys : tmem + kColS;
                 mma_state_dim_n<true>(ksN, d, dC, dH, idY, q.shared ? 1u : 0u);
-                mma_commit(&bs->y_full[q.ys]);
                 mma_commit(&bs->h_free);
                 mma_commit(&bs->tb_empty[q.cb]);
                 return true;
@@ -546,12 +563,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int mh = 0; mh < K::kMH; ++mh)
                             mma_tokens_smem(tmem + kColS + 64 * mh, dSA + (uint64_t)((2 * mh * kAtom) >> 4), dX, idS);
                         mma_commit(&bs->s_full);
+                        mma_commit(&bs->tb_empty[tbB]);    // this tile's B has served G and S
+                        // the state term C (2^L h)^T onto Y'': its operand needs only the state
+                        // entering the tile, so it goes ahead of the masked product
+                        if (!issue_r(Pend{i, ys, tbC, true})) goto drain;
                         if (!wait_bar(&bs->p_full, psh & 1, bs, err)) goto drain;
                         ++psh;
                         tc_fence_after();
                         mma_tokens_tmem(tmem + kColY + 128 * ys, tmem + kColP, dX, idY);
                         mma_commit(&bs->x_empty[xs]);
                         mma_commit(&bs->g_empty_mma);
+                        mma_commit(&bs->y_full[ys]);
                     } else {
                         // per head Y = P x with the raw tile (P in the S slot), then S once
                         // the tile is scaled in place
@@ -568,10 +590,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                             mma_tokens_smem(tmem + kColS + 64 * mh, dSA + (uint64_t)((2 * mh * kAtom) >> 4), dX, idS);
                         mma_commit(&bs->s_full);
                         mma_commit(&bs->x_empty[xs]);
+                        mma_commit(&bs->tb_empty[tbB]);    // this tile's B has served G and S
+                        // C h^T goes into the S slot once the chain group has read S
+                        if (!wait_bar(&bs->s_read, nrd & 1, bs, err)) goto drain;
+                        ++nrd;
+                        if (!issue_r(Pend{i, ys, tbC, false})) goto drain;
+                        mma_commit(&bs->y_full[ys]);
                     }
                     prev_shared = shared;
-                    mma_commit(&bs->tb_empty[tbB]);    // this tile's B has served its S
-                    if (!issue_r(Pend{i, ys, tbC, shared})) goto drain;
                 }
             }
         drain:
@@ -922,33 +948,44 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // the state entering the unit (its flag was acquired before the tile's
                 // Y'' info was published)
                 if (t == U.t_begin) load_entry(U);
+                // the operand of the tile's state term, from the state entering the tile:
+                // 2^L h (factored) or h, once the previous tile's product has read it
                 if (!wait_bar_all(&bs->h_free, (i & 1) ^ 1, bs, err)) goto done;
+#pragma unroll
+                for (int v = 0; v < V; ++v) {
+                    if (v >= nv) break;
+                    const float sc = shared ? yi[kYiEL + v / K::kMH] : 1.f;
+                    uint8_t* ha = smem + K::kOffH + v * kAtom;
+#pragma unroll
+                    for (int pc = 0; pc < 4; ++pc) {   // 8 head-dim columns at a time
+                        uint32_t op[4];
+#pragma unroll
+                        for (int e2 = 0; e2 < 4; ++e2)
+                            op[e2] = pack_bf16(sc * hv[v][8 * pc + 2 * e2], sc * hv[v][8 * pc + 2 * e2 + 1]);
+                        *reinterpret_cast<uint4*>(ha + swz(r, 4 * ph + pc)) = make_uint4(op[0], op[1], op[2], op[3]);
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(&bs->h_full);
+                // then the state leaving the tile: h <- 2^L h + S
                 if (!wait_bar_all(&bs->s_full, i & 1, bs, err)) goto done;
                 tc_fence_after();
 #pragma unroll
                 for (int v = 0; v < V; ++v) {
                     if (v >= nv) break;
                     const float eL = yi[kYiEL + v / K::kMH];
-                    const float sc = shared ? eL : 1.f;   // the operand: 2^L h, or h
-                    uint8_t* ha = smem + K::kOffH + v * kAtom;
 #pragma unroll
-                    for (int pc = 0; pc < 4; ++pc) {   // 8 head-dim columns at a time
+                    for (int pc = 0; pc < 4; ++pc) {
                         float sv[8];
                         tmem_ld8(tmem + lb + kColS + 64 * v + 32 * ph + 8 * pc, sv);
                         tmem_ld_wait_regs(sv);
-                        uint32_t op[4];
-#pragma unroll
-                        for (int e2 = 0; e2 < 4; ++e2)
-                            op[e2] = pack_bf16(sc * hv[v][8 * pc + 2 * e2], sc * hv[v][8 * pc + 2 * e2 + 1]);
-                        *reinterpret_cast<uint4*>(ha + swz(r, 4 * ph + pc)) = make_uint4(op[0], op[1], op[2], op[3]);
 #pragma unroll
                         for (int e2 = 0; e2 < 8; ++e2) hv[v][8 * pc + e2] = fmaf(eL, hv[v][8 * pc + e2], sv[e2]);
                     }
                 }
-                fence_proxy_async_smem();
                 tc_fence_before();
-                if (shared) mbar_arrive(&bs->s_empty);
-                mbar_arrive(&bs->h_full);
+                mbar_arrive(shared ? &bs->s_empty : &bs->s_read);
             }
             // the state leaving the unit
             if (!wait_bar_all(&bs->pub_empty[m & 1], ((m >> 1) & 1) ^ 1, bs, err)) goto done;
