@@ -49,7 +49,7 @@ struct SCfg {
     static constexpr uint32_t kOffX = kOffB + kBSlots * kBTile;
     static constexpr uint32_t kOffW = kOffX + kXSlots * kAtom;        // w per x slot
     static constexpr uint32_t kOffTot = kOffW + kXSlots * kTile * 4;  // tile totals [heads][tiles]
-    static constexpr uint32_t kOffBar = kOffTot + kMaxHeads * kMaxSegTiles * 4;
+    static constexpr uint32_t kOffBar = kOffTot + 2 * kMaxHeads * kMaxSegTiles * 4;   // totals, suffix sums
     static constexpr uint32_t kSmem = kOffBar + 1024;
     static_assert(kSmem <= 232448, "shared memory budget");
     static_assert(kMaxHeads * 64 * kMH * kAccBufs <= 512, "tensor memory budget");
@@ -244,44 +244,67 @@ __global__ void __launch_bounds__(kThreads, 1)
         // + (tile total - inclusive sum to i), and the segment's decay 2^E.
         float* tot = reinterpret_cast<float*>(smem + K::kOffTot);
         int nx = 0;
+        // dt of one tile for the unit's heads: lane l holds tokens 4l..4l+3; every load
+        // of a tile is issued before any is used, so a tile costs one memory latency
+        auto load_dt = [&](const SUnit& U, int tt, float (&dv)[kMaxHeads][4]) {
+            const int64_t t0 = (int64_t)(U.t_begin + tt) * kTile + lane * 4;
+#pragma unroll
+            for (int k = 0; k < kMaxHeads; ++k)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    dv[k][e] = (k < kh && t0 + e < T)
+                                   ? __ldg(prm.dt + ((int64_t)U.b * T + t0 + e) * H + U.hb * kh + k)
+                                   : 0.f;
+        };
         for (int u = blockIdx.x; u < prm.nunits; u += gridDim.x) {
             const SUnit U = sdecode(prm, u);
             const int nt = U.t_end - U.t_begin;
-            for (int k = 0; k < kh; ++k) {
-                const int h = U.hb * kh + k;
-                const float a2 = __ldg(prm.A + h) * kLog2e;
-                float E = 0.f;
-                for (int tt = 0; tt < nt; ++tt) {
-                    const int64_t t0 = (int64_t)(U.t_begin + tt) * kTile;
-                    float sdt = 0.f;
+            float a2[kMaxHeads];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int64_t t = t0 + lane * 4 + e;
-                        sdt += t < T ? __ldg(prm.dt + ((int64_t)U.b * T + t) * H + h) : 0.f;
-                    }
+            for (int k = 0; k < kMaxHeads; ++k) a2[k] = k < kh ? __ldg(prm.A + U.hb * kh + k) * kLog2e : 0.f;
+            // tile totals of dt A per head, the next tile's dt loading during this one's sums
+            float dv[kMaxHeads][4], dn[kMaxHeads][4];
+            load_dt(U, 0, dv);
+            for (int tt = 0; tt < nt; ++tt) {
+                if (tt + 1 < nt) load_dt(U, tt + 1, dn);
+#pragma unroll
+                for (int k = 0; k < kMaxHeads; ++k) {
+                    float sdt = dv[k][0] + dv[k][1] + dv[k][2] + dv[k][3];
 #pragma unroll
                     for (int off = 16; off > 0; off >>= 1) sdt += __shfl_xor_sync(0xffffffffu, sdt, off);
-                    if (lane == 0) tot[k * kMaxSegTiles + tt] = sdt * a2;
-                    E += sdt * a2;
+                    if (lane == 0 && k < kh) tot[k * kMaxSegTiles + tt] = sdt * a2[k];
                 }
-                if (lane == 0) prm.decay[((int64_t)U.b * prm.nseg + U.s) * H + h] = ex2(E);
+#pragma unroll
+                for (int k = 0; k < kMaxHeads; ++k)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) dv[k][e] = dn[k][e];
             }
             __syncwarp();
+            // suffix sums over later tiles, in place of the totals' copy kept per head:
+            // lane k walks head k's tiles backwards; the segment's decay 2^E
+            float* later = tot + kMaxHeads * kMaxSegTiles;
+            if (lane < kh) {
+                float acc = 0.f;
+                for (int tt = nt - 1; tt >= 0; --tt) {
+                    later[lane * kMaxSegTiles + tt] = acc;
+                    acc += tot[lane * kMaxSegTiles + tt];
+                }
+                prm.decay[((int64_t)U.b * prm.nseg + U.s) * H + U.hb * kh + lane] = ex2(acc);
+            }
+            __syncwarp();
+            load_dt(U, 0, dv);
             for (int tt = 0; tt < nt; ++tt) {
-                const int64_t t0 = (int64_t)(U.t_begin + tt) * kTile;
-                for (int k = 0; k < kh; ++k, ++nx) {
-                    const int h = U.hb * kh + k;
-                    const float a2 = __ldg(prm.A + h) * kLog2e;
-                    float later = 0.f;   // sum over the segment's tiles after this one
-                    for (int t2 = tt + 1; t2 < nt; ++t2) later += tot[k * kMaxSegTiles + t2];
+                if (tt + 1 < nt) load_dt(U, tt + 1, dn);
+#pragma unroll
+                for (int k = 0; k < kMaxHeads; ++k) {
+                    if (k >= kh) break;
+                    const float lat = later[k * kMaxSegTiles + tt];
                     const int xs = nx % K::kXSlots;
                     if (!swait_all(&bs->w_empty[xs], ((nx / K::kXSlots) & 1) ^ 1, bs, err)) goto done;
-                    float dtv[4], run = 0.f, v[4];
+                    float run = 0.f, v[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int64_t t = t0 + lane * 4 + e;
-                        dtv[e] = t < T ? __ldg(prm.dt + ((int64_t)U.b * T + t) * H + h) : 0.f;
-                        run += dtv[e] * a2;
+                        run += dv[k][e] * a2[k];
                         v[e] = run;
                     }
                     float incl = run;
@@ -294,11 +317,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float ttot = __shfl_sync(0xffffffffu, incl, 31);
                     float* w = reinterpret_cast<float*>(smem + K::kOffW + xs * kTile * 4);
                     reinterpret_cast<float4*>(w)[lane] = make_float4(
-                        ex2(later + ttot - (excl + v[0])) * dtv[0], ex2(later + ttot - (excl + v[1])) * dtv[1],
-                        ex2(later + ttot - (excl + v[2])) * dtv[2], ex2(later + ttot - (excl + v[3])) * dtv[3]);
+                        ex2(lat + ttot - (excl + v[0])) * dv[k][0], ex2(lat + ttot - (excl + v[1])) * dv[k][1],
+                        ex2(lat + ttot - (excl + v[2])) * dv[k][2], ex2(lat + ttot - (excl + v[3])) * dv[k][3]);
                     __syncwarp();
                     mbar_arrive(&bs->w_full[xs]);
+                    ++nx;
                 }
+#pragma unroll
+                for (int k = 0; k < kMaxHeads; ++k)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) dv[k][e] = dn[k][e];
             }
             __syncwarp();
         }
