@@ -454,6 +454,69 @@ def measure_varlen(ssd, dev, stream, steps, warmup, seed=0):
             "gpu_launches": steps * 2}   # document ordering + the single-pass kernel
 
 
+# ------------------------------------------------------------------ forward + gate, fused
+GATED_METRIC = ("SSD fwd + gate + RMSNorm (per-head groups of 64) Mtokens/s at 2.7B layer shape, "
+                "gate fused into the forward's stores")
+
+
+def measure_fwd_gated(ssd, dev, stream, steps, warmup, seed=0):
+    """ssd_fwd_gated at the 2.7B layer shape with norm groups of 64 channels (one head):
+    the single-pass kernel gates and normalises each row before storing it, so y never
+    reaches HBM. Timed beside the same work as two calls (ssd_fwd, then
+    ssd_gated_rmsnorm), which writes y and reads it back."""
+    w = WORKLOAD
+    inp = W.workload_inputs(w, seed=seed)
+    d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+    g = torch.Generator().manual_seed(seed + 11)
+    z = (torch.randn(w.batch, w.seqlen, w.nheads, w.headdim, generator=g) * 2.0).to(torch.bfloat16).to(dev)
+    nw = (torch.rand(w.nheads * w.headdim, generator=g) + 0.5).float().to(dev)
+    gs = 64
+    shp = ssd.make_shape(d["x"], d["B"], w.chunk_size)
+    ws = torch.empty(max(ssd.ssd_fwd_gated_workspace_size(shp, gs), ssd.ssd_fwd_workspace_size(shp), 1),
+                     dtype=torch.uint8, device=dev)
+    out = torch.empty_like(d["x"])
+    y = torch.empty_like(d["x"])
+    fin = torch.empty((w.batch, w.nheads, w.headdim, w.dstate), dtype=torch.float32, device=dev)
+
+    def fused():
+        ssd.ssd_fwd_gated(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], z=z, norm_weight=nw, group_size=gs,
+                          eps=1e-5, chunk_size=w.chunk_size, out=out, final_states=fin,
+                          return_final_states=True, workspace=ws, stream=stream)
+
+    def separate():
+        ssd.ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], chunk_size=w.chunk_size, y=y,
+                    final_states=fin, return_final_states=True, workspace=ws, stream=stream)
+        ssd.ssd_gated_rmsnorm(y, z, nw, group_size=gs, eps=1e-5, out=out, stream=stream)
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+    ms_f = timed(fused)
+    ms_s = timed(separate)
+    _, by = alg_counts(w, with_final=True)
+    by += 2.0 * w.batch * w.seqlen * w.nheads * w.headdim + 4.0 * w.nheads * w.headdim   # z, weight
+    pk, pk_kind = peaks()
+    ach = by / (ms_f / 1e3) / 1e9
+    return {"metric": GATED_METRIC, "value": w.tokens / (ms_f / 1e3) / 1e6, "unit": UNIT,
+            "ms_per_step": ms_f, "steps": steps, "warmup": warmup, "dtype": "bf16",
+            "config": {"workload": w.name, **w.shape_dict(), "group_size": gs, "eps": 1e-5,
+                       "plan": ssd.ssd_fwd_plan(shp)[0]},
+            "separate_ms_per_step": ms_s, "saved_ms_per_step": ms_s - ms_f,
+            "y_round_trip_bytes_saved": 2.0 * 2.0 * w.batch * w.seqlen * w.nheads * w.headdim,
+            "roofline": {"kernel": "ssd_fused_kernel (gated stores)", "bound": "hbm", "achieved": ach,
+                         "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": ach / pk["hbm_gbs"],
+                         "alg_bytes_per_step": by, "traffic": None, "peak_source": pk_kind},
+            "gpu_launches": steps}
+
+
 # ------------------------------------------------------------------ context parallelism
 CP = W.LONG_CONTEXT
 CP_METRIC = ("SSD fwd Mtokens/s, long context (b1 T65536 H32 P64 N128 G8) split over the "
@@ -796,6 +859,7 @@ def run_ours(args):
     gate = None
     varlen = None
     sweeps = None
+    gated = None
     if not args.profile:
         # secondary rows, measured after the headline: a failure here is reported in
         # its own entry and does not take the headline line down with it
@@ -814,6 +878,7 @@ def run_ours(args):
         gate = guarded(measure_gate, ssd, dev, stream, 100, 5, seed=rank)
         varlen = guarded(measure_varlen, ssd, dev, stream, 20, 3, seed=rank)
         sweeps = guarded(measure_sweeps, ssd, dev, stream, seed=rank)
+        gated = guarded(measure_fwd_gated, ssd, dev, stream, 50, 5, seed=rank)
 
     if rank == 0:
         line = {
@@ -834,7 +899,7 @@ def run_ours(args):
             "clocks": clk,
             "workload_rows": sweeps,
             "next_rows": {"decode_step": decode, "context_parallel": cp, "gate_norm": gate,
-                          "packed_docs": varlen},
+                          "fwd_gate_fused": gated, "packed_docs": varlen},
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -231,6 +231,36 @@ SSD_API ssd_status_t ssd_fwd_varlen_check(const ssd_shape_t* shape, int64_t n_do
                                           void* stream);
 
 /*
+ * The forward followed by the gate and normalisation of the Mamba-2 block
+ * (Knowl 6, step 4), without the layer output y ever reaching memory:
+ *     y   = ssd_fwd(x, dt, A, B, C, D, initial_states)
+ *     out = ssd_gated_rmsnorm(y, z, norm_weight, group_size, eps)
+ * with y rounded to dtype in between, as the two separate calls would have it.
+ * When ssd_fwd_plan names the single-pass kernel and group_size divides a
+ * head's 64 channels (8, 16, 32 or 64) the kernel gates and normalises each
+ * staged row before storing it: out is written instead of y and y costs no
+ * memory traffic. Otherwise y is written to the workspace and the gate kernel
+ * follows (two launches more).
+ *   z                  [b, T, H, P] in dtype (16-byte aligned), the gate branch.
+ *   norm_weight        [H * P] fp32, 16-byte aligned.
+ *   group_size, eps    as for ssd_gated_rmsnorm (group_size divides H * P).
+ *   out                [b, T, H, P] in dtype, in y's place for every rule of ssd_fwd.
+ *   final_states       as for ssd_fwd.
+ *   workspace          ssd_fwd_gated_workspace_size() bytes: ssd_fwd's workspace,
+ *                      plus room for y when the gate does not fuse.
+ * z, norm_weight must not overlap out, final_states or the workspace.
+ */
+SSD_API ssd_status_t ssd_fwd_gated_workspace_size(const ssd_shape_t* shape, int64_t group_size,
+                                                  size_t* bytes);
+SSD_API ssd_status_t ssd_fwd_gated(const ssd_shape_t* shape,
+                                   const void* x, const float* dt, const float* A,
+                                   const void* B, const void* C, const float* D,
+                                   const float* initial_states,
+                                   const void* z, const float* norm_weight, int64_t group_size,
+                                   float eps, void* out, float* final_states,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Recurrent (linear) form for the decoding mode of the layer (Knowl 1, linear
  * form: each new token costs O(P N) per head, however long the context): runs
  * shape->seqlen tokens per batch row from `state` and leaves the state after

@@ -24,7 +24,7 @@ from ._lib import (SSD_BF16, SSD_F32, SSDError, ShapeT, check, lib, lib_path,  #
 
 __all__ = ["ssd_fwd", "ssd_fwd_host", "ssd_fwd_workspace_size", "ssd_fwd_plan", "ssd_fwd_check",
            "ssd_step", "ssd_fwd_cp", "ssd_cp_begin", "ssd_cp_end", "ssd_cp_record_floats",
-           "ssd_gated_rmsnorm", "ssd_fwd_varlen", "ssd_fwd_varlen_workspace_size",
+           "ssd_gated_rmsnorm", "ssd_fwd_gated", "ssd_fwd_gated_workspace_size", "ssd_fwd_varlen", "ssd_fwd_varlen_workspace_size",
            "ssd_fwd_varlen_check", "ssd_chunk_cumsum",
            "ssd_chunk_state", "ssd_state_passing", "ssd_chunk_scan", "SSDError", "make_shape",
            "lib_path"]
@@ -110,6 +110,39 @@ def check_cu_seqlens(cu_seqlens, T: int) -> list[int]:
     if len(cu) < 2 or cu[0] != 0 or cu[-1] != T or any(b < a for a, b in zip(cu, cu[1:])):
         raise ValueError("cu_seqlens must run from 0 to T, non-decreasing")
     return cu
+
+
+def ssd_fwd_gated_workspace_size(shape: ShapeT, group_size: int) -> int:
+    n = ctypes.c_size_t(0)
+    check(lib().ssd_fwd_gated_workspace_size(ctypes.byref(shape), ctypes.c_int64(group_size), ctypes.byref(n)),
+          "ssd_fwd_gated_workspace_size")
+    return int(n.value)
+
+
+def ssd_fwd_gated(x, dt, A, B, C, D=None, z=None, norm_weight=None, group_size: int = 64,
+                  eps: float = 1e-5, chunk_size: int = 256, initial_states=None,
+                  return_final_states: bool = False, out=None, final_states=None, workspace=None,
+                  stream=None):
+    """The forward, then y * SiLU(z) RMS-normalised over channel groups times norm_weight
+    (Knowl 6), without storing y when the single-pass kernel can apply the gate (groups
+    of 8, 16, 32 or 64 channels). Returns out, or (out, final_states)."""
+    _need(x, "x")
+    _need(z, "z", x.dtype)
+    _need(norm_weight, "norm_weight", torch.float32)
+    shape = make_shape(x, B, chunk_size)
+    if out is None:
+        out = torch.empty_like(x)
+    if final_states is None and return_final_states:
+        final_states = torch.empty((x.shape[0], x.shape[2], x.shape[3], B.shape[3]),
+                                   dtype=torch.float32, device=x.device)
+    nbytes = ssd_fwd_gated_workspace_size(shape, group_size)
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=x.device)
+    check(lib().ssd_fwd_gated(ctypes.byref(shape), _p(x), _p(dt), _p(A), _p(B), _p(C), _p(D),
+                              _p(initial_states), _p(z), _p(norm_weight), ctypes.c_int64(group_size),
+                              ctypes.c_float(eps), _p(out), _p(final_states), _p(workspace),
+                              ctypes.c_size_t(nbytes), _stream(stream)), "ssd_fwd_gated")
+    return (out, final_states) if return_final_states else out
 
 
 def ssd_fwd_varlen_workspace_size(shape: ShapeT, n_docs: int) -> int:

@@ -53,6 +53,10 @@ _SIGS = {
                        + [ctypes.c_size_t, _VP], ctypes.c_int),
     "ssd_fwd_varlen_check": ([ctypes.POINTER(ShapeT), ctypes.c_int64, _VP, ctypes.c_size_t, _VP],
                              ctypes.c_int),
+    "ssd_fwd_gated_workspace_size": ([ctypes.POINTER(ShapeT), ctypes.c_int64,
+                                      ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
+    "ssd_fwd_gated": ([ctypes.POINTER(ShapeT)] + [_VP] * 9 + [ctypes.c_int64, ctypes.c_float]
+                      + [_VP] * 3 + [ctypes.c_size_t, _VP], ctypes.c_int),
     "ssd_step": ([ctypes.POINTER(ShapeT)] + [_VP] * 9, ctypes.c_int),
     "ssd_cp_record_floats": ([ctypes.POINTER(ShapeT), ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
     "ssd_cp_workspace_size": ([ctypes.POINTER(ShapeT), ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),

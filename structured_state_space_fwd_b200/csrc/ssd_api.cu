@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -257,9 +258,18 @@ int test_stall() {
 #endif
 }
 
+// The gate and norm applied in the single-pass kernel's stores (z null: none).
+struct FusedGate {
+    const void* z = nullptr;
+    const float* w = nullptr;
+    int64_t group_size = 0;
+    float eps = 0.f;
+};
+
 ssd_status_t run_fwd(const ssd::Dims& d, const void* x, const float* dt, const float* A,
                      const void* B, const void* C, const float* D, const float* init, void* y,
-                     float* final_states, void* workspace, cudaStream_t stream) {
+                     float* final_states, void* workspace, cudaStream_t stream,
+                     const FusedGate& gate = FusedGate()) {
     if (d.b == 0) return SSD_OK;
     if (d.T == 0) return cuda_status("final states", ssd::launch_copy_or_zero_states(d, init, final_states, stream));
     const FwdWorkspace w = fwd_workspace(d);
@@ -303,6 +313,10 @@ ssd_status_t run_fwd(const ssd::Dims& d, const void* x, const float* dt, const f
         a.chained = w.sp.chained ? 1 : 0;
         a.stall = test_stall();
         a.y = y;
+        a.z = gate.z;
+        a.nw = gate.w;
+        a.gs = (int)gate.group_size;
+        a.eps = gate.eps;
         return cuda_status("fused forward", ssd::launch_fused(a, stream));
     }
     float* cs = (float*)(ws + w.off_cs);
@@ -559,6 +573,65 @@ ssd_status_t ssd_fwd(const ssd_shape_t* shape, const void* x, const float* dt, c
     if (st != SSD_OK) return st;
     return run_fwd(ssd::make_dims(*shape), x, dt, A, B, C, D, initial_states, y, final_states,
                    workspace, (cudaStream_t)stream);
+}
+
+// Forward plus the gate and norm of the block: the single-pass kernel applies them
+// in its stores when the plan is single-pass and the groups lie inside a head;
+// otherwise y goes to the workspace and the separate gate kernel follows.
+bool gated_fuses(const ssd::Dims& d, int64_t group_size) {
+    const Path p = pick_path(d);
+    return (p == Path::Fused || p == Path::Segmented) && ssd::fused_gate_ok(group_size);
+}
+
+ssd_status_t ssd_fwd_gated_workspace_size(const ssd_shape_t* shape, int64_t group_size, size_t* bytes) {
+    if (!bytes) return SSD_ERR_INVALID_ARG;
+    ssd_status_t st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    const ssd::Dims d = ssd::make_dims(*shape);
+    if (group_size < 1 || (d.H * d.P) % group_size != 0) return SSD_ERR_INVALID_ARG;
+    const size_t fw = fwd_workspace(d).total;
+    *bytes = gated_fuses(d, group_size) ? fw : align_up(fw, 256) + sizes_of(d).x;
+    return SSD_OK;
+}
+
+ssd_status_t ssd_fwd_gated(const ssd_shape_t* shape, const void* x, const float* dt, const float* A,
+                           const void* B, const void* C, const float* D, const float* initial_states,
+                           const void* z, const float* norm_weight, int64_t group_size, float eps,
+                           void* out, float* final_states, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+    size_t need = 0;
+    ssd_status_t st = ssd_fwd_gated_workspace_size(shape, group_size, &need);
+    if (st != SSD_OK) return st;
+    if (workspace_bytes < need || !(eps >= 0.f) || !std::isfinite(eps)) return SSD_ERR_INVALID_ARG;
+    const ssd::Dims d = ssd::make_dims(*shape);
+    const Sizes z0 = sizes_of(d);
+    if ((!z && z0.x) || !norm_weight || !aligned(z, 16) || !aligned(norm_weight, 16)) return SSD_ERR_INVALID_ARG;
+    const Range zr[] = {{z, z0.x}, {norm_weight, (size_t)(d.H * d.P) * 4}};
+    for (const Range& r : zr)
+        if (overlaps(r, Range{out, z0.x}) || overlaps(r, Range{final_states, final_states ? z0.st : 0}) ||
+            overlaps(r, Range{workspace, need}))
+            return SSD_ERR_INVALID_ARG;
+    if (gated_fuses(d, group_size)) {
+        // out takes y's place: every check of ssd_fwd applies to it
+        if ((st = check_fwd_args(shape, x, dt, A, B, C, D, initial_states, out, final_states, workspace,
+                                 workspace_bytes)) != SSD_OK)
+            return st;
+        FusedGate g;
+        g.z = z;
+        g.w = norm_weight;
+        g.group_size = group_size;
+        g.eps = eps;
+        return run_fwd(d, x, dt, A, B, C, D, initial_states, out, final_states, workspace, (cudaStream_t)stream, g);
+    }
+    char* yb = (char*)workspace + align_up(fwd_workspace(d).total, 256);
+    if ((st = check_fwd_args(shape, x, dt, A, B, C, D, initial_states, yb, final_states, workspace,
+                             fwd_workspace(d).total)) != SSD_OK)
+        return st;
+    if (overlaps(Range{out, z0.x}, Range{workspace, need})) return SSD_ERR_INVALID_ARG;
+    if ((st = run_fwd(d, x, dt, A, B, C, D, initial_states, yb, final_states, workspace,
+                      (cudaStream_t)stream)) != SSD_OK)
+        return st;
+    return ssd_gated_rmsnorm(shape, yb, z, norm_weight, group_size, eps, out, stream);
 }
 
 // Host-buffer variant: [fwd workspace | x | dt | A | B | C | D | init | y | final]

@@ -43,7 +43,9 @@
 //   warps 8-15  chain group (thread = state row, half of the head dim): carries
 //               the state, per tile the bf16 operand of C (2^L h)^T
 //   warps 16-19 epilogue group (thread = token row): per tile and head
-//               y = q Y'', staged in shared memory, one TMA store per warp
+//               y = q Y'', staged in shared memory (optionally gated by SiLU(z)
+//               and RMS-normalised over groups within the head), one TMA store
+//               per warp
 //
 // Every wait is bounded; a wait that gives up sets the error word and makes
 // every role leave its loop, after which the CTA drains its MMAs and exits.
@@ -126,7 +128,12 @@ struct Params {
     int* ticket;
     int* error;
     int* flags;           // [b*nseg*nhb] state entering the segment written (chained)
-    void* y;              // [b,T,H,P] bf16, for rows a tile store must not cover
+    void* y;              // [b,T,H,P] bf16 (the gated output when z is set), for rows a
+                          // tile store must not cover
+    const __nv_bfloat16* z;   // gate branch [b,T,H,P] bf16, or null: y is stored as is
+    const float* nw;      // norm weight [H*P] fp32 (with z)
+    int gs;               // norm group size, dividing 64 and a multiple of 8 (with z)
+    float eps;            // norm epsilon (with z)
     const int* cu;        // packed documents: token offsets [ndoc+1] in batch row 0, or null
     const int* order;     // packed documents: unit order (documents, longest first)
     int64_t T;
@@ -347,7 +354,68 @@ __device__ __forceinline__ void mma_tokens_tmem(uint32_t d, uint32_t a, uint64_t
         mma_bf16_tmem_a(d, a + 8 * kk, dB + (uint64_t)(kk * 128), idesc, 1u);
 }
 
-template <int NS>
+// One group size's pass of gate_row below (v recomputed for the scaling rather than
+// held, to stay inside the registers).
+template <int GC>   // 16-byte chunks (8 channels) per group
+__device__ __forceinline__ void gate_row_g(const uint4 (&zv)[8], const float* w, float eps, uint8_t* stg, int r) {
+    constexpr float kInvGs = 1.f / (8 * GC);
+    auto gated = [&](int c, float (&v)[8]) {
+        const uint4 yv = *reinterpret_cast<const uint4*>(stg + swz(r, c));
+        const uint32_t ys4[4] = {yv.x, yv.y, yv.z, yv.w};
+        const uint32_t zs4[4] = {zv[c].x, zv[c].y, zv[c].z, zv[c].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 y2 = unpack_bf16(ys4[k]), z2 = unpack_bf16(zs4[k]);
+            v[2 * k] = y2.x * __fdividef(z2.x, 1.f + ex2(-z2.x * kLog2e));
+            v[2 * k + 1] = y2.y * __fdividef(z2.y, 1.f + ex2(-z2.y * kLog2e));
+        }
+    };
+#pragma unroll
+    for (int c0 = 0; c0 < 8; c0 += GC) {
+        float ss = 0.f;
+#pragma unroll
+        for (int c = c0; c < c0 + GC; ++c) {
+            float v[8];
+            gated(c, v);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) ss = fmaf(v[k], v[k], ss);
+        }
+        const float inv = rsqrtf(ss * kInvGs + eps);
+#pragma unroll
+        for (int c = c0; c < c0 + GC; ++c) {
+            float v[8];
+            gated(c, v);
+            const float4 w0 = __ldg(reinterpret_cast<const float4*>(w + 8 * c));
+            const float4 w1 = __ldg(reinterpret_cast<const float4*>(w + 8 * c + 4));
+            const float wk[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+            uint32_t o[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) o[k] = pack_bf16(v[2 * k] * inv * wk[2 * k], v[2 * k + 1] * inv * wk[2 * k + 1]);
+            *reinterpret_cast<uint4*>(stg + swz(r, c)) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+    }
+}
+// The gate and normalisation after the layer ("Transformers are SSMs", Knowl 6,
+// step 4) on one staged row of 64 channels (head hh of one token, bf16 y in the
+// 128-byte-swizzled staging row r), in place: v = y * SiLU(z), then each group
+// of gs channels is divided by sqrt(mean(v^2) + eps) and scaled by the weight.
+// y is the bf16 value a separate pass would read back. zrow indexes [b,T,H] of z.
+__device__ __forceinline__ void gate_row(const __nv_bfloat16* z, const float* nw, int gs, float eps, uint8_t* stg,
+                                     int r, int64_t zrow, int hh) {
+    const uint4* zp = reinterpret_cast<const uint4*>(z + zrow * kP);
+    uint4 zv[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) zv[c] = __ldcs(zp + c);   // read once: streamed past L1
+    const float* w = nw + (int64_t)hh * kP;
+    switch (gs) {
+        case 8: gate_row_g<1>(zv, w, eps, stg, r); break;
+        case 16: gate_row_g<2>(zv, w, eps, stg, r); break;
+        case 32: gate_row_g<4>(zv, w, eps, stg, r); break;
+        default: gate_row_g<8>(zv, w, eps, stg, r); break;
+    }
+}
+
+template <int NS, bool kGate>
 __global__ void __launch_bounds__(kThreads, 1)
     ssd_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_B,
                      const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ CUtensorMap tm_y,
@@ -1055,26 +1123,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                             *reinterpret_cast<uint4*>(stg + swz(r, 2 * pc + cc)) = make_uint4(o[0], o[1], o[2], o[3]);
                         }
                     }
+                    if (e == np - 1) {
+                        // the tile's accumulators are read: free them before the stores
+                        tc_fence_before();
+                        mbar_arrive(&bs->y_empty[ys]);
+                        if (!shared) mbar_arrive_cnt(&bs->s_empty, 2);
+                    }
+                    const int hh = U.hb * np + e;
+                    if (kGate && t0 + r < U.len)
+                        gate_row(prm.z, prm.nw, prm.gs, prm.eps, stg, r, ((int64_t)U.b * T + U.tok0 + t0 + r) * H + hh, hh);
                     const int64_t row0 = t0 + 32 * q;   // the warp's first row in the sequence
                     if (row0 + 32 <= U.len) {
                         fence_proxy_async_smem();
                         __syncwarp();
                         if (lane == 0) {
-                            tma_store_4d(&tm_y, stg + q * (kAtom / 4), 0, U.hb * np + e, (int)(U.tok0 + row0), U.b);
+                            tma_store_4d(&tm_y, stg + q * (kAtom / 4), 0, hh, (int)(U.tok0 + row0), U.b);
                             bulk_commit_group();
                         }
                     } else if (t0 + r < U.len) {
                         // the sequence ends inside the warp's rows: the rows after it belong to
                         // the next document (or lie past the row), so each thread stores its own
                         uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(prm.y) +
-                            (((int64_t)U.b * T + U.tok0 + t0 + r) * H + U.hb * np + e) * kP);
+                            (((int64_t)U.b * T + U.tok0 + t0 + r) * H + hh) * kP);
 #pragma unroll
                         for (int c = 0; c < 8; ++c) dst[c] = *reinterpret_cast<const uint4*>(stg + swz(r, c));
                     }
                 }
-                tc_fence_before();
-                mbar_arrive(&bs->y_empty[ys]);
-                if (!shared) mbar_arrive_cnt(&bs->s_empty, 2);
             }
         }
     }
@@ -1093,15 +1167,15 @@ int num_sms() {
     return n > 0 ? n : 148;
 }
 
-template <int NS>
+template <int NS, bool kGate>
 cudaError_t launch_ns(const FusedLaunch& a, const Params& prm, cudaStream_t st) {
     using K = Cfg<NS>;
-    cudaError_t e = cudaFuncSetAttribute(ssd_fused_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)K::kSmem);
+    auto kern = ssd_fused_kernel<NS, kGate>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K::kSmem);
     if (e != cudaSuccess) return e;
     const int sms = num_sms();
     const int grid = prm.nunits < sms ? prm.nunits : sms;
-    ssd_fused_kernel<NS><<<grid, kThreads, K::kSmem, st>>>(a.maps[0], a.maps[1], a.maps[2], a.maps[3], prm);
+    kern<<<grid, kThreads, K::kSmem, st>>>(a.maps[0], a.maps[1], a.maps[2], a.maps[3], prm);
     return cudaGetLastError();
 }
 
@@ -1174,6 +1248,11 @@ cudaError_t launch_fused(const FusedLaunch& a, cudaStream_t st) {
     prm.error = a.sync_ints + 1;
     prm.flags = a.sync_ints + 2;
     prm.y = a.y;
+    prm.z = static_cast<const __nv_bfloat16*>(a.z);
+    prm.nw = a.nw;
+    prm.gs = a.gs;
+    prm.eps = a.eps;
+    if (a.z && (!a.nw || !fused_gate_ok(a.gs))) return cudaErrorInvalidValue;
     prm.cu = a.cu;
     prm.order = a.order;
     prm.T = d.T;
@@ -1197,7 +1276,8 @@ cudaError_t launch_fused(const FusedLaunch& a, cudaStream_t st) {
     prm.nseg = a.nseg;
     prm.chained = a.chained;
     prm.stall = a.stall;
-    return ns == 128 ? launch_ns<128>(a, prm, st) : launch_ns<256>(a, prm, st);
+    if (a.z) return ns == 128 ? launch_ns<128, true>(a, prm, st) : launch_ns<256, true>(a, prm, st);
+    return ns == 128 ? launch_ns<128, false>(a, prm, st) : launch_ns<256, false>(a, prm, st);
 }
 
 }  // namespace ssd

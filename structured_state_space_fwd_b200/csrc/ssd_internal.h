@@ -68,6 +68,13 @@ struct FusedLaunch {
     int chained;               // segment s > 0 takes its entering state from segment s - 1's unit
     int stall;                 // test builds: make chain waits run out
     void* y;                   // [b,T,H,P] bf16 (the map's tensor): rows of partial tiles
+    // gate and norm after the layer, fused into the stores (z null: y stored as is):
+    // out = RMSNorm over groups of gs channels of y * SiLU(z), times nw; y is then the
+    // output buffer and the map is over it. gs divides 64 and is a multiple of 8.
+    const void* z;
+    const float* nw;
+    int gs;
+    float eps;
     // packed documents (d.b == 1, nseg == 1): document k is tokens cu[k] .. cu[k+1]-1;
     // init / finalbuf are [ndoc,H,P,N]; units run in `order` (varlen_order output)
     const int* cu;
@@ -75,6 +82,12 @@ struct FusedLaunch {
     int ndoc;
 };
 cudaError_t launch_fused(const FusedLaunch& a, cudaStream_t st);
+
+// Whether the single-pass kernel's stores can apply the gate and norm for this
+// group size (groups inside one head's 64 channels).
+inline bool fused_gate_ok(int64_t group_size) {
+    return group_size >= 8 && group_size <= 64 && 64 % group_size == 0 && group_size % 8 == 0;
+}
 
 // Packed documents: order[ndoc] = documents by decreasing length (ties by index;
 // identity order above varlen_sort_max() documents), and *bad = 1 when cu is not a

@@ -1,0 +1,132 @@
+"""ssd_fwd_gated: the forward followed by the gate and RMSNorm of the Mamba-2 block
+(Knowl 6, step 4). Groups inside a head (8..64 channels) are applied in the
+single-pass kernel's stores; others go through the workspace.
+
+Two bars:
+  * the gate's own arithmetic: out against the fp64 oracle's gated_rmsnorm of the
+    layer output the library computes (ssd_fwd, the same kernel and arithmetic
+    without the gate), max|out - ref| / max|ref| <= 5e-3;
+  * the whole composition against gated_rmsnorm(recurrence(...).y) in fp64, with
+    the error bound the normalisation puts on a y held to 5e-3 of max|y|: per
+    group g, v = y * SiLU(z) and out = w * v / rms(v), whose Jacobian in v has
+    norm 1 / rms(v), so ||out - ref||_g <= max|w_g| * ||dy * SiLU(z)||_g / rms_g
+    with |dy| <= 5e-3 max|y|, plus the output's bf16 rounding. A group of small
+    rms amplifies the forward's error, which is why the 5e-3 of max|out| is not
+    the bar for the composition.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import ssd_inputs as W
+from ssd_inputs import make_inputs
+
+pytestmark = pytest.mark.gpu
+TOL = 5e-3
+
+
+@pytest.fixture(scope="module")
+def ssd(cuda_device):
+    from structured_state_space_fwd_b200 import build
+    build.build()
+    import structured_state_space_fwd_b200 as m
+    return m
+
+
+def gate_inputs(b, T, H, P, seed):
+    rng = np.random.Generator(np.random.PCG64(seed))
+    z = torch.from_numpy(rng.standard_normal((b, T, H, P)) * 2.0).to(torch.bfloat16)
+    w = torch.from_numpy(rng.uniform(0.5, 1.5, H * P)).float()
+    return z, w
+
+
+def run_case(ssd, monkeypatch, b, T, H, G, N, gs, seed, path=None, scale=None, eps=1e-5):
+    if path is None:
+        monkeypatch.delenv("SSD_PATH", raising=False)
+    else:
+        monkeypatch.setenv("SSD_PATH", path)
+    inp = make_inputs(b, T, H, 64, G, N, dtype="bf16", initial_states=True, seed=seed)
+    if scale is not None:
+        inp["dt"] = inp["dt"] * scale
+    z, w = gate_inputs(b, T, H, 64, seed + 1)
+    d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+    out, fin = ssd.ssd_fwd_gated(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], z=z.cuda(),
+                                 norm_weight=w.cuda(), group_size=gs, eps=eps,
+                                 initial_states=d["initial_states"], return_final_states=True)
+    torch.cuda.synchronize()
+    y_ref, f_ref, _ = oracle.recurrence(**inp)
+    oc = out.float().cpu()
+    assert torch.isfinite(oc).all()
+    assert oracle.rel_err(fin.cpu(), f_ref) <= TOL
+    y = ssd.ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], initial_states=d["initial_states"])
+    sep = ssd.ssd_gated_rmsnorm(y, z.cuda(), w.cuda(), group_size=gs, eps=eps)
+    torch.cuda.synchronize()
+    check_gate(oc, y.float().cpu(), y_ref, z, w, gs, eps)
+    # the two separate calls agree up to the bf16 rounding of the output
+    assert oracle.rel_err(oc, sep.float().cpu()) <= 8e-3
+    return ssd.ssd_fwd_plan(ssd.make_shape(d["x"], d["B"], 256))[0]
+
+
+def check_gate(oc, y_dev, y_ref, z, w, gs, eps):
+    """Both bars of the module docstring."""
+    assert oracle.rel_err(y_dev, y_ref) <= TOL
+    e = oracle.rel_err(oc, oracle.gated_rmsnorm(y_dev, z, w, gs, eps))
+    assert e <= TOL, f"gate arithmetic: rel err {e:.3e}"
+    ref = oracle.gated_rmsnorm(y_ref, z, w, gs, eps)
+    C = y_ref.shape[-2] * y_ref.shape[-1]
+    zz = oracle._f64(z).reshape(-1, C // gs, gs)
+    silu = zz / (1.0 + np.exp(-zz))
+    v = np.asarray(y_ref).reshape(-1, C // gs, gs) * silu
+    rms = np.sqrt(np.mean(v * v, axis=-1) + eps)
+    wmax = np.abs(oracle._f64(w)).reshape(C // gs, gs).max(axis=-1)
+    dy = TOL * np.abs(np.asarray(y_ref)).max()
+    bound = 1.5 * wmax * dy * np.linalg.norm(silu, axis=-1) / rms
+    refg = np.asarray(ref).reshape(-1, C // gs, gs)
+    bound = bound + 2.0 ** -8 * np.linalg.norm(refg, axis=-1) + 1e-30
+    err = np.linalg.norm(oracle._f64(oc).reshape(-1, C // gs, gs) - refg, axis=-1)
+    worst = float((err / bound).max())
+    assert worst <= 1.0, f"composition: a group's error is {worst:.2f} of its bound"
+
+
+@pytest.mark.parametrize("gs", [8, 16, 32, 64])
+def test_fused_gate_groups_in_a_head(ssd, monkeypatch, gs):
+    plan = run_case(ssd, monkeypatch, 2, 700, 8, 2, 128, gs, seed=gs)
+    assert plan == "fused"
+
+
+@pytest.mark.parametrize("N,H,G", [(256, 4, 2), (64, 6, 3), (128, 5, 5)])
+def test_fused_gate_state_sizes(ssd, monkeypatch, N, H, G):
+    run_case(ssd, monkeypatch, 2, 300, H, G, N, 64, seed=N + H)
+
+
+def test_fused_gate_unfactored_tiles(ssd, monkeypatch):
+    # strong decay: tiles take the unfactored form (y = Y'' + 2^cs R in the epilogue)
+    run_case(ssd, monkeypatch, 2, 600, 4, 1, 128, 32, seed=77, scale=64.0)
+
+
+def test_fused_gate_segmented(ssd, monkeypatch):
+    run_case(ssd, monkeypatch, 1, 128 * 12 + 5, 4, 1, 128, 64, seed=78, path="segmented")
+
+
+@pytest.mark.parametrize("gs,path", [(128, None), (512, None), (64, "steps")])
+def test_gate_through_workspace(ssd, monkeypatch, gs, path):
+    # groups wider than a head, or a plan without the single-pass kernel: y goes through
+    # the workspace and the gate kernel
+    run_case(ssd, monkeypatch, 2, 333, 8, 2, 128, gs, seed=gs + 3, path=path)
+
+
+def test_fused_gate_full_size(ssd, monkeypatch):
+    # the 2.7B layer with per-head groups, every element
+    monkeypatch.delenv("SSD_PATH", raising=False)
+    w_ = W.MAMBA2_27B_LAYER
+    inp = W.workload_inputs(w_)
+    z, w = gate_inputs(w_.batch, w_.seqlen, w_.nheads, w_.headdim, 5)
+    d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+    out = ssd.ssd_fwd_gated(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], z=z.cuda(), norm_weight=w.cuda(),
+                            group_size=64, eps=1e-5, initial_states=d["initial_states"])
+    torch.cuda.synchronize()
+    y = ssd.ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], initial_states=d["initial_states"])
+    torch.cuda.synchronize()
+    y_ref, _, _ = oracle.recurrence(**inp)
+    check_gate(out.float().cpu(), y.float().cpu(), y_ref, z, w, 64, 1e-5)

@@ -402,3 +402,32 @@ def test_full_long_context(ssd, path_env):
 def test_full_mamba2_layer_other_path(ssd, path_env, path):
     # the 2.7B layer in the path ssd_fwd does not pick for it, every element too
     full_check(ssd, path_env, W.MAMBA2_27B_LAYER, reps=1, path=path)
+
+
+def test_fused_with_other_work_on_the_gpu(ssd, path_env):
+    # Units are handed out by an atomic ticket to CTAs that are already running, so
+    # a chained segment's predecessor is always taken before it. Here another
+    # stream's elementwise kernel holds SMs while the forward starts, so the fused
+    # kernel's CTAs become resident at different times; the result and the device
+    # status must not depend on that.
+    path_env(None)
+    inp = make_inputs(batch=4, seqlen=1024 + 77, nheads=80, headdim=64, ngroups=1, dstate=128,
+                      dtype="bf16", initial_states=True, seed=4242)
+    d = to_dev(inp)
+    shp = ssd.make_shape(d["x"], d["B"], 256)
+    assert ssd.ssd_fwd_plan(shp)[0] == "fused"
+    ws = torch.empty(ssd.ssd_fwd_workspace_size(shp), dtype=torch.uint8, device="cuda")
+    big = torch.ones(1 << 28, dtype=torch.float32, device="cuda")   # 1 GiB
+    side = torch.cuda.Stream()
+    y_ref, f_ref, _ = oracle.recurrence(**inp)
+    for _ in range(3):
+        torch.cuda.synchronize()
+        with torch.cuda.stream(side):
+            for _ in range(4):
+                big.mul_(1.0000001)
+        y, f = ssd.ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], chunk_size=256,
+                           initial_states=d["initial_states"], return_final_states=True, workspace=ws)
+        ssd.ssd_fwd_check(shp, ws)      # raises on a device-side timeout
+        torch.cuda.synchronize()
+        assert oracle.rel_err(y.float().cpu(), y_ref) <= TOL["bf16"]
+        assert oracle.rel_err(f.cpu(), f_ref) <= TOL["bf16"]
