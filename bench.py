@@ -543,6 +543,16 @@ def cp_setup(ssd, dev, w, nranks, rank, seed=0):
     return d, Ts
 
 
+def cp_kernels_per_step(ssd, d, w, rank):
+    """Launches of one rank's ssd_cp_begin + ssd_cp_end: on the single-pass plan the
+    segment-state pass and its scan, the fold (ranks > 0) and the slice's forward;
+    otherwise chunk cumsum, chunk states, state passing and the slice decay, then the
+    fold, state passing and the chunk scan."""
+    path, nk = ssd.ssd_fwd_plan(ssd.make_shape(d["x"], d["B"], w.chunk_size))
+    fold = 1 if rank > 0 else 0
+    return 2 + fold + nk if path in ("fused", "segmented") else 4 + fold + 2
+
+
 def measure_cp_slice(ssd, dev, stream, steps, warmup, nranks=8):
     """One rank's work in an nranks-way split of the long-context sequence, timed on
     one GPU: ssd_cp_begin, then ssd_cp_end of the last rank (which folds the most
@@ -577,7 +587,7 @@ def measure_cp_slice(ssd, dev, stream, steps, warmup, nranks=8):
                     f"(rank {rank}); the all-gather of {nranks} records of "
                     f"{4 * w.batch * w.nheads * (w.headdim * w.dstate + 1) / 2**20:.2f} MiB is not timed",
             "ms_per_rank_step": ms, "slice_tokens": Ts, "workload": w.name,
-            "kernels_per_rank_step": 7,
+            "kernels_per_rank_step": cp_kernels_per_step(ssd, d, w, rank),
             "roofline": {"bound": "hbm", "achieved": by / (ms / 1e3) / 1e9, "peak": pk["hbm_gbs"],
                          "unit": "GB/s", "frac": by / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
                          "alg_bytes_per_rank_step": by, "traffic": None,

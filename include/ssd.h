@@ -313,7 +313,7 @@ SSD_API ssd_status_t ssd_gated_rmsnorm(const ssd_shape_t* shape, const void* y, 
  * lengths, zero allowed); all ranks share batch, nheads, headdim, ngroups,
  * dstate, chunk_size and dtype, seqlen being the rank's own slice length. Per
  * rank and call:
- *   1. ssd_cp_begin: chunk cumsum and chunk states of the slice, then this
+ *   1. ssd_cp_begin: the state the slice reaches, then this
  *      rank's record = [s (b H P N floats) | alpha (b H floats) | pad], where
  *      s is the state the slice reaches from a zero state (rank 0: from the
  *      sequence's initial_states) and alpha[b,h] = prod_{t in slice} a_t.
@@ -321,13 +321,16 @@ SSD_API ssd_status_t ssd_gated_rmsnorm(const ssd_shape_t* shape, const void* y, 
  *      one buffer of R * record_floats floats (NCCL all-gather, or any
  *      collective with that result);
  *   3. ssd_cp_end: rank r's entering state h_in = fold over k < r of
- *      h <- alpha_k h + s_k from h = 0 (rank 0: initial_states), then the state
- *      passing from h_in and the chunk scan of the slice: y of the slice and,
- *      in final_states, the state after the slice (on the last rank, the
- *      sequence's final state).
- * The result equals ssd_fwd over the whole sequence up to rounding. Each step
- * runs the four-step kernels (tensor cores where ssd_fwd's steps path would);
- * the exchange is one record per rank (about 1 MiB at 32 heads x 64 x 128). */
+ *      h <- alpha_k h + s_k from h = 0 (rank 0: initial_states), then the
+ *      slice's forward from h_in: y of the slice and, in final_states, the
+ *      state after the slice (on the last rank, the sequence's final state).
+ * The result equals ssd_fwd over the whole sequence up to rounding. Where
+ * ssd_fwd takes the single-pass kernel (bf16, head dim 64, state a multiple of
+ * 16 up to 256), step 1 is the segment-state pass over the slice with its scan
+ * (two launches) and step 3 is the fold plus ssd_fwd from h_in; otherwise both
+ * run the four-step kernels (chunk cumsum and chunk states in step 1, state
+ * passing and chunk scan in step 3). The exchange is one record per rank
+ * (about 1 MiB at 32 heads x 64 x 128). */
 
 /* Floats in one rank's record (b*H*P*N + b*H, rounded up to a multiple of 4). */
 SSD_API ssd_status_t ssd_cp_record_floats(const ssd_shape_t* shape, size_t* floats);
@@ -338,7 +341,9 @@ SSD_API ssd_status_t ssd_cp_workspace_size(const ssd_shape_t* shape, size_t* byt
 /* Step 1 on this rank's slice. initial_states: the sequence's initial state on
  * rank 0, NULL on every other rank (and NULL on rank 0 for a zero state).
  * record: ssd_cp_record_floats() floats (16-byte aligned) receiving the record.
- * workspace: ssd_cp_workspace_size() bytes, kept untouched until ssd_cp_end. */
+ * workspace: ssd_cp_workspace_size() bytes, kept untouched until ssd_cp_end
+ * (it carries what step 3 needs from step 1: A, or the slice's chunk sums and
+ * chunk states). */
 SSD_API ssd_status_t ssd_cp_begin(const ssd_shape_t* shape,
                                   const void* x, const float* dt, const float* A,
                                   const void* B, const float* initial_states,

@@ -359,19 +359,51 @@ ssd_status_t read_device_status(const ssd::Dims& d, const void* workspace, cudaS
     return SSD_ERR_TIMEOUT;
 }
 
-// Sequence-parallel workspace (ssd_cp_begin fills cs and S, ssd_cp_end reads them):
-//   [cs | chunk states S | entry states | entering state h_in], regions 256-byte aligned.
+// Sequence-parallel workspace. Shapes the single-pass kernel takes: ssd_cp_begin
+// runs the segment-state pass over the slice and its scan (the record is the state
+// after the last segment, and the product of the segment decays) and keeps A for
+// ssd_cp_end, which folds the records into the entering state and runs the forward
+// from it:
+//   [A | status words | segment states [b, nseg+1, H, P, N] | segment decays [b, nseg, H]]
+//   with, after A, [entering state h_in | forward workspace] overlapping (end).
+// Other shapes (step paths; begin leaves cs and S for end):
+//   [cs | chunk states S | entry states | entering state h_in].
+// Regions are 256-byte aligned.
 struct CpWorkspace {
+    bool single_pass;
+    int kh, seg_tiles, nseg;                  // single pass: the segment-state pass
+    size_t off_sync, off_seg, off_decay;      // single pass, begin
+    size_t off_A, off_fwd;                    // single pass: A kept by begin; end (h_in at off_hin)
     size_t off_cs, off_S, off_entry, off_hin, total;
 };
 CpWorkspace cp_workspace(const ssd::Dims& d) {
     const Sizes z = sizes_of(d);
-    CpWorkspace w;
-    w.off_cs = 0;
-    w.off_S = align_up(z.cs, 256);
-    w.off_entry = w.off_S + align_up(z.chunk_states, 256);
-    w.off_hin = w.off_entry + align_up(z.chunk_states, 256);
-    w.total = w.off_hin + align_up(z.st, 256);
+    CpWorkspace w = {};
+    w.single_pass = fused_ok(d) && d.T > 0;
+    if (w.single_pass) {
+        const int64_t ntiles = (d.T + 127) / 128;
+        w.kh = ssd::pick_kheads(d.H / d.G);
+        const int64_t units_per_seg = std::max<int64_t>(1, d.b * (d.H / w.kh));
+        int64_t nseg = std::max<int64_t>(1, std::min<int64_t>(ntiles, (kTargetUnits + units_per_seg - 1) / units_per_seg));
+        int64_t K = std::min<int64_t>((ntiles + nseg - 1) / nseg, ssd::segment_max_tiles());
+        w.seg_tiles = (int)K;
+        w.nseg = (int)((ntiles + K - 1) / K);
+        w.off_A = 0;
+        w.off_sync = align_up(z.hv, 256);
+        w.off_seg = w.off_sync + 256;
+        w.off_decay = w.off_seg + align_up(z.st * (size_t)(w.nseg + 1), 256);
+        const size_t begin_total = w.off_decay + align_up((size_t)(d.b * d.H * w.nseg) * 4, 256);
+        w.off_hin = w.off_sync;
+        w.off_fwd = w.off_hin + align_up(z.st, 256);
+        const size_t end_total = w.off_fwd + align_up(fwd_workspace(d).total, 256);
+        w.total = std::max(begin_total, end_total);
+    } else {
+        w.off_cs = 0;
+        w.off_S = align_up(z.cs, 256);
+        w.off_entry = w.off_S + align_up(z.chunk_states, 256);
+        w.off_hin = w.off_entry + align_up(z.chunk_states, 256);
+        w.total = w.off_hin + align_up(z.st, 256);
+    }
     if (d.b == 0) w.total = 0;
     return w;
 }
@@ -948,6 +980,27 @@ ssd_status_t ssd_cp_begin(const ssd_shape_t* shape, const void* x, const float* 
         return cuda_status("slice decay", ssd::launch_slice_decay(d, nullptr, alpha, s));
     }
     char* ws = (char*)workspace;
+    if (w.single_pass) {
+        CUtensorMap maps[4];
+        if (!ssd::make_tc_maps(d, x, B, B, nullptr, maps)) {
+            ssd::set_error_detail("tensor map encoding failed");
+            return SSD_ERR_CUDA;
+        }
+        int* sync = (int*)(ws + w.off_sync);
+        float* segbuf = (float*)(ws + w.off_seg);
+        float* decay = (float*)(ws + w.off_decay);
+        const int nslot = w.nseg + 1;
+        if ((st = cuda_status("status word", cudaMemsetAsync(sync, 0, 16, s))) != SSD_OK ||
+            (st = cuda_status("A for the slice's forward", cudaMemcpyAsync(ws + w.off_A, A, z.hv,
+                                                                           cudaMemcpyDeviceToDevice, s))) != SSD_OK)
+            return st;
+        if ((st = cuda_status("segment states",
+                              ssd::launch_segment_states(d, maps, dt, A, segbuf, decay, sync + 1, w.seg_tiles,
+                                                         w.nseg, nslot, w.nseg, w.kh, s))) != SSD_OK)
+            return st;
+        return cuda_status("segment scan", ssd::launch_segment_scan(d, initial_states, segbuf, decay, w.nseg,
+                                                                    nslot, w.nseg, record, s, alpha));
+    }
     float* cs = (float*)(ws + w.off_cs);
     float* S = (float*)(ws + w.off_S);
     if ((st = cuda_status("chunk cumsum", ssd::launch_chunk_cumsum(d, dt, A, cs, s))) != SSD_OK) return st;
@@ -1006,6 +1059,8 @@ ssd_status_t ssd_cp_end(const ssd_shape_t* shape, int nranks, int rank, const fl
     }
     if (d.T == 0)
         return cuda_status("final states", ssd::launch_copy_or_zero_states(d, h_in, final_states, s));
+    if (w.single_pass)
+        return run_fwd(d, x, dt, (const float*)(ws + w.off_A), B, C, D, h_in, y, final_states, ws + w.off_fwd, s);
     const float* cs = (const float*)(ws + w.off_cs);
     const float* S = (const float*)(ws + w.off_S);
     float* entry = (float*)(ws + w.off_entry);

@@ -101,7 +101,8 @@ cudaError_t launch_varlen_order(const int* cu, int ndoc, int64_t T, int* order, 
 // its decay 2^(sum dt A log2 e) to decay[b,nseg,H] at s. The scan over segments then
 // turns slot s (1 <= s <= nseg_out) into the state entering segment s (init entering
 // segment 0) and, when `final_out` is given, writes the state after segment
-// nseg_out - 1 there. Bounded waits that give up set *error.
+// nseg_out - 1 there (and with `alpha_out` [b,H] the decay over segments
+// 0 .. nseg_out - 1). Bounded waits that give up set *error.
 int segment_max_tiles();
 cudaError_t launch_segment_states(const Dims& d, const CUtensorMap* maps, const float* dt,
                                   const float* A, float* segbuf, float* decay, int* error,
@@ -109,7 +110,7 @@ cudaError_t launch_segment_states(const Dims& d, const CUtensorMap* maps, const 
                                   cudaStream_t st);
 cudaError_t launch_segment_scan(const Dims& d, const float* init, float* segbuf, const float* decay,
                                 int nseg, int nslot, int nseg_out, float* final_out,
-                                cudaStream_t st);
+                                cudaStream_t st, float* alpha_out = nullptr);
 
 // Recurrent form for a few tokens per sequence, state [b,H,P,N] updated in place.
 struct StepLayout {

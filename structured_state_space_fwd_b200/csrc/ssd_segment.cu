@@ -403,23 +403,29 @@ done:
 
 // h_{s+1} = decay_s h_s + S_s over the segments, in place: slot s (s >= 1) holds
 // S_{s-1} on entry and the state entering segment s on exit.
+// With alpha_out, the thread of each (b, h)'s first vector also writes the product of
+// the decays of segments 0 .. nseg_out - 1 there: the decay over all of them.
 __global__ void segment_scan_kernel(const float* __restrict__ init, float* segbuf,
                                     const float* __restrict__ decay, int64_t nvec, int64_t H,
-                                    int64_t PN4, int nseg, int nslot, int nseg_out, float* final_out) {
+                                    int64_t PN4, int nseg, int nslot, int nseg_out, float* final_out,
+                                    float* alpha_out) {
     const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (e >= nvec) return;
     const int64_t bh = e / PN4, off = e % PN4;
     const int64_t bi = bh / H, h = bh % H;
     float4 cur = init ? reinterpret_cast<const float4*>(init)[bh * PN4 + off] : make_float4(0.f, 0.f, 0.f, 0.f);
     float4* sb = reinterpret_cast<float4*>(segbuf);
+    float prod = 1.f;
     for (int s = 1; s <= nseg_out; ++s) {
         const float f = __ldg(decay + (bi * nseg + s - 1) * H + h);
+        prod *= f;
         const int64_t idx = ((bi * nslot + s) * H + h) * PN4 + off;
         const float4 v = __ldcg(sb + idx);
         cur = make_float4(fmaf(f, cur.x, v.x), fmaf(f, cur.y, v.y), fmaf(f, cur.z, v.z), fmaf(f, cur.w, v.w));
         if (s < nslot) __stcg(sb + idx, cur);
     }
     if (final_out) reinterpret_cast<float4*>(final_out)[bh * PN4 + off] = cur;
+    if (alpha_out && off == 0) alpha_out[bh] = prod;
 }
 
 int sms_now() {
@@ -476,7 +482,7 @@ cudaError_t launch_segment_states(const Dims& d, const CUtensorMap* maps, const 
 }
 
 cudaError_t launch_segment_scan(const Dims& d, const float* init, float* segbuf, const float* decay, int nseg,
-                                int nslot, int nseg_out, float* final_out, cudaStream_t st) {
+                                int nslot, int nseg_out, float* final_out, cudaStream_t st, float* alpha_out) {
     if ((d.P * d.N) % 4 != 0) return cudaErrorInvalidValue;
     const int64_t PN4 = d.P * d.N / 4;
     const int64_t nvec = d.b * d.H * PN4;
@@ -485,7 +491,7 @@ cudaError_t launch_segment_scan(const Dims& d, const float* init, float* segbuf,
     const int64_t blocks = (nvec + threads - 1) / threads;
     if (blocks > INT32_MAX) return cudaErrorInvalidValue;
     segment_scan_kernel<<<(unsigned)blocks, threads, 0, st>>>(init, segbuf, decay, nvec, d.H, PN4, nseg, nslot,
-                                                              nseg_out, final_out);
+                                                              nseg_out, final_out, alpha_out);
     return cudaGetLastError();
 }
 
