@@ -456,14 +456,14 @@ def measure_varlen(ssd, dev, stream, steps, warmup, seed=0):
 
 # ------------------------------------------------------------------ forward + gate, fused
 GATED_METRIC = ("SSD fwd + gate + RMSNorm (per-head groups of 64) Mtokens/s at 2.7B layer shape, "
-                "gate fused into the forward's stores")
+                "gate in the forward's stores (fuse)")
 
 
 def measure_fwd_gated(ssd, dev, stream, steps, warmup, seed=0):
-    """ssd_fwd_gated at the 2.7B layer shape with norm groups of 64 channels (one head):
-    the single-pass kernel gates and normalises each row before storing it, so y never
-    reaches HBM. Timed beside the same work as two calls (ssd_fwd, then
-    ssd_gated_rmsnorm), which writes y and reads it back."""
+    """ssd_fwd_gated at the 2.7B layer shape with norm groups of 64 channels (one head),
+    both ways: fuse (the single-pass kernel gates and normalises each row before storing
+    it, so y never reaches HBM and needs no buffer) and separate (y through the
+    workspace, then the gate kernel)."""
     w = WORKLOAD
     inp = W.workload_inputs(w, seed=seed)
     d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
@@ -472,45 +472,40 @@ def measure_fwd_gated(ssd, dev, stream, steps, warmup, seed=0):
     nw = (torch.rand(w.nheads * w.headdim, generator=g) + 0.5).float().to(dev)
     gs = 64
     shp = ssd.make_shape(d["x"], d["B"], w.chunk_size)
-    ws = torch.empty(max(ssd.ssd_fwd_gated_workspace_size(shp, gs), ssd.ssd_fwd_workspace_size(shp), 1),
-                     dtype=torch.uint8, device=dev)
     out = torch.empty_like(d["x"])
-    y = torch.empty_like(d["x"])
     fin = torch.empty((w.batch, w.nheads, w.headdim, w.dstate), dtype=torch.float32, device=dev)
+    wss = {f: torch.empty(max(ssd.ssd_fwd_gated_workspace_size(shp, gs, f), 1), dtype=torch.uint8, device=dev)
+           for f in (True, False)}
 
-    def fused():
+    def run(f):
         ssd.ssd_fwd_gated(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], z=z, norm_weight=nw, group_size=gs,
-                          eps=1e-5, chunk_size=w.chunk_size, out=out, final_states=fin,
-                          return_final_states=True, workspace=ws, stream=stream)
+                          eps=1e-5, fuse=f, chunk_size=w.chunk_size, out=out, final_states=fin,
+                          return_final_states=True, workspace=wss[f], stream=stream)
 
-    def separate():
-        ssd.ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], chunk_size=w.chunk_size, y=y,
-                    final_states=fin, return_final_states=True, workspace=ws, stream=stream)
-        ssd.ssd_gated_rmsnorm(y, z, nw, group_size=gs, eps=1e-5, out=out, stream=stream)
-
-    def timed(fn):
+    def timed(f):
         for _ in range(warmup):
-            fn()
+            run(f)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(steps):
-            fn()
+            run(f)
         e1.record(stream)
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / steps
-    ms_f = timed(fused)
-    ms_s = timed(separate)
+    ms_f = timed(True)
+    ms_s = timed(False)
     _, by = alg_counts(w, with_final=True)
     by += 2.0 * w.batch * w.seqlen * w.nheads * w.headdim + 4.0 * w.nheads * w.headdim   # z, weight
     pk, pk_kind = peaks()
     ach = by / (ms_f / 1e3) / 1e9
+    ybytes = 2.0 * w.batch * w.seqlen * w.nheads * w.headdim
     return {"metric": GATED_METRIC, "value": w.tokens / (ms_f / 1e3) / 1e6, "unit": UNIT,
             "ms_per_step": ms_f, "steps": steps, "warmup": warmup, "dtype": "bf16",
             "config": {"workload": w.name, **w.shape_dict(), "group_size": gs, "eps": 1e-5,
                        "plan": ssd.ssd_fwd_plan(shp)[0]},
-            "separate_ms_per_step": ms_s, "saved_ms_per_step": ms_s - ms_f,
-            "y_round_trip_bytes_saved": 2.0 * 2.0 * w.batch * w.seqlen * w.nheads * w.headdim,
+            "separate_ms_per_step": ms_s, "fused_minus_separate_ms": ms_f - ms_s,
+            "y_round_trip_bytes_saved": 2.0 * ybytes, "y_buffer_bytes_saved": ybytes,
             "roofline": {"kernel": "ssd_fused_kernel (gated stores)", "bound": "hbm", "achieved": ach,
                          "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": ach / pk["hbm_gbs"],
                          "alg_bytes_per_step": by, "traffic": None, "peak_source": pk_kind},
@@ -654,12 +649,13 @@ def run_cp(args):
                            "slice_tokens": Ts, "exchange": "NCCL all-gather of per-rank records"
                            if world > 1 else "none (one rank)",
                            "l2": "per-rank slice inputs 34 MB + outputs; timed back to back"},
-                "roofline": {"kernel": "rank step (7 kernels + all-gather)", "bound": "hbm",
+                "roofline": {"kernel": f"rank step ({cp_kernels_per_step(ssd, d, w, rank)} kernels + all-gather)",
+                             "bound": "hbm",
                              "achieved": by / (ms / 1e3) / 1e9, "peak": pk["hbm_gbs"],
                              "unit": "GB/s", "frac": by / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
                              "traffic": None, "alg_bytes_per_rank_step": by,
                              "peak_source": pk_kind + " (burst copy, MEASURED_PEAKS hbm_gbs)"},
-                "gpu_launches": 7 * args.steps, "clocks": clk}
+                "gpu_launches": cp_kernels_per_step(ssd, d, w, rank) * args.steps, "clocks": clk}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

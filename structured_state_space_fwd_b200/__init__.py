@@ -112,20 +112,21 @@ def check_cu_seqlens(cu_seqlens, T: int) -> list[int]:
     return cu
 
 
-def ssd_fwd_gated_workspace_size(shape: ShapeT, group_size: int) -> int:
+def ssd_fwd_gated_workspace_size(shape: ShapeT, group_size: int, fuse: bool = True) -> int:
     n = ctypes.c_size_t(0)
-    check(lib().ssd_fwd_gated_workspace_size(ctypes.byref(shape), ctypes.c_int64(group_size), ctypes.byref(n)),
-          "ssd_fwd_gated_workspace_size")
+    check(lib().ssd_fwd_gated_workspace_size(ctypes.byref(shape), ctypes.c_int64(group_size), ctypes.c_int(int(fuse)),
+                                             ctypes.byref(n)), "ssd_fwd_gated_workspace_size")
     return int(n.value)
 
 
 def ssd_fwd_gated(x, dt, A, B, C, D=None, z=None, norm_weight=None, group_size: int = 64,
-                  eps: float = 1e-5, chunk_size: int = 256, initial_states=None,
+                  eps: float = 1e-5, fuse: bool = True, chunk_size: int = 256, initial_states=None,
                   return_final_states: bool = False, out=None, final_states=None, workspace=None,
                   stream=None):
     """The forward, then y * SiLU(z) RMS-normalised over channel groups times norm_weight
-    (Knowl 6), without storing y when the single-pass kernel can apply the gate (groups
-    of 8, 16, 32 or 64 channels). Returns out, or (out, final_states)."""
+    (Knowl 6). With fuse, y is never stored when the single-pass kernel can apply the gate
+    (groups of 8, 16, 32 or 64 channels); otherwise y passes through the workspace.
+    Returns out, or (out, final_states)."""
     _need(x, "x")
     _need(z, "z", x.dtype)
     _need(norm_weight, "norm_weight", torch.float32)
@@ -135,12 +136,13 @@ def ssd_fwd_gated(x, dt, A, B, C, D=None, z=None, norm_weight=None, group_size: 
     if final_states is None and return_final_states:
         final_states = torch.empty((x.shape[0], x.shape[2], x.shape[3], B.shape[3]),
                                    dtype=torch.float32, device=x.device)
-    nbytes = ssd_fwd_gated_workspace_size(shape, group_size)
+    nbytes = ssd_fwd_gated_workspace_size(shape, group_size, fuse)
     if workspace is None or workspace.numel() < nbytes:
         workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=x.device)
     check(lib().ssd_fwd_gated(ctypes.byref(shape), _p(x), _p(dt), _p(A), _p(B), _p(C), _p(D),
                               _p(initial_states), _p(z), _p(norm_weight), ctypes.c_int64(group_size),
-                              ctypes.c_float(eps), _p(out), _p(final_states), _p(workspace),
+                              ctypes.c_float(eps), ctypes.c_int(int(fuse)), _p(out), _p(final_states),
+                              _p(workspace),
                               ctypes.c_size_t(nbytes), _stream(stream)), "ssd_fwd_gated")
     return (out, final_states) if return_final_states else out
 

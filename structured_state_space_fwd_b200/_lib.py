@@ -53,9 +53,9 @@ _SIGS = {
                        + [ctypes.c_size_t, _VP], ctypes.c_int),
     "ssd_fwd_varlen_check": ([ctypes.POINTER(ShapeT), ctypes.c_int64, _VP, ctypes.c_size_t, _VP],
                              ctypes.c_int),
-    "ssd_fwd_gated_workspace_size": ([ctypes.POINTER(ShapeT), ctypes.c_int64,
+    "ssd_fwd_gated_workspace_size": ([ctypes.POINTER(ShapeT), ctypes.c_int64, ctypes.c_int,
                                       ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
-    "ssd_fwd_gated": ([ctypes.POINTER(ShapeT)] + [_VP] * 9 + [ctypes.c_int64, ctypes.c_float]
+    "ssd_fwd_gated": ([ctypes.POINTER(ShapeT)] + [_VP] * 9 + [ctypes.c_int64, ctypes.c_float, ctypes.c_int]
                       + [_VP] * 3 + [ctypes.c_size_t, _VP], ctypes.c_int),
     "ssd_step": ([ctypes.POINTER(ShapeT)] + [_VP] * 9, ctypes.c_int),
     "ssd_cp_record_floats": ([ctypes.POINTER(ShapeT), ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),

@@ -607,32 +607,33 @@ ssd_status_t ssd_fwd(const ssd_shape_t* shape, const void* x, const float* dt, c
                    workspace, (cudaStream_t)stream);
 }
 
-// Forward plus the gate and norm of the block: the single-pass kernel applies them
-// in its stores when the plan is single-pass and the groups lie inside a head;
-// otherwise y goes to the workspace and the separate gate kernel follows.
-bool gated_fuses(const ssd::Dims& d, int64_t group_size) {
+// Forward plus the gate and norm of the block: with `fuse`, the single-pass kernel
+// applies them in its stores when the plan is single-pass and the groups lie inside
+// a head; otherwise y goes to the workspace and the separate gate kernel follows.
+bool gated_fuses(const ssd::Dims& d, int64_t group_size, int fuse) {
     const Path p = pick_path(d);
-    return (p == Path::Fused || p == Path::Segmented) && ssd::fused_gate_ok(group_size);
+    return fuse && (p == Path::Fused || p == Path::Segmented) && ssd::fused_gate_ok(group_size);
 }
 
-ssd_status_t ssd_fwd_gated_workspace_size(const ssd_shape_t* shape, int64_t group_size, size_t* bytes) {
+ssd_status_t ssd_fwd_gated_workspace_size(const ssd_shape_t* shape, int64_t group_size, int fuse,
+                                          size_t* bytes) {
     if (!bytes) return SSD_ERR_INVALID_ARG;
     ssd_status_t st = check_shape(shape);
     if (st != SSD_OK) return st;
     const ssd::Dims d = ssd::make_dims(*shape);
     if (group_size < 1 || (d.H * d.P) % group_size != 0) return SSD_ERR_INVALID_ARG;
     const size_t fw = fwd_workspace(d).total;
-    *bytes = gated_fuses(d, group_size) ? fw : align_up(fw, 256) + sizes_of(d).x;
+    *bytes = gated_fuses(d, group_size, fuse) ? fw : align_up(fw, 256) + sizes_of(d).x;
     return SSD_OK;
 }
 
 ssd_status_t ssd_fwd_gated(const ssd_shape_t* shape, const void* x, const float* dt, const float* A,
                            const void* B, const void* C, const float* D, const float* initial_states,
                            const void* z, const float* norm_weight, int64_t group_size, float eps,
-                           void* out, float* final_states, void* workspace, size_t workspace_bytes,
-                           void* stream) {
+                           int fuse, void* out, float* final_states, void* workspace,
+                           size_t workspace_bytes, void* stream) {
     size_t need = 0;
-    ssd_status_t st = ssd_fwd_gated_workspace_size(shape, group_size, &need);
+    ssd_status_t st = ssd_fwd_gated_workspace_size(shape, group_size, fuse, &need);
     if (st != SSD_OK) return st;
     if (workspace_bytes < need || !(eps >= 0.f) || !std::isfinite(eps)) return SSD_ERR_INVALID_ARG;
     const ssd::Dims d = ssd::make_dims(*shape);
@@ -643,7 +644,7 @@ ssd_status_t ssd_fwd_gated(const ssd_shape_t* shape, const void* x, const float*
         if (overlaps(r, Range{out, z0.x}) || overlaps(r, Range{final_states, final_states ? z0.st : 0}) ||
             overlaps(r, Range{workspace, need}))
             return SSD_ERR_INVALID_ARG;
-    if (gated_fuses(d, group_size)) {
+    if (gated_fuses(d, group_size, fuse)) {
         // out takes y's place: every check of ssd_fwd applies to it
         if ((st = check_fwd_args(shape, x, dt, A, B, C, D, initial_states, out, final_states, workspace,
                                  workspace_bytes)) != SSD_OK)

@@ -354,8 +354,17 @@ __device__ __forceinline__ void mma_tokens_tmem(uint32_t d, uint32_t a, uint64_t
         mma_bf16_tmem_a(d, a + 8 * kk, dB + (uint64_t)(kk * 128), idesc, 1u);
 }
 
-// One group size's pass of gate_row below (v recomputed for the scaling rather than
-// held, to stay inside the registers).
+// SiLU(z) = z sigmoid(z) = z (1 + tanh(z / 2)) / 2: one special-function
+// instruction (tanh.approx, a relative error near 2^-11, under the bf16 output's
+// rounding).
+__device__ __forceinline__ float silu_fast(float z) {
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * z));
+    return 0.5f * z * (1.f + t);
+}
+
+// One group size's pass of gate_row below: v is held in registers between the sum
+// of squares and the scaling for groups of up to 32 channels, recomputed for 64.
 template <int GC>   // 16-byte chunks (8 channels) per group
 __device__ __forceinline__ void gate_row_g(const uint4 (&zv)[8], const float* w, float eps, uint8_t* stg, int r) {
     constexpr float kInvGs = 1.f / (8 * GC);
@@ -366,25 +375,35 @@ __device__ __forceinline__ void gate_row_g(const uint4 (&zv)[8], const float* w,
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const float2 y2 = unpack_bf16(ys4[k]), z2 = unpack_bf16(zs4[k]);
-            v[2 * k] = y2.x * __fdividef(z2.x, 1.f + ex2(-z2.x * kLog2e));
-            v[2 * k + 1] = y2.y * __fdividef(z2.y, 1.f + ex2(-z2.y * kLog2e));
+            v[2 * k] = y2.x * silu_fast(z2.x);
+            v[2 * k + 1] = y2.y * silu_fast(z2.y);
         }
     };
 #pragma unroll
     for (int c0 = 0; c0 < 8; c0 += GC) {
+        constexpr int kHold = GC <= 4 ? GC : 1;   // chunks whose v stays in registers
+        float vh[kHold][8];
         float ss = 0.f;
 #pragma unroll
         for (int c = c0; c < c0 + GC; ++c) {
             float v[8];
             gated(c, v);
 #pragma unroll
-            for (int k = 0; k < 8; ++k) ss = fmaf(v[k], v[k], ss);
+            for (int k = 0; k < 8; ++k) {
+                ss = fmaf(v[k], v[k], ss);
+                if (GC <= 4) vh[(c - c0) % kHold][k] = v[k];
+            }
         }
         const float inv = rsqrtf(ss * kInvGs + eps);
 #pragma unroll
         for (int c = c0; c < c0 + GC; ++c) {
             float v[8];
-            gated(c, v);
+            if (GC <= 4) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) v[k] = vh[(c - c0) % kHold][k];
+            } else {
+                gated(c, v);
+            }
             const float4 w0 = __ldg(reinterpret_cast<const float4*>(w + 8 * c));
             const float4 w1 = __ldg(reinterpret_cast<const float4*>(w + 8 * c + 4));
             const float wk[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
@@ -400,12 +419,12 @@ __device__ __forceinline__ void gate_row_g(const uint4 (&zv)[8], const float* w,
 // 128-byte-swizzled staging row r), in place: v = y * SiLU(z), then each group
 // of gs channels is divided by sqrt(mean(v^2) + eps) and scaled by the weight.
 // y is the bf16 value a separate pass would read back. zrow indexes [b,T,H] of z.
-__device__ __forceinline__ void gate_row(const __nv_bfloat16* z, const float* nw, int gs, float eps, uint8_t* stg,
+__device__ __noinline__ void gate_row(const __nv_bfloat16* z, const float* nw, int gs, float eps, uint8_t* stg,
                                      int r, int64_t zrow, int hh) {
     const uint4* zp = reinterpret_cast<const uint4*>(z + zrow * kP);
     uint4 zv[8];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) zv[c] = __ldcs(zp + c);   // read once: streamed past L1
+    for (int c = 0; c < 8; ++c) zv[c] = __ldg(zp + c);    // each 32-byte sector over two loads: via L1
     const float* w = nw + (int64_t)hh * kP;
     switch (gs) {
         case 8: gate_row_g<1>(zv, w, eps, stg, r); break;

@@ -9,7 +9,7 @@
 //     out_c = v_c / sqrt(mean_group(v^2) + eps) * weight_c
 //
 // HBM-bound: y and z are read once and out written once (6 bytes per channel
-// in bf16). A group is handled by TPG threads (32..256) of a 256-thread CTA;
+// in bf16). A group is handled by TPG threads (4..256) of a 256-thread CTA;
 // each thread keeps up to kMaxVec 16-byte vectors of v in registers between
 // the sum of squares and the scaled write, and groups larger than that are
 // re-read (from L2) for the write.
@@ -107,9 +107,10 @@ __global__ void __launch_bounds__(kGateThreads, 5) gated_rmsnorm_kernel(
 #pragma unroll
         for (int e = 0; e < VW; ++e) ss = fmaf(g[e], g[e], ss);
     }
-    // sum over the group's threads: within the warp, then across its warps
+        // sum over the group's threads: within the warp (or the group's lanes of it, which
+    // are aligned), then across its warps
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    for (int off = (TPG < 32 ? TPG : 32) / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
     if constexpr (WPG > 1) {
         if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
         __syncthreads();
@@ -145,13 +146,17 @@ cudaError_t launch_gate_vw(const E* y, const E* z, const float* w, E* out, int64
                            int64_t gs, float eps, cudaStream_t st) {
     const int64_t nvec = gs / VW;
     const int64_t groups = rows * (C / gs);
-    // threads per group: enough for kMaxVec vectors each, at least a warp
-    int tpg = 32;
+    // threads per group: enough for kMaxVec vectors each, at least 4 (a small group
+    // shares its warp with others rather than leaving lanes idle)
+    int tpg = 4;
     while (tpg < kGateThreads && (int64_t)tpg * kMaxVec < nvec) tpg <<= 1;
     const int64_t gpb = kGateThreads / tpg;
     const unsigned grid = (unsigned)((groups + gpb - 1) / gpb);
     const int64_t gpr = C / gs;
     switch (tpg) {
+        case 4: gated_rmsnorm_kernel<E, VW, 4><<<grid, kGateThreads, 0, st>>>(y, z, w, out, groups, gpr, gs, eps); break;
+        case 8: gated_rmsnorm_kernel<E, VW, 8><<<grid, kGateThreads, 0, st>>>(y, z, w, out, groups, gpr, gs, eps); break;
+        case 16: gated_rmsnorm_kernel<E, VW, 16><<<grid, kGateThreads, 0, st>>>(y, z, w, out, groups, gpr, gs, eps); break;
         case 32: gated_rmsnorm_kernel<E, VW, 32><<<grid, kGateThreads, 0, st>>>(y, z, w, out, groups, gpr, gs, eps); break;
         case 64: gated_rmsnorm_kernel<E, VW, 64><<<grid, kGateThreads, 0, st>>>(y, z, w, out, groups, gpr, gs, eps); break;
         case 128: gated_rmsnorm_kernel<E, VW, 128><<<grid, kGateThreads, 0, st>>>(y, z, w, out, groups, gpr, gs, eps); break;

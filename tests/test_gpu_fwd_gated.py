@@ -1,6 +1,7 @@
 """ssd_fwd_gated: the forward followed by the gate and RMSNorm of the Mamba-2 block
 (Knowl 6, step 4). Groups inside a head (8..64 channels) are applied in the
-single-pass kernel's stores; others go through the workspace.
+single-pass kernel's stores when the caller asks for it (fuse); others, and every
+case without fuse, go through the workspace and the gate kernel.
 
 Two bars:
   * the gate's own arithmetic: out against the fp64 oracle's gated_rmsnorm of the
@@ -41,7 +42,7 @@ def gate_inputs(b, T, H, P, seed):
     return z, w
 
 
-def run_case(ssd, monkeypatch, b, T, H, G, N, gs, seed, path=None, scale=None, eps=1e-5):
+def run_case(ssd, monkeypatch, b, T, H, G, N, gs, seed, path=None, scale=None, eps=1e-5, fuse=True):
     if path is None:
         monkeypatch.delenv("SSD_PATH", raising=False)
     else:
@@ -52,7 +53,7 @@ def run_case(ssd, monkeypatch, b, T, H, G, N, gs, seed, path=None, scale=None, e
     z, w = gate_inputs(b, T, H, 64, seed + 1)
     d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
     out, fin = ssd.ssd_fwd_gated(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], z=z.cuda(),
-                                 norm_weight=w.cuda(), group_size=gs, eps=eps,
+                                 norm_weight=w.cuda(), group_size=gs, eps=eps, fuse=fuse,
                                  initial_states=d["initial_states"], return_final_states=True)
     torch.cuda.synchronize()
     y_ref, f_ref, _ = oracle.recurrence(**inp)
@@ -89,9 +90,10 @@ def check_gate(oc, y_dev, y_ref, z, w, gs, eps):
     assert worst <= 1.0, f"composition: a group's error is {worst:.2f} of its bound"
 
 
+@pytest.mark.parametrize("fuse", [True, False])
 @pytest.mark.parametrize("gs", [8, 16, 32, 64])
-def test_fused_gate_groups_in_a_head(ssd, monkeypatch, gs):
-    plan = run_case(ssd, monkeypatch, 2, 700, 8, 2, 128, gs, seed=gs)
+def test_fused_gate_groups_in_a_head(ssd, monkeypatch, gs, fuse):
+    plan = run_case(ssd, monkeypatch, 2, 700, 8, 2, 128, gs, seed=gs, fuse=fuse)
     assert plan == "fused"
 
 
@@ -124,7 +126,7 @@ def test_fused_gate_full_size(ssd, monkeypatch):
     z, w = gate_inputs(w_.batch, w_.seqlen, w_.nheads, w_.headdim, 5)
     d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
     out = ssd.ssd_fwd_gated(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], z=z.cuda(), norm_weight=w.cuda(),
-                            group_size=64, eps=1e-5, initial_states=d["initial_states"])
+                            group_size=64, eps=1e-5, fuse=True, initial_states=d["initial_states"])
     torch.cuda.synchronize()
     y = ssd.ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], initial_states=d["initial_states"])
     torch.cuda.synchronize()
