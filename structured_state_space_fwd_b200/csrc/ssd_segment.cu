@@ -128,6 +128,32 @@ __device__ __forceinline__ SUnit sdecode(const SParams& p, int u) {
     return r;
 }
 
+// w o x in place for x tile nx (its slot's weights from the decay-weight warp),
+// row j by this thread; false if a wait gave up.
+template <int NS>
+__device__ __forceinline__ bool scale_x_ns(uint8_t* smem, SBars* bs, int* err, int nx, int j) {
+    using K = SCfg<NS>;
+    const int xs = nx % K::kXSlots;
+    if (!swait_all(&bs->x_full[xs], (nx / K::kXSlots) & 1, bs, err)) return false;
+    if (!swait_all(&bs->w_full[xs], (nx / K::kXSlots) & 1, bs, err)) return false;
+    const float w = reinterpret_cast<const float*>(smem + K::kOffW + xs * kTile * 4)[j];
+    mbar_arrive(&bs->w_empty[xs]);
+    const float2 w2 = make_float2(w, w);
+    uint8_t* sx = smem + K::kOffX + xs * kAtom;
+#pragma unroll
+    for (int c8 = 0; c8 < 8; ++c8) {
+        const uint32_t off = sw128_off(j, c8);
+        const uint4 xv = *reinterpret_cast<const uint4*>(sx + off);
+        float2 a = __fmul2_rn(w2, unpack2(xv.x)), b = __fmul2_rn(w2, unpack2(xv.y));
+        float2 c = __fmul2_rn(w2, unpack2(xv.z)), d = __fmul2_rn(w2, unpack2(xv.w));
+        *reinterpret_cast<uint4*>(sx + off) =
+            make_uint4(pack2(a.x, a.y), pack2(b.x, b.y), pack2(c.x, c.y), pack2(d.x, d.y));
+    }
+    fence_proxy_async_smem();
+    mbar_arrive(&bs->wx_full[xs]);
+    return true;
+}
+
 template <int NS>
 __global__ void __launch_bounds__(kThreads, 1)
     segment_state_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_B,
@@ -165,6 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool misaligned = (smem_u32(smem) & 1023u) != 0;
     const uint32_t tmem = bs->tmem;
     const int kh = prm.kheads;
+    auto scale_x = [](uint8_t* sm, SBars* b, int* e, int n, int row) { return scale_x_ns<NS>(sm, b, e, n, row); };
     const int H = prm.H;
     const int64_t T = prm.T;
     const int natoms = (prm.N + 63) / 64;
@@ -332,32 +359,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp >= 4 && warp < 8) {
         // ---------------------------------------------------------------- scale group
+        // w o x in place for the even x tiles (the epilogue warps take the odd ones)
         const int j = tid - 128;
         int nx = 0;
         for (int u = blockIdx.x; u < prm.nunits; u += gridDim.x) {
             const SUnit U = sdecode(prm, u);
-            for (int t = U.t_begin; t < U.t_end; ++t) {
-                for (int k = 0; k < kh; ++k, ++nx) {
-                    const int xs = nx % K::kXSlots;
-                    if (!swait_all(&bs->x_full[xs], (nx / K::kXSlots) & 1, bs, err)) goto done;
-                    if (!swait_all(&bs->w_full[xs], (nx / K::kXSlots) & 1, bs, err)) goto done;
-                    const float w = reinterpret_cast<const float*>(smem + K::kOffW + xs * kTile * 4)[j];
-                    mbar_arrive(&bs->w_empty[xs]);
-                    const float2 w2 = make_float2(w, w);
-                    uint8_t* sx = smem + K::kOffX + xs * kAtom;
-#pragma unroll
-                    for (int c8 = 0; c8 < 8; ++c8) {
-                        const uint32_t off = sw128_off(j, c8);
-                        const uint4 xv = *reinterpret_cast<const uint4*>(sx + off);
-                        float2 a = __fmul2_rn(w2, unpack2(xv.x)), b = __fmul2_rn(w2, unpack2(xv.y));
-                        float2 c = __fmul2_rn(w2, unpack2(xv.z)), d = __fmul2_rn(w2, unpack2(xv.w));
-                        *reinterpret_cast<uint4*>(sx + off) =
-                            make_uint4(pack2(a.x, a.y), pack2(b.x, b.y), pack2(c.x, c.y), pack2(d.x, d.y));
-                    }
-                    fence_proxy_async_smem();
-                    mbar_arrive(&bs->wx_full[xs]);
-                }
-            }
+            for (int t = U.t_begin; t < U.t_end; ++t)
+                for (int k = 0; k < kh; ++k, ++nx)
+                    if (!(nx & 1) && !scale_x(smem, bs, err, nx, j)) goto done;
         }
     } else if (warp >= 8) {
         // ---------------------------------------------------------------- epilogue
@@ -367,9 +376,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lb = (uint32_t)(q * 32) << 16;
         const int N = prm.N;
         const int64_t PN = (int64_t)kP * N;
-        int nu = 0;
+        int nu = 0, nx = 0;
         for (int u = blockIdx.x; u < prm.nunits; u += gridDim.x, ++nu) {
             const SUnit U = sdecode(prm, u);
+            // first this unit's odd x tiles (every product of the unit needs them)
+            for (int t = U.t_begin; t < U.t_end; ++t)
+                for (int k = 0; k < kh; ++k, ++nx)
+                    if ((nx & 1) && !scale_x(smem, bs, err, nx, r)) goto done;
             const int ab = nu % K::kAccBufs;
             if (!swait_all(&bs->acc_full[ab], (nu / K::kAccBufs) & 1, bs, err)) goto done;
             tc_fence_after();
@@ -402,27 +415,50 @@ done:
 }
 
 // h_{s+1} = decay_s h_s + S_s over the segments, in place: slot s (s >= 1) holds
-// S_{s-1} on entry and the state entering segment s on exit.
-// With alpha_out, the thread of each (b, h)'s first vector also writes the product of
-// the decays of segments 0 .. nseg_out - 1 there: the decay over all of them.
-__global__ void segment_scan_kernel(const float* __restrict__ init, float* segbuf,
+// S_{s-1} on entry and the state entering segment s on exit. With alpha_out, the
+// thread of each (b, h)'s first vector also writes the product of the decays of
+// segments 0 .. nseg_out - 1 there: the decay over all of them. The walk over the
+// segments is a dependent chain of FMAs; the loads of the next kScanAhead slots are
+// in flight while it runs.
+constexpr int kScanAhead = 4;
+__global__ void segment_scan_kernel(const float* __restrict__ init, float* __restrict__ segbuf,
                                     const float* __restrict__ decay, int64_t nvec, int64_t H,
-                                    int64_t PN4, int nseg, int nslot, int nseg_out, float* final_out,
-                                    float* alpha_out) {
+                                    int64_t PN4, int nseg, int nslot, int nseg_out, float* __restrict__ final_out,
+                                    float* __restrict__ alpha_out) {
     const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (e >= nvec) return;
     const int64_t bh = e / PN4, off = e % PN4;
     const int64_t bi = bh / H, h = bh % H;
     float4 cur = init ? reinterpret_cast<const float4*>(init)[bh * PN4 + off] : make_float4(0.f, 0.f, 0.f, 0.f);
     float4* sb = reinterpret_cast<float4*>(segbuf);
+    auto slot = [&](int s) { return ((bi * nslot + s) * H + h) * PN4 + off; };
+    float4 ring[kScanAhead];
+    float fr[kScanAhead];
+#pragma unroll
+    for (int k = 0; k < kScanAhead; ++k) {
+        const int s = 1 + k;
+        if (s <= nseg_out) {
+            ring[k] = __ldcg(sb + slot(s));
+            fr[k] = __ldg(decay + (bi * nseg + s - 1) * H + h);
+        }
+    }
     float prod = 1.f;
-    for (int s = 1; s <= nseg_out; ++s) {
-        const float f = __ldg(decay + (bi * nseg + s - 1) * H + h);
-        prod *= f;
-        const int64_t idx = ((bi * nslot + s) * H + h) * PN4 + off;
-        const float4 v = __ldcg(sb + idx);
-        cur = make_float4(fmaf(f, cur.x, v.x), fmaf(f, cur.y, v.y), fmaf(f, cur.z, v.z), fmaf(f, cur.w, v.w));
-        if (s < nslot) __stcg(sb + idx, cur);
+    for (int s0 = 1; s0 <= nseg_out; s0 += kScanAhead) {
+#pragma unroll
+        for (int k = 0; k < kScanAhead; ++k) {
+            const int s = s0 + k;
+            if (s > nseg_out) break;
+            const float f = fr[k];
+            const float4 v = ring[k];
+            const int sn = s + kScanAhead;   // refill this ring entry with slot sn
+            if (sn <= nseg_out) {
+                ring[k] = __ldcg(sb + slot(sn));
+                fr[k] = __ldg(decay + (bi * nseg + sn - 1) * H + h);
+            }
+            prod *= f;
+            cur = make_float4(fmaf(f, cur.x, v.x), fmaf(f, cur.y, v.y), fmaf(f, cur.z, v.z), fmaf(f, cur.w, v.w));
+            if (s < nslot) __stcg(sb + slot(s), cur);
+        }
     }
     if (final_out) reinterpret_cast<float4*>(final_out)[bh * PN4 + off] = cur;
     if (alpha_out && off == 0) alpha_out[bh] = prod;
