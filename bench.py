@@ -540,12 +540,13 @@ def cp_setup(ssd, dev, w, nranks, rank, seed=0):
 
 def cp_kernels_per_step(ssd, d, w, rank):
     """Launches of one rank's ssd_cp_begin + ssd_cp_end: on the single-pass plan the
-    segment-state pass and its scan, the fold (ranks > 0) and the slice's forward;
-    otherwise chunk cumsum, chunk states, state passing and the slice decay, then the
-    fold, state passing and the chunk scan."""
-    path, nk = ssd.ssd_fwd_plan(ssd.make_shape(d["x"], d["B"], w.chunk_size))
+    segment-state pass and its scan, then the fold (ranks > 0), the scan from the
+    entering state and the single-pass kernel over the slice's segments; otherwise
+    chunk cumsum, chunk states, state passing and the slice decay, then the fold,
+    state passing and the chunk scan (slices of several segments assumed)."""
+    path, _ = ssd.ssd_fwd_plan(ssd.make_shape(d["x"], d["B"], w.chunk_size))
     fold = 1 if rank > 0 else 0
-    return 2 + fold + nk if path in ("fused", "segmented") else 4 + fold + 2
+    return 2 + fold + 2 if path in ("fused", "segmented") else 4 + fold + 2
 
 
 def measure_cp_slice(ssd, dev, stream, steps, warmup, nranks=8):

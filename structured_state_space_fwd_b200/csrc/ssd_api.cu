@@ -360,12 +360,13 @@ ssd_status_t read_device_status(const ssd::Dims& d, const void* workspace, cudaS
 }
 
 // Sequence-parallel workspace. Shapes the single-pass kernel takes: ssd_cp_begin
-// runs the segment-state pass over the slice and its scan (the record is the state
-// after the last segment, and the product of the segment decays) and keeps A for
-// ssd_cp_end, which folds the records into the entering state and runs the forward
-// from it:
-//   [A | status words | segment states [b, nseg+1, H, P, N] | segment decays [b, nseg, H]]
-//   with, after A, [entering state h_in | forward workspace] overlapping (end).
+// runs the segment-state pass over the slice and a scan that only reads it (the
+// record is the state after the last segment and the product of the segment
+// decays), and keeps A; ssd_cp_end folds the records into the entering state, scans
+// the same segment states from it (the states entering every segment) and runs the
+// single-pass kernel over the segments side by side:
+//   [A | status words | segment states [b, nseg+1, H, P, N] | segment decays [b, nseg, H]
+//    | entering state h_in | the kernel's ticket, status and flags].
 // Other shapes (step paths; begin leaves cs and S for end):
 //   [cs | chunk states S | entry states | entering state h_in].
 // Regions are 256-byte aligned.
@@ -373,7 +374,7 @@ struct CpWorkspace {
     bool single_pass;
     int kh, seg_tiles, nseg;                  // single pass: the segment-state pass
     size_t off_sync, off_seg, off_decay;      // single pass, begin
-    size_t off_A, off_fwd;                    // single pass: A kept by begin; end (h_in at off_hin)
+    size_t off_A, off_fwd;                    // single pass: A kept by begin; the kernel's sync ints (end)
     size_t off_cs, off_S, off_entry, off_hin, total;
 };
 CpWorkspace cp_workspace(const ssd::Dims& d) {
@@ -392,11 +393,9 @@ CpWorkspace cp_workspace(const ssd::Dims& d) {
         w.off_sync = align_up(z.hv, 256);
         w.off_seg = w.off_sync + 256;
         w.off_decay = w.off_seg + align_up(z.st * (size_t)(w.nseg + 1), 256);
-        const size_t begin_total = w.off_decay + align_up((size_t)(d.b * d.H * w.nseg) * 4, 256);
-        w.off_hin = w.off_sync;
+        w.off_hin = w.off_decay + align_up((size_t)(d.b * d.H * w.nseg) * 4, 256);
         w.off_fwd = w.off_hin + align_up(z.st, 256);
-        const size_t end_total = w.off_fwd + align_up(fwd_workspace(d).total, 256);
-        w.total = std::max(begin_total, end_total);
+        w.total = w.off_fwd + align_up(sizeof(int) * ssd::fused_sync_ints(d, w.nseg), 256);
     } else {
         w.off_cs = 0;
         w.off_S = align_up(z.cs, 256);
@@ -999,8 +998,9 @@ ssd_status_t ssd_cp_begin(const ssd_shape_t* shape, const void* x, const float* 
                               ssd::launch_segment_states(d, maps, dt, A, segbuf, decay, sync + 1, w.seg_tiles,
                                                          w.nseg, nslot, w.nseg, w.kh, s))) != SSD_OK)
             return st;
+        // the slots keep the states from zero: ssd_cp_end scans them again from h_in
         return cuda_status("segment scan", ssd::launch_segment_scan(d, initial_states, segbuf, decay, w.nseg,
-                                                                    nslot, w.nseg, record, s, alpha));
+                                                                    nslot, w.nseg, record, s, alpha, false));
     }
     float* cs = (float*)(ws + w.off_cs);
     float* S = (float*)(ws + w.off_S);
@@ -1060,8 +1060,43 @@ ssd_status_t ssd_cp_end(const ssd_shape_t* shape, int nranks, int rank, const fl
     }
     if (d.T == 0)
         return cuda_status("final states", ssd::launch_copy_or_zero_states(d, h_in, final_states, s));
-    if (w.single_pass)
-        return run_fwd(d, x, dt, (const float*)(ws + w.off_A), B, C, D, h_in, y, final_states, ws + w.off_fwd, s);
+    if (w.single_pass) {
+        // the states entering segments 1.. from h_in, over the segment states begin left,
+        // then every segment of the slice at once
+        float* segbuf = (float*)(ws + w.off_seg);
+        const float* decay = (const float*)(ws + w.off_decay);
+        const int nslot = w.nseg + 1;
+        if (w.nseg > 1 &&
+            (st = cuda_status("segment scan", ssd::launch_segment_scan(d, h_in, segbuf, decay, w.nseg, nslot,
+                                                                       w.nseg - 1, nullptr, s))) != SSD_OK)
+            return st;
+        CUtensorMap maps[4];
+        if (!ssd::make_tc_maps(d, x, B, C, y, maps)) {
+            ssd::set_error_detail("tensor map encoding failed");
+            return SSD_ERR_CUDA;
+        }
+        int* sync = (int*)(ws + w.off_fwd);
+        if ((st = cuda_status("sync area", cudaMemsetAsync(sync, 0, sizeof(int) * ssd::fused_sync_ints(d, w.nseg),
+                                                           s))) != SSD_OK)
+            return st;
+        ssd::FusedLaunch a = {};
+        a.d = d;
+        a.maps = maps;
+        a.dt = dt;
+        a.A = (const float*)(ws + w.off_A);
+        a.D = D;
+        a.init = h_in;
+        a.finalbuf = final_states;
+        a.segbuf = w.nseg > 1 ? segbuf : nullptr;
+        a.sync_ints = sync;
+        a.kheads = ssd::fused_kheads(d.H, d.G, ssd::fused_state_capacity(d.N));
+        a.seg_tiles = w.seg_tiles;
+        a.nseg = w.nseg;
+        a.nslot = nslot;
+        a.chained = 0;
+        a.y = y;
+        return cuda_status("fused forward", ssd::launch_fused(a, s));
+    }
     const float* cs = (const float*)(ws + w.off_cs);
     const float* S = (const float*)(ws + w.off_S);
     float* entry = (float*)(ws + w.off_entry);

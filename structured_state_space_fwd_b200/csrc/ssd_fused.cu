@@ -138,6 +138,7 @@ struct Params {
     const int* order;     // packed documents: unit order (documents, longest first)
     int64_t T;
     int H, G, N, kheads, batch, nunits, ntiles, seg_tiles, nseg;
+    int nslot;            // segbuf slots per batch row (nseg, or more)
     int chained;          // entering states come from the previous segment's unit
     int stall;            // test builds only: chain flags awaited at a value never reached
 };
@@ -305,14 +306,14 @@ __device__ __forceinline__ int64_t flag_index(const Params& p, int b, int s, int
 __device__ __forceinline__ const float* entry_src(const Params& p, const Unit& U, int h) {
     const int64_t PN = (int64_t)kP * p.N;
     if (U.s == 0) return p.init ? p.init + ((int64_t)U.doc * p.H + h) * PN : nullptr;
-    return p.segbuf + (((int64_t)U.b * p.nseg + U.s) * p.H + h) * PN;
+    return p.segbuf + (((int64_t)U.b * p.nslot + U.s) * p.H + h) * PN;
 }
 // where the state leaving the unit goes for head h (null: nowhere)
 __device__ __forceinline__ float* exit_dst(const Params& p, const Unit& U, int h) {
     const int64_t PN = (int64_t)kP * p.N;
     if (U.s == p.nseg - 1) return p.finalbuf ? p.finalbuf + ((int64_t)U.doc * p.H + h) * PN : nullptr;
     if (!p.chained) return nullptr;
-    return p.segbuf + (((int64_t)U.b * p.nseg + U.s + 1) * p.H + h) * PN;
+    return p.segbuf + (((int64_t)U.b * p.nslot + U.s + 1) * p.H + h) * PN;
 }
 
 // Byte offset of row `row`, 16-byte chunk `c` in a 128-byte-swizzled tile.
@@ -1293,6 +1294,8 @@ cudaError_t launch_fused(const FusedLaunch& a, cudaStream_t st) {
     prm.ntiles = (int)ntiles;
     prm.seg_tiles = a.seg_tiles;
     prm.nseg = a.nseg;
+    prm.nslot = a.nslot > 0 ? a.nslot : a.nseg;
+    if (prm.nslot < a.nseg) return cudaErrorInvalidValue;
     prm.chained = a.chained;
     prm.stall = a.stall;
     if (a.z) return ns == 128 ? launch_ns<128, true>(a, prm, st) : launch_ns<256, true>(a, prm, st);

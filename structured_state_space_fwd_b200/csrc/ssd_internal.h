@@ -62,10 +62,11 @@ struct FusedLaunch {
     const float* D;
     const float* init;         // [b,H,P,N] or null
     float* finalbuf;           // [b,H,P,N] final states, or null
-    float* segbuf;             // [b,nseg,H,P,N] states entering segments 1.. (nseg > 1)
+    float* segbuf;             // [b,nslot,H,P,N] states entering segments 1.. (nseg > 1)
     int* sync_ints;            // fused_sync_ints ints, zeroed by the caller
     int kheads, seg_tiles, nseg;
     int chained;               // segment s > 0 takes its entering state from segment s - 1's unit
+    int nslot;                 // segbuf slots per batch row; 0: nseg
     int stall;                 // test builds: make chain waits run out
     void* y;                   // [b,T,H,P] bf16 (the map's tensor): rows of partial tiles
     // gate and norm after the layer, fused into the stores (z null: y stored as is):
@@ -102,7 +103,8 @@ cudaError_t launch_varlen_order(const int* cu, int ndoc, int64_t T, int* order, 
 // turns slot s (1 <= s <= nseg_out) into the state entering segment s (init entering
 // segment 0) and, when `final_out` is given, writes the state after segment
 // nseg_out - 1 there (and with `alpha_out` [b,H] the decay over segments
-// 0 .. nseg_out - 1). Bounded waits that give up set *error.
+// 0 .. nseg_out - 1); with store = false the slots are left as they are (only
+// final_out and alpha_out are written). Bounded waits that give up set *error.
 int segment_max_tiles();
 cudaError_t launch_segment_states(const Dims& d, const CUtensorMap* maps, const float* dt,
                                   const float* A, float* segbuf, float* decay, int* error,
@@ -110,7 +112,7 @@ cudaError_t launch_segment_states(const Dims& d, const CUtensorMap* maps, const 
                                   cudaStream_t st);
 cudaError_t launch_segment_scan(const Dims& d, const float* init, float* segbuf, const float* decay,
                                 int nseg, int nslot, int nseg_out, float* final_out,
-                                cudaStream_t st, float* alpha_out = nullptr);
+                                cudaStream_t st, float* alpha_out = nullptr, bool store = true);
 
 // Recurrent form for a few tokens per sequence, state [b,H,P,N] updated in place.
 struct StepLayout {

@@ -419,12 +419,12 @@ done:
 // thread of each (b, h)'s first vector also writes the product of the decays of
 // segments 0 .. nseg_out - 1 there: the decay over all of them. The walk over the
 // segments is a dependent chain of FMAs; the loads of the next kScanAhead slots are
-// in flight while it runs.
+// in flight while it runs. With store = 0 the slots are only read.
 constexpr int kScanAhead = 4;
 __global__ void segment_scan_kernel(const float* __restrict__ init, float* __restrict__ segbuf,
                                     const float* __restrict__ decay, int64_t nvec, int64_t H,
                                     int64_t PN4, int nseg, int nslot, int nseg_out, float* __restrict__ final_out,
-                                    float* __restrict__ alpha_out) {
+                                    float* __restrict__ alpha_out, int store) {
     const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (e >= nvec) return;
     const int64_t bh = e / PN4, off = e % PN4;
@@ -457,7 +457,7 @@ __global__ void segment_scan_kernel(const float* __restrict__ init, float* __res
             }
             prod *= f;
             cur = make_float4(fmaf(f, cur.x, v.x), fmaf(f, cur.y, v.y), fmaf(f, cur.z, v.z), fmaf(f, cur.w, v.w));
-            if (s < nslot) __stcg(sb + slot(s), cur);
+            if (store && s < nslot) __stcg(sb + slot(s), cur);
         }
     }
     if (final_out) reinterpret_cast<float4*>(final_out)[bh * PN4 + off] = cur;
@@ -518,7 +518,8 @@ cudaError_t launch_segment_states(const Dims& d, const CUtensorMap* maps, const 
 }
 
 cudaError_t launch_segment_scan(const Dims& d, const float* init, float* segbuf, const float* decay, int nseg,
-                                int nslot, int nseg_out, float* final_out, cudaStream_t st, float* alpha_out) {
+                                int nslot, int nseg_out, float* final_out, cudaStream_t st, float* alpha_out,
+                                bool store) {
     if ((d.P * d.N) % 4 != 0) return cudaErrorInvalidValue;
     const int64_t PN4 = d.P * d.N / 4;
     const int64_t nvec = d.b * d.H * PN4;
@@ -527,7 +528,7 @@ cudaError_t launch_segment_scan(const Dims& d, const float* init, float* segbuf,
     const int64_t blocks = (nvec + threads - 1) / threads;
     if (blocks > INT32_MAX) return cudaErrorInvalidValue;
     segment_scan_kernel<<<(unsigned)blocks, threads, 0, st>>>(init, segbuf, decay, nvec, d.H, PN4, nseg, nslot,
-                                                              nseg_out, final_out, alpha_out);
+                                                              nseg_out, final_out, alpha_out, store ? 1 : 0);
     return cudaGetLastError();
 }
 
