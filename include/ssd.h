@@ -135,13 +135,18 @@ SSD_API ssd_status_t ssd_fwd(const ssd_shape_t* shape,
  *   served too. All calls on a device share the one array and
  *   it keeps the last call's contents, which no call relies on; calls that can
  *   overlap on the GPU (different streams, or different host threads without
- *   ordering) race on it and must be serialized by the caller.
+ *   ordering) race on it and must be serialized by the caller. A bounded wait
+ *   that gave up inside the kernel is reported by ssd_fwd_no_alloc_check.
  */
 SSD_API ssd_status_t ssd_fwd_no_alloc(const ssd_shape_t* shape,
                                       const void* x, const float* dt, const float* A,
                                       const void* B, const void* C, const float* D,
                                       const float* initial_states,
                                       void* y, float* final_states, void* stream);
+
+/* Device-side status of the last ssd_fwd_no_alloc on the current device (same
+ * shape): ssd_fwd_check on the static scratch array. Waits for `stream`. */
+SSD_API ssd_status_t ssd_fwd_no_alloc_check(const ssd_shape_t* shape, void* stream);
 
 /*
  * Device-side status of the last ssd_fwd that ran with `workspace` (same shape

@@ -46,6 +46,7 @@ _SIGS = {
     "ssd_fwd_host_workspace_size": ([ctypes.POINTER(ShapeT), ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
     "ssd_fwd_host": ([ctypes.POINTER(ShapeT)] + [_VP] * 10 + [ctypes.c_size_t, _VP], ctypes.c_int),
     "ssd_fwd_no_alloc": ([ctypes.POINTER(ShapeT)] + [_VP] * 10, ctypes.c_int),
+    "ssd_fwd_no_alloc_check": ([ctypes.POINTER(ShapeT), _VP], ctypes.c_int),
     "ssd_fwd_check": ([ctypes.POINTER(ShapeT), _VP, ctypes.c_size_t, _VP], ctypes.c_int),
     "ssd_fwd_varlen_workspace_size": ([ctypes.POINTER(ShapeT), ctypes.c_int64,
                                        ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),

@@ -67,3 +67,11 @@ extern "C" ssd_status_t ssd_fwd_no_alloc(const ssd_shape_t* shape, const void* x
     return ssd_fwd(shape, x, dt, A, B, C, D, initial_states, y, final_states, scratch,
                    kNoAllocScratchBytes, stream);
 }
+
+extern "C" ssd_status_t ssd_fwd_no_alloc_check(const ssd_shape_t* shape, void* stream) {
+    void* scratch = scratch_for_current_device();
+    if (!scratch) return SSD_ERR_CUDA;
+    // the last ssd_fwd_no_alloc on this device left its status words where any
+    // ssd_fwd call on a workspace leaves them: at the start of the scratch array
+    return ssd_fwd_check(shape, scratch, kNoAllocScratchBytes, stream);
+}

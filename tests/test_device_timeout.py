@@ -59,11 +59,25 @@ try:
 except SSDError as e:
     assert e.status == SSD_ERR_TIMEOUT, e
 
+# and the no-alloc entry point, through its own status check
+import ctypes
+p = lambda t: ctypes.c_void_p(t.data_ptr()) if t is not None else None  # noqa: E731
+yb = torch.empty_like(d["x"])
+fb = torch.empty_like(d["initial_states"])
+st = ssd.lib().ssd_fwd_no_alloc(ctypes.byref(shape), p(d["x"]), p(d["dt"]), p(d["A"]), p(d["B"]), p(d["C"]),
+                                p(d["D"]), p(d["initial_states"]), p(yb), p(fb), None)
+assert st == 0, st
+st = ssd.lib().ssd_fwd_no_alloc_check(ctypes.byref(shape), None)
+assert st == SSD_ERR_TIMEOUT, st
+
 # the context is still usable: the next call is correct and reports OK
 del os.environ["SSD_TEST_STALL_CHAIN"]
 y, f = ssd.ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], chunk_size=256,
                    initial_states=d["initial_states"], return_final_states=True, workspace=ws)
 ssd.ssd_fwd_check(shape, ws)
+st = ssd.lib().ssd_fwd_no_alloc(ctypes.byref(shape), p(d["x"]), p(d["dt"]), p(d["A"]), p(d["B"]), p(d["C"]),
+                                p(d["D"]), p(d["initial_states"]), p(yb), p(fb), None)
+assert st == 0 and ssd.lib().ssd_fwd_no_alloc_check(ctypes.byref(shape), None) == 0
 torch.cuda.synchronize()
 y_ref, f_ref, _ = oracle.recurrence(**inp)
 assert oracle.rel_err(y.float().cpu(), y_ref) <= 5e-3
