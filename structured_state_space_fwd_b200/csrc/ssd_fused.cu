@@ -355,6 +355,158 @@ __device__ __forceinline__ void mma_tokens_tmem(uint32_t d, uint32_t a, uint64_t
         mma_bf16_tmem_a(d, a + 8 * kk, dB + (uint64_t)(kk * 128), idesc, 1u);
 }
 
+// The skip term D x_j / q_j (or D x_j) of one head into its 64 columns of the
+// tile's Y'' (taddr: this warp's lanes, the head's first column), from the thread's
+// bf16 row of x.
+__device__ __forceinline__ void preload_skip(uint32_t taddr, const uint4 (&xv)[8], float dq) {
+    const float2 d2 = make_float2(dq, dq);
+#pragma unroll
+    for (int h4 = 0; h4 < 4; ++h4) {
+        uint32_t pre[16];
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            const uint32_t xw[4] = {xv[2 * h4 + cc].x, xv[2 * h4 + cc].y, xv[2 * h4 + cc].z, xv[2 * h4 + cc].w};
+#pragma unroll
+            for (int e2 = 0; e2 < 4; ++e2) {
+                const float2 v = mul2(d2, unpack_bf16(xw[e2]));
+                pre[8 * cc + 2 * e2] = __float_as_uint(v.x);
+                pre[8 * cc + 2 * e2 + 1] = __float_as_uint(v.y);
+            }
+        }
+        tmem_st16(taddr + 16 * h4, pre);
+    }
+}
+
+// The mask group's work on a tile in the unfactored form (a head decays by more than
+// 2^96 over it), for thread j (token row j, TMEM lanes at tl = tmem base + lane
+// quarter): per head the skip term, the row's factor 2^cs_j, and its
+// P = G o exp(cs_j - cs_i) dt_i (exponent per element) in the S slot; then, after the
+// products with the raw x tiles, w o x in place. Kept out of line: it is rare, and
+// its registers would otherwise weigh on the common path. False if a wait gave up.
+__device__ __noinline__ bool mask_unfactored_tile(Bars* bs, int* err, const float* cs_base, float* yi,
+                                                  uint8_t* sxp, uint32_t tl, int ys, int xs, int hi, int np,
+                                                  int i, int nsh, int j, int wq) {
+    // the per-head masks need G and go into the S slot (free once the previous tile's
+    // S, or C h^T, has been read)
+    if (!wait_bar_all(&bs->g_full, i & 1, bs, err)) return false;
+    if (!wait_bar_all(&bs->s_empty, (i & 1) ^ 1, bs, err)) return false;
+    tc_fence_after();
+    __syncwarp();
+    float wv[2];
+    for (int e = 0; e < np; ++e) {
+        const int c = (hi + e) % kCsSlots;
+        if (!wait_bar_all(&bs->cs_full[c], ((hi + e) / kCsSlots) & 1, bs, err)) return false;
+        const float* cs = cs_base + c * (kCsSlotBytes / 4);
+        const float L = cs[kCsL], csj = cs[j];
+        wv[e] = ex2(L - csj) * cs[kTile + j];
+        yi[e * kTile + j] = ex2(csj);
+        if (j == 0) yi[kYiEL + e] = ex2(L);
+        uint8_t* sx = sxp + e * kAtom;
+        uint4 xv[8];
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) xv[c8] = *reinterpret_cast<const uint4*>(sx + swz(j, c8));
+        preload_skip(tl + kColY + 128 * ys + 64 * e, xv, cs[kCsD]);
+        const float* dts = cs + kTile;
+#pragma unroll 1
+        for (int blk = 0; blk < 4; ++blk) {
+            uint32_t pk[16];
+            if (blk > wq) {
+#pragma unroll
+                for (int q2 = 0; q2 < 16; ++q2) pk[q2] = 0u;
+            } else {
+                float gv[32];
+                tmem_ld32(tl + kColG + 32 * blk, gv);
+                tmem_ld_wait_regs(gv);
+#pragma unroll
+                for (int q2 = 0; q2 < 16; ++q2) {
+                    const int i0 = 32 * blk + 2 * q2;
+                    const float p0 = i0 <= j ? gv[2 * q2] * ex2(csj - cs[i0]) * dts[i0] : 0.f;
+                    const float p1 = i0 + 1 <= j ? gv[2 * q2 + 1] * ex2(csj - cs[i0 + 1]) * dts[i0 + 1] : 0.f;
+                    pk[q2] = pack_bf16(p0, p1);
+                }
+            }
+            tmem_st16(tl + kColS + 64 * e + 16 * blk, pk);
+        }
+    }
+    if (j == 0) yi[kYiMode] = 0.f;
+    tmem_st_wait();
+    mbar_arrive(&bs->yi_full[ys]);
+    if (j == 0) bs->xmode[xs] = 0;
+    tc_fence_before();
+    mbar_arrive(&bs->wx_full[xs]);
+    mbar_arrive(&bs->g_empty_mask);     // G has served the masks
+    // the products with the raw x tiles have read them: now scale in place
+    if (!wait_bar_all(&bs->xr_done, nsh & 1, bs, err)) return false;
+    for (int e = 0; e < np; ++e) {
+        uint8_t* sx = sxp + e * kAtom;
+        const float2 w2 = make_float2(wv[e], wv[e]);
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) {
+            const uint4 xr = *reinterpret_cast<const uint4*>(sx + swz(j, c8));
+            *reinterpret_cast<uint4*>(sx + swz(j, c8)) =
+                make_uint4(pack_bf16(mul2(w2, unpack_bf16(xr.x))), pack_bf16(mul2(w2, unpack_bf16(xr.y))),
+                           pack_bf16(mul2(w2, unpack_bf16(xr.z))), pack_bf16(mul2(w2, unpack_bf16(xr.w))));
+        }
+    }
+    fence_proxy_async_smem();
+    mbar_arrive(&bs->wx2_full);
+    return true;
+}
+
+// The MMA issuer's work on a tile in the unfactored form, after G: per head Y = P x
+// with the raw x tile (P in the S slot), S once the tile is scaled in place, and C h^T
+// into the S slot once the chain group has read S. Out of line for the same reason
+// as the mask group's. False if a wait gave up.
+__device__ __noinline__ bool mma_unfactored_tile(Bars* bs, int* err, uint32_t tmem, int ys, int xs, int tbB,
+                                                 int tbC, int item, int nsh, int nrd, int np, int kmh, int ksN,
+                                                 uint64_t dX, uint64_t dSA, uint64_t dC, uint64_t dH, uint32_t idS,
+                                                 uint32_t idY) {
+    constexpr uint32_t idY1 = idesc_bf16(128, 64, 0, 1);   // one head
+    tc_fence_after();
+    for (int e = 0; e < np; ++e)
+        mma_tokens_tmem(tmem + kColY + 128 * ys + 64 * e, tmem + kColS + 64 * e, dX + (uint64_t)((e * kAtom) >> 4),
+                        idY1);
+    mma_commit(&bs->xr_done);
+    if (!wait_bar(&bs->wx2_full, nsh & 1, bs, err)) return false;
+    tc_fence_after();
+    for (int mh = 0; mh < kmh; ++mh)
+        mma_tokens_smem(tmem + kColS + 64 * mh, dSA + (uint64_t)((2 * mh * kAtom) >> 4), dX, idS);
+    mma_commit(&bs->s_full);
+    mma_commit(&bs->x_empty[xs]);
+    mma_commit(&bs->tb_empty[tbB]);    // this tile's B has served G and S
+    if (!wait_bar(&bs->s_read, nrd & 1, bs, err)) return false;
+    if (!wait_bar(&bs->h_full, item & 1, bs, err)) return false;
+    tc_fence_after();
+    mma_state_dim_n<true>(ksN, tmem + kColS, dC, dH, idY, 0u);
+    mma_commit(&bs->h_free);
+    mma_commit(&bs->tb_empty[tbC]);
+    mma_commit(&bs->y_full[ys]);
+    return true;
+}
+
+// The epilogue's row of an unfactored tile for head e: y = Y'' + f R (f = 2^cs_r, R
+// in the S slot), bf16 into the staging row r. Out of line, as the rest of that form.
+__device__ __noinline__ void stage_unfactored_row(uint32_t tl, int ys, int e, float f, uint8_t* stg, int r) {
+    const float2 f2 = make_float2(f, f);
+#pragma unroll 1
+    for (int pc = 0; pc < 4; ++pc) {
+        float yv[16], rv[16];
+        tmem_ld16(tl + kColY + 128 * ys + 64 * e + 16 * pc, yv);
+        tmem_ld16(tl + kColS + 64 * e + 16 * pc, rv);
+        tmem_ld_wait_regs(yv, rv);
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            uint32_t o[4];
+#pragma unroll
+            for (int e2 = 0; e2 < 4; ++e2) {
+                const int x0 = 8 * cc + 2 * e2;
+                o[e2] = pack_bf16(fma2(f2, make_float2(rv[x0], rv[x0 + 1]), make_float2(yv[x0], yv[x0 + 1])));
+            }
+            *reinterpret_cast<uint4*>(stg + swz(r, 2 * pc + cc)) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+    }
+}
+
 // SiLU(z) = z sigmoid(z) = z (1 + tanh(z / 2)) / 2: one special-function
 // instruction (tanh.approx, a relative error near 2^-11, under the bf16 output's
 // rounding).
@@ -592,7 +744,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t idG = idesc_bf16(128, 128, 0, 0);   // C (K-major) x B (K-major)
             const uint32_t idS = np == 2 ? idesc_bf16(128, 128, 1, 1) : idesc_bf16(128, 64, 1, 1);
             const uint32_t idY = np == 2 ? idesc_bf16(128, 128, 0, 1) : idesc_bf16(128, 64, 0, 1);
-            constexpr uint32_t idY1 = idesc_bf16(128, 64, 0, 1);   // one head (unfactored masked product)
             const uint64_t dH = sw128_desc(smem_u32(smem + K::kOffH), kAtom, 1024);
             struct Pend {
                 int item, ys, cb;   // cb: tile buffer of the tile's C
@@ -663,27 +814,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_commit(&bs->g_empty_mma);
                         mma_commit(&bs->y_full[ys]);
                     } else {
-                        // per head Y = P x with the raw tile (P in the S slot), then S once
-                        // the tile is scaled in place
-                        tc_fence_after();
-                        for (int e = 0; e < np; ++e)
-                            mma_tokens_tmem(tmem + kColY + 128 * ys + 64 * e, tmem + kColS + 64 * e,
-                                            dX + (uint64_t)((e * kAtom) >> 4), idY1);
-                        mma_commit(&bs->xr_done);
-                        if (!wait_bar(&bs->wx2_full, nsh & 1, bs, err)) goto drain;
+                        // the rare form, out of line
+                        if (!mma_unfactored_tile(bs, err, tmem, ys, xs, tbB, tbC, i, nsh, nrd, np, K::kMH, ksN, dX,
+                                                 dSA, sw128_desc(smem_u32(smem + K::kOffBC + tbC * K::kBCTile), 16, 1024),
+                                                 dH, idS, idY))
+                            goto drain;
                         ++nsh;
-                        tc_fence_after();
-#pragma unroll
-                        for (int mh = 0; mh < K::kMH; ++mh)
-                            mma_tokens_smem(tmem + kColS + 64 * mh, dSA + (uint64_t)((2 * mh * kAtom) >> 4), dX, idS);
-                        mma_commit(&bs->s_full);
-                        mma_commit(&bs->x_empty[xs]);
-                        mma_commit(&bs->tb_empty[tbB]);    // this tile's B has served G and S
-                        // C h^T goes into the S slot once the chain group has read S
-                        if (!wait_bar(&bs->s_read, nrd & 1, bs, err)) goto drain;
                         ++nrd;
-                        if (!issue_r(Pend{i, ys, tbC, false})) goto drain;
-                        mma_commit(&bs->y_full[ys]);
                     }
                     prev_shared = shared;
                 }
@@ -842,52 +979,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool shared = cs_base[(hi % kCsSlots) * (kCsSlotBytes / 4) + kCsMode] != 0.f;
                 if (!wait_bar_all(&bs->x_full[xs], (i / K::kXSlots) & 1, bs, err)) goto done;
                 if (!wait_bar_all(&bs->y_empty[ys], ((i / kYSlots) & 1) ^ 1, bs, err)) goto done;
-                if (!shared) {
-                    // the per-head masks need G and go into the S slot (free once the
-                    // previous tile's S, or C h^T, has been read)
-                    if (!wait_bar_all(&bs->g_full, i & 1, bs, err)) goto done;
-                    if (!wait_bar_all(&bs->s_empty, (i & 1) ^ 1, bs, err)) goto done;
-                }
                 float* yi = reinterpret_cast<float*>(smem + K::kOffYInfo + ys * kYInfoBytes);
                 uint8_t* sxp = smem + K::kOffX + xs * K::kXBytes;
-                tc_fence_after();
-                __syncwarp();
-                float wv[2];
-                for (int e = 0; e < np; ++e) {
-                    const int c = (hi + e) % kCsSlots;
-                    if (!wait_bar_all(&bs->cs_full[c], ((hi + e) / kCsSlots) & 1, bs, err)) goto done;
-                    const float* cs = cs_base + c * (kCsSlotBytes / 4);
-                    const float L = cs[kCsL], csj = cs[j];
-                    const float up = ex2(L - csj);                  // 2^(L - cs_j) <= 1
-                    wv[e] = up * cs[kTile + j];                     // w_j = 2^(L - cs_j) dt_j
-                    const float dq = cs[kCsD] * (shared ? up : 1.f);  // D / q_j, or D
-                    // what the chain and epilogue groups need, kept with the tile's Y''
-                    yi[e * kTile + j] = shared ? ex2(csj - L) : ex2(csj);   // q_j, or 2^cs_j
-                    if (j == 0) yi[kYiEL + e] = ex2(L);
-                    uint8_t* sx = sxp + e * kAtom;
-                    uint4 xv[8];
+                if (!shared) {
+                    // the rare form (a head decays by more than 2^96 over the tile): out of
+                    // line, so that its registers and code stay off the common path
+                    if (!mask_unfactored_tile(bs, err, cs_base, yi, sxp, tmem + lb, ys, xs, hi, np, i, nsh, j, wq))
+                        goto done;
+                    ++nsh;
+                } else {
+                    tc_fence_after();
+                    __syncwarp();
+                    for (int e = 0; e < np; ++e) {
+                        const int c = (hi + e) % kCsSlots;
+                        if (!wait_bar_all(&bs->cs_full[c], ((hi + e) / kCsSlots) & 1, bs, err)) goto done;
+                        const float* cs = cs_base + c * (kCsSlotBytes / 4);
+                        const float L = cs[kCsL], csj = cs[j];
+                        const float up = ex2(L - csj);              // 2^(L - cs_j) <= 1
+                        const float w = up * cs[kTile + j];         // w_j = 2^(L - cs_j) dt_j
+                        const float dq = cs[kCsD] * up;             // D / q_j
+                        // what the chain and epilogue groups need, kept with the tile's Y''
+                        yi[e * kTile + j] = ex2(csj - L);           // q_j
+                        if (j == 0) yi[kYiEL + e] = ex2(L);
+                        uint8_t* sx = sxp + e * kAtom;
+                        uint4 xv[8];
 #pragma unroll
-                    for (int c8 = 0; c8 < 8; ++c8) xv[c8] = *reinterpret_cast<const uint4*>(sx + swz(j, c8));
-                    // skip term into head e's 64 columns of the tile's Y''
-                    const float2 d2 = make_float2(dq, dq);
-#pragma unroll
-                    for (int h4 = 0; h4 < 4; ++h4) {
-                        uint32_t pre[16];
-#pragma unroll
-                        for (int cc = 0; cc < 2; ++cc) {
-                            const uint32_t xw[4] = {xv[2 * h4 + cc].x, xv[2 * h4 + cc].y, xv[2 * h4 + cc].z,
-                                                    xv[2 * h4 + cc].w};
-#pragma unroll
-                            for (int e2 = 0; e2 < 4; ++e2) {
-                                const float2 v = mul2(d2, unpack_bf16(xw[e2]));
-                                pre[8 * cc + 2 * e2] = __float_as_uint(v.x);
-                                pre[8 * cc + 2 * e2 + 1] = __float_as_uint(v.y);
-                            }
-                        }
-                        tmem_st16(tmem + lb + kColY + 128 * ys + 64 * e + 16 * h4, pre);
-                    }
-                    if (shared) {
-                        const float2 w2 = make_float2(wv[e], wv[e]);
+                        for (int c8 = 0; c8 < 8; ++c8) xv[c8] = *reinterpret_cast<const uint4*>(sx + swz(j, c8));
+                        // skip term into head e's 64 columns of the tile's Y''
+                        preload_skip(tmem + lb + kColY + 128 * ys + 64 * e, xv, dq);
+                        const float2 w2 = make_float2(w, w);
 #pragma unroll
                         for (int c8 = 0; c8 < 8; ++c8)
                             *reinterpret_cast<uint4*>(sx + swz(j, c8)) =
@@ -895,36 +1015,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                                            pack_bf16(mul2(w2, unpack_bf16(xv[c8].y))),
                                            pack_bf16(mul2(w2, unpack_bf16(xv[c8].z))),
                                            pack_bf16(mul2(w2, unpack_bf16(xv[c8].w))));
-                    } else {
-                        // head e's P = G o exp(cs_j - cs_i) dt_i (exact exponent per element)
-                        const float* dts = cs + kTile;
-#pragma unroll 1
-                        for (int blk = 0; blk < 4; ++blk) {
-                            uint32_t pk[16];
-                            if (blk > wq) {
-#pragma unroll
-                                for (int q2 = 0; q2 < 16; ++q2) pk[q2] = 0u;
-                            } else {
-                                float gv[32];
-                                tmem_ld32(tmem + lb + kColG + 32 * blk, gv);
-                                tmem_ld_wait_regs(gv);
-#pragma unroll
-                                for (int q2 = 0; q2 < 16; ++q2) {
-                                    const int i0 = 32 * blk + 2 * q2;
-                                    const float p0 = i0 <= j ? gv[2 * q2] * ex2(csj - cs[i0]) * dts[i0] : 0.f;
-                                    const float p1 =
-                                        i0 + 1 <= j ? gv[2 * q2 + 1] * ex2(csj - cs[i0 + 1]) * dts[i0 + 1] : 0.f;
-                                    pk[q2] = pack_bf16(p0, p1);
-                                }
-                            }
-                            tmem_st16(tmem + lb + kColS + 64 * e + 16 * blk, pk);
-                        }
                     }
-                }
-                if (j == 0) yi[kYiMode] = shared ? 1.f : 0.f;
-                tmem_st_wait();
-                mbar_arrive(&bs->yi_full[ys]);
-                if (shared) {
+                    if (j == 0) yi[kYiMode] = 1.f;
+                    tmem_st_wait();
+                    mbar_arrive(&bs->yi_full[ys]);
                     fence_proxy_async_smem();
                     if (j == 0) bs->xmode[xs] = 1;
                     tc_fence_before();
@@ -959,27 +1053,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_st_wait();
                     tc_fence_before();
                     mbar_arrive(&bs->p_full);
-                } else {
-                    if (j == 0) bs->xmode[xs] = 0;
-                    tc_fence_before();
-                    mbar_arrive(&bs->wx_full[xs]);
-                    mbar_arrive(&bs->g_empty_mask);     // G has served the masks
-                    // the products with the raw x tiles have read them: now scale in place
-                    if (!wait_bar_all(&bs->xr_done, nsh & 1, bs, err)) goto done;
-                    ++nsh;
-                    for (int e = 0; e < np; ++e) {
-                        uint8_t* sx = sxp + e * kAtom;
-                        const float2 w2 = make_float2(wv[e], wv[e]);
-#pragma unroll
-                        for (int c8 = 0; c8 < 8; ++c8) {
-                            const uint4 xr = *reinterpret_cast<const uint4*>(sx + swz(j, c8));
-                            *reinterpret_cast<uint4*>(sx + swz(j, c8)) =
-                                make_uint4(pack_bf16(mul2(w2, unpack_bf16(xr.x))), pack_bf16(mul2(w2, unpack_bf16(xr.y))),
-                                           pack_bf16(mul2(w2, unpack_bf16(xr.z))), pack_bf16(mul2(w2, unpack_bf16(xr.w))));
-                        }
-                    }
-                    fence_proxy_async_smem();
-                    mbar_arrive(&bs->wx2_full);
                 }
                 for (int e = 0; e < np; ++e) mbar_arrive(&bs->cs_empty[(hi + e) % kCsSlots]);
                 hi += np;
@@ -1121,27 +1194,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // the warp's previous store has read its staging rows
                     if (lane == 0) bulk_wait_group_read0();
                     __syncwarp();
+                    if (shared) {
 #pragma unroll 1
-                    for (int pc = 0; pc < 4; ++pc) {
-                        float yv[16], rv[16];
-                        tmem_ld16(tmem + lb + kColY + 128 * ys + 64 * e + 16 * pc, yv);
-                        if (shared) {
+                        for (int pc = 0; pc < 4; ++pc) {
+                            float yv[16];
+                            tmem_ld16(tmem + lb + kColY + 128 * ys + 64 * e + 16 * pc, yv);
                             tmem_ld_wait_regs(yv);
-                        } else {
-                            tmem_ld16(tmem + lb + kColS + 64 * e + 16 * pc, rv);
-                            tmem_ld_wait_regs(yv, rv);
-                        }
 #pragma unroll
-                        for (int cc = 0; cc < 2; ++cc) {
-                            uint32_t o[4];
+                            for (int cc = 0; cc < 2; ++cc) {
+                                uint32_t o[4];
 #pragma unroll
-                            for (int e2 = 0; e2 < 4; ++e2) {
-                                const int x0 = 8 * cc + 2 * e2;
-                                const float2 yy = make_float2(yv[x0], yv[x0 + 1]);
-                                o[e2] = pack_bf16(shared ? mul2(f2, yy) : fma2(f2, make_float2(rv[x0], rv[x0 + 1]), yy));
+                                for (int e2 = 0; e2 < 4; ++e2) {
+                                    const int x0 = 8 * cc + 2 * e2;
+                                    o[e2] = pack_bf16(mul2(f2, make_float2(yv[x0], yv[x0 + 1])));
+                                }
+                                *reinterpret_cast<uint4*>(stg + swz(r, 2 * pc + cc)) = make_uint4(o[0], o[1], o[2], o[3]);
                             }
-                            *reinterpret_cast<uint4*>(stg + swz(r, 2 * pc + cc)) = make_uint4(o[0], o[1], o[2], o[3]);
                         }
+                    } else {
+                        stage_unfactored_row(tmem + lb, ys, e, f, stg, r);
                     }
                     if (e == np - 1) {
                         // the tile's accumulators are read: free them before the stores
