@@ -331,15 +331,20 @@ __device__ __forceinline__ void mma_state_dim(uint32_t d, uint64_t dA, uint64_t 
         mma_bf16(d, dA + kofs, dB + (kBRows ? (uint64_t)(kk * (2048 >> 4)) : kofs), idesc, kk > 0 ? 1u : acc0);
     }
 }
-template <bool kBRows>
+// ks: 1, 2, 4 or 8 with a state capacity of 128; always 16 with 256 (a state above 128)
+template <bool kBRows, int NS>
 __device__ __forceinline__ void mma_state_dim_n(int ks, uint32_t d, uint64_t dA, uint64_t dB, uint32_t idesc,
                                                 uint32_t acc0) {
-    switch (ks) {
-        case 1: mma_state_dim<1, kBRows>(d, dA, dB, idesc, acc0); break;
-        case 2: mma_state_dim<2, kBRows>(d, dA, dB, idesc, acc0); break;
-        case 4: mma_state_dim<4, kBRows>(d, dA, dB, idesc, acc0); break;
-        case 8: mma_state_dim<8, kBRows>(d, dA, dB, idesc, acc0); break;
-        default: mma_state_dim<16, kBRows>(d, dA, dB, idesc, acc0); break;
+    if constexpr (NS == 256) {
+        mma_state_dim<16, kBRows>(d, dA, dB, idesc, acc0);
+    } else {
+        switch (ks) {
+            case 1: mma_state_dim<1, kBRows>(d, dA, dB, idesc, acc0); break;
+            case 2: mma_state_dim<2, kBRows>(d, dA, dB, idesc, acc0); break;
+            case 4: mma_state_dim<4, kBRows>(d, dA, dB, idesc, acc0); break;
+            case 8: mma_state_dim<8, kBRows>(d, dA, dB, idesc, acc0); break;
+            default: mma_state_dim<16, kBRows>(d, dA, dB, idesc, acc0); break;
+        }
     }
 }
 // 8 steps of K = 16 over the tile's tokens: A from shared memory (B^T, N-contiguous)
@@ -457,6 +462,7 @@ __device__ __noinline__ bool mask_unfactored_tile(Bars* bs, int* err, const floa
 // with the raw x tile (P in the S slot), S once the tile is scaled in place, and C h^T
 // into the S slot once the chain group has read S. Out of line for the same reason
 // as the mask group's. False if a wait gave up.
+template <int NS>
 __device__ __noinline__ bool mma_unfactored_tile(Bars* bs, int* err, uint32_t tmem, int ys, int xs, int tbB,
                                                  int tbC, int item, int nsh, int nrd, int np, int kmh, int ksN,
                                                  uint64_t dX, uint64_t dSA, uint64_t dC, uint64_t dH, uint32_t idS,
@@ -477,7 +483,7 @@ __device__ __noinline__ bool mma_unfactored_tile(Bars* bs, int* err, uint32_t tm
     if (!wait_bar(&bs->s_read, nrd & 1, bs, err)) return false;
     if (!wait_bar(&bs->h_full, item & 1, bs, err)) return false;
     tc_fence_after();
-    mma_state_dim_n<true>(ksN, tmem + kColS, dC, dH, idY, 0u);
+    mma_state_dim_n<true, NS>(ksN, tmem + kColS, dC, dH, idY, 0u);
     mma_commit(&bs->h_free);
     mma_commit(&bs->tb_empty[tbC]);
     mma_commit(&bs->y_full[ys]);
@@ -757,7 +763,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const uint64_t dC = sw128_desc(smem_u32(smem + K::kOffBC + q.cb * K::kBCTile), 16, 1024);
                 const uint32_t d = q.shared ? tmem + kColY + 128 * q.ys : tmem + kColS;
-                mma_state_dim_n<true>(ksN, d, dC, dH, idY, q.shared ? 1u : 0u);
+                mma_state_dim_n<true, NS>(ksN, d, dC, dH, idY, q.shared ? 1u : 0u);
                 mma_commit(&bs->h_free);
                 mma_commit(&bs->tb_empty[q.cb]);
                 return true;
@@ -789,7 +795,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                     tc_fence_after();
-                    mma_state_dim_n<false>(ksN, tmem + kColG, sw128_desc(bcC, 16, 1024), sw128_desc(bcB, 16, 1024), idG, 0u);
+                    mma_state_dim_n<false, NS>(ksN, tmem + kColG, sw128_desc(bcC, 16, 1024), sw128_desc(bcB, 16, 1024), idG, 0u);
                     mma_commit(&bs->g_full);
                     const uint64_t dSA = sw128_desc(bcB, kAtom, 1024);
                     if (!wait_bar(&bs->wx_full[xs], (i / K::kXSlots) & 1, bs, err)) goto drain;
@@ -815,7 +821,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_commit(&bs->y_full[ys]);
                     } else {
                         // the rare form, out of line
-                        if (!mma_unfactored_tile(bs, err, tmem, ys, xs, tbB, tbC, i, nsh, nrd, np, K::kMH, ksN, dX,
+                        if (!mma_unfactored_tile<NS>(bs, err, tmem, ys, xs, tbB, tbC, i, nsh, nrd, np, K::kMH, ksN, dX,
                                                  dSA, sw128_desc(smem_u32(smem + K::kOffBC + tbC * K::kBCTile), 16, 1024),
                                                  dH, idS, idY))
                             goto drain;
