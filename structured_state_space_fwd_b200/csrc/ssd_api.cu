@@ -118,6 +118,10 @@ constexpr int64_t kChainedMinChains = SSD_CHAINED_MIN_CHAINS;  // fewer chains: 
 constexpr int64_t kSegmentMinTiles = 8;
 constexpr int64_t kTargetUnits = SSD_TARGET_UNITS;             // units wanted: about four waves of CTAs
 constexpr int64_t kSmCount = 148;
+#ifndef SSD_FIRST_SEG_PCT
+#define SSD_FIRST_SEG_PCT 75
+#endif
+constexpr int64_t kFirstSegPct = SSD_FIRST_SEG_PCT;   // two chained segments: the first's share of the tiles
 
 int64_t fused_chains(const ssd::Dims& d) {
     const int ns = ssd::fused_state_capacity(d.N);
@@ -151,7 +155,7 @@ bool steps_use_tc(const ssd::Dims& d) {
 // segment (unit), segments; chained = entering states come from the previous
 // segment's unit, otherwise from the segment-state pass and scan.
 struct SegPlan {
-    int kh, seg_tiles, nseg;
+    int kh, seg_tiles, nseg, seg_first;
     bool chained;
 };
 SegPlan seg_plan(const ssd::Dims& d, Path path) {
@@ -165,12 +169,25 @@ SegPlan seg_plan(const ssd::Dims& d, Path path) {
     // chains than SMs splitting them only adds hand-offs to the critical path.
     int64_t nseg = (kTargetUnits + chains - 1) / chains;
     if (sp.chained && chains <= kSmCount) nseg = 1;
+#ifdef SSD_MAX_CHAINED_SEG
+    if (sp.chained) nseg = std::min<int64_t>(nseg, SSD_MAX_CHAINED_SEG);
+#endif
     if (path == Path::Segmented) nseg = std::max<int64_t>(2, nseg);
     nseg = std::max<int64_t>(1, std::min(nseg, ntiles));
     int64_t K = (ntiles + nseg - 1) / nseg;
     K = std::min<int64_t>(K, ssd::segment_max_tiles());
     sp.seg_tiles = (int)K;
     sp.nseg = (int)((ntiles + K - 1) / K);
+    sp.seg_first = sp.seg_tiles;
+    if (sp.chained && sp.nseg == 2) {
+        // Two chained segments: the second ones, taken last, are the shorter, so that
+        // the CTAs that take one more unit than others take a short one.
+        const int64_t first = std::min<int64_t>(ntiles - 1, (ntiles * kFirstSegPct + 50) / 100);
+        if (first > sp.seg_tiles) {
+            sp.seg_first = (int)first;
+            sp.seg_tiles = (int)(ntiles - first);
+        }
+    }
     return sp;
 }
 
@@ -309,6 +326,7 @@ ssd_status_t run_fwd(const ssd::Dims& d, const void* x, const float* dt, const f
         a.sync_ints = sync;
         a.kheads = w.sp.kh;
         a.seg_tiles = w.sp.seg_tiles;
+        a.seg_first = w.sp.seg_first;
         a.nseg = w.sp.nseg;
         a.chained = w.sp.chained ? 1 : 0;
         a.stall = test_stall();

@@ -35,12 +35,12 @@
 //   warp 0      TMA producer; takes units from the ticket and hands their ids to
 //               every role through a small ring
 //   warp 1      TMEM owner and MMA issuer (one thread)
-//   warp 2      per tile and head: dt loads, cumulative sum; per unit the flag of
-//               the state entering it (acquire)
+//   warp 2      per tile and head: dt loads, cumulative sum
 //   warp 3      per unit: makes the leaving state visible and releases its flag
 //   warps 4-7   mask group (thread = token row): per tile tril(C B^T) into TMEM,
 //               the skip-term preload and w o x in place of the x tiles
-//   warps 8-15  chain group (thread = state row, half of the head dim): carries
+//   warps 8-15  chain group (thread = state row, half of the head dim): per unit
+//               the flag of the state entering it (acquire) and that state; carries
 //               the state, per tile the bf16 operand of C (2^L h)^T
 //   warps 16-19 epilogue group (thread = token row): per tile and head
 //               y = q Y'', staged in shared memory (optionally gated by SiLU(z)
@@ -138,6 +138,7 @@ struct Params {
     const int* order;     // packed documents: unit order (documents, longest first)
     int64_t T;
     int H, G, N, kheads, batch, nunits, ntiles, seg_tiles, nseg;
+    int seg_first;        // tiles of segment 0 (the others: seg_tiles)
     int nslot;            // segbuf slots per batch row (nseg, or more)
     int chained;          // entering states come from the previous segment's unit
     int stall;            // test builds only: chain flags awaited at a value never reached
@@ -295,12 +296,27 @@ __device__ __forceinline__ Unit decode(const Params& p, int u) {
     r.doc = r.b;
     r.tok0 = 0;
     r.len = (int)p.T;
-    r.t_begin = r.s * p.seg_tiles;
-    r.t_end = min(p.ntiles, r.t_begin + p.seg_tiles);
+    r.t_begin = r.s == 0 ? 0 : p.seg_first + (r.s - 1) * p.seg_tiles;
+    r.t_end = min(p.ntiles, r.s == 0 ? p.seg_first : r.t_begin + p.seg_tiles);
     return r;
 }
 __device__ __forceinline__ int64_t flag_index(const Params& p, int b, int s, int hb) {
     return ((int64_t)b * p.nseg + s) * (p.H / p.kheads) + hb;
+}
+// Waits (bounded) for the flag of the state entering a chained unit and acquires
+// it; false (error word and abort set) when the wait runs out.
+__device__ __forceinline__ bool acquire_entry_flag(const Params& p, const Unit& U, Bars* bs, int* err) {
+    const int* f = p.flags + flag_index(p, U.b, U.s, U.hb);
+    const int want = 1 + (p.stall ? (1 << 30) : 0);
+    const uint64_t t0 = global_ns();
+    for (uint32_t it = 0;; ++it) {
+        if (ld_acquire(f) >= want) return true;
+        if (it >= 2) __nanosleep(128);
+        if ((it & 15) == 15 && (*(volatile int*)&bs->abort || global_ns() - t0 > kWaitLimitNs)) break;
+    }
+    *(volatile int*)&bs->abort = 1;
+    atomicExch(err, 1);
+    return false;
 }
 // state entering the unit for head h (null: zeros)
 __device__ __forceinline__ const float* entry_src(const Params& p, const Unit& U, int h) {
@@ -838,8 +854,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 2) {
         // ------------------------------------------------------------ cumsum warp
-        // Per unit: the flag of the state entering it (written by the previous
-        // segment's unit). Per tile: the dt of the pair's heads, the tile's form
+        // Per tile: the dt of the pair's heads, the tile's form
         // (factored unless a head decays by more than 2^96 over it), and per head
         // the cumulative sum of dt A (log2 units) into a slot for the mask group.
         int m = 0, hi = 0;
@@ -851,31 +866,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&bs->u_empty[ur]);
             if (u < 0) break;
             const Unit U = decode(prm, u);
-            if (prm.chained && U.s > 0) {
-                int bad = 0;
-                if (lane == 0) {
-                    const int* f = prm.flags + flag_index(prm, U.b, U.s, U.hb);
-                    const int want = 1 + (prm.stall ? (1 << 30) : 0);
-                    bool ok = false;
-                    const uint64_t t0 = global_ns();
-                    for (uint32_t it = 0;; ++it) {
-                        if (ld_acquire(f) >= want) {
-                            ok = true;
-                            break;
-                        }
-                        if (it >= 2) __nanosleep(128);
-                        if ((it & 15) == 15 &&
-                            (*(volatile int*)&bs->abort || global_ns() - t0 > kWaitLimitNs))
-                            break;
-                    }
-                    if (!ok) {
-                        *(volatile int*)&bs->abort = 1;
-                        atomicExch(err, 1);
-                        bad = 1;
-                    }
-                }
-                if (__any_sync(0xffffffffu, bad)) goto done;
-            }
             for (int t = U.t_begin; t < U.t_end; ++t) {
                 const int64_t t0 = (int64_t)t * kTile;
                 // tokens past the sequence's end get dt = 0: they neither move the
@@ -1105,16 +1095,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&bs->u_empty[ur]);
             if (u < 0) break;
             const Unit U = decode(prm, u);
-            // an empty document has no tiles: its final state is its initial state
-            if (U.t_begin == U.t_end) load_entry(U);
+            // The state entering the unit, loaded before its first tile is ready, so that
+            // the loads overlap the mask group's work on that tile: a chained unit's
+            // comes from the previous segment's unit once its flag is set (acquired by
+            // one thread; the chain group's barrier orders the others' loads after it).
+            // An empty document has no tiles: its final state is its initial state.
+            if (prm.chained && U.s > 0) {
+                const bool bad = tid == 256 && !acquire_entry_flag(prm, U, bs, err);
+                if (named_bar_or(1, 256, bad)) goto done;
+            }
+            load_entry(U);
             for (int t = U.t_begin; t < U.t_end; ++t, ++i) {
                 const int ys = i % kYSlots;
                 if (!wait_bar_all(&bs->yi_full[ys], (i / kYSlots) & 1, bs, err)) goto done;
                 const float* yi = reinterpret_cast<const float*>(smem + K::kOffYInfo + ys * kYInfoBytes);
                 const bool shared = yi[kYiMode] != 0.f;
-                // the state entering the unit (its flag was acquired before the tile's
-                // Y'' info was published)
-                if (t == U.t_begin) load_entry(U);
                 // the operand of the tile's state term, from the state entering the tile:
                 // 2^L h (factored) or h, once the previous tile's product has read it
                 if (!wait_bar_all(&bs->h_free, (i & 1) ^ 1, bs, err)) goto done;
@@ -1365,11 +1360,14 @@ cudaError_t launch_fused(const FusedLaunch& a, cudaStream_t st) {
     // tokens form one document
     const int64_t ntiles = (d.T + kTile - 1) / kTile + (packed ? 1 : 0);
     const int64_t nunits = (packed ? (int64_t)a.ndoc : (int64_t)a.nseg * d.b) * (d.H / a.kheads);
-    if (nunits > INT32_MAX / 2 || d.T > INT32_MAX / 2 || (!packed && (int64_t)a.seg_tiles * a.nseg < ntiles))
+    const int seg_first = a.seg_first > 0 ? a.seg_first : a.seg_tiles;
+    if (nunits > INT32_MAX / 2 || d.T > INT32_MAX / 2 ||
+        (!packed && seg_first + (int64_t)a.seg_tiles * (a.nseg - 1) < ntiles) || (!a.chained && seg_first != a.seg_tiles))
         return cudaErrorInvalidValue;
     prm.nunits = (int)nunits;
     prm.ntiles = (int)ntiles;
     prm.seg_tiles = a.seg_tiles;
+    prm.seg_first = seg_first;
     prm.nseg = a.nseg;
     prm.nslot = a.nslot > 0 ? a.nslot : a.nseg;
     if (prm.nslot < a.nseg) return cudaErrorInvalidValue;

@@ -65,6 +65,7 @@ struct FusedLaunch {
     float* segbuf;             // [b,nslot,H,P,N] states entering segments 1.. (nseg > 1)
     int* sync_ints;            // fused_sync_ints ints, zeroed by the caller
     int kheads, seg_tiles, nseg;
+    int seg_first;             // tiles of segment 0 (chained only; 0: seg_tiles)
     int chained;               // segment s > 0 takes its entering state from segment s - 1's unit
     int nslot;                 // segbuf slots per batch row; 0: nseg
     int stall;                 // test builds: make chain waits run out
