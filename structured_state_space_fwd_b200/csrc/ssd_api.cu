@@ -117,6 +117,20 @@ bool fused_ok(const ssd::Dims& d) {
 constexpr int64_t kChainedMinChains = SSD_CHAINED_MIN_CHAINS;  // fewer chains: compute entering states first
 constexpr int64_t kSegmentMinTiles = 8;
 constexpr int64_t kTargetUnits = SSD_TARGET_UNITS;             // units wanted: about four waves of CTAs
+#ifndef SSD_SEG_TARGET_UNITS
+#define SSD_SEG_TARGET_UNITS (2 * 148)
+#endif
+// Segments whose entering states come from the segment-state pass and scan: fewer,
+// longer ones (about two waves), since every segment adds a state slot to both
+// passes and a pipeline fill to each of its units.
+constexpr int64_t kSegTargetUnits = SSD_SEG_TARGET_UNITS;
+#ifndef SSD_CP_TARGET_UNITS
+#define SSD_CP_TARGET_UNITS 148
+#endif
+// A context-parallel slice: its segment-state pass and scan run twice per rank step
+// (record, then entering states), so fewer segments still (about one wave of the
+// segment-state pass).
+constexpr int64_t kCpTargetUnits = SSD_CP_TARGET_UNITS;
 constexpr int64_t kSmCount = 148;
 #ifndef SSD_FIRST_SEG_PCT
 #define SSD_FIRST_SEG_PCT 75
@@ -167,7 +181,8 @@ SegPlan seg_plan(const ssd::Dims& d, Path path) {
     const int64_t chains = std::max<int64_t>(1, d.b * (d.H / sp.kh));
     // Chained segments of one chain run one after another, so with no more
     // chains than SMs splitting them only adds hand-offs to the critical path.
-    int64_t nseg = (kTargetUnits + chains - 1) / chains;
+    const int64_t target = sp.chained ? kTargetUnits : kSegTargetUnits;
+    int64_t nseg = (target + chains - 1) / chains;
     if (sp.chained && chains <= kSmCount) nseg = 1;
 #ifdef SSD_MAX_CHAINED_SEG
     if (sp.chained) nseg = std::min<int64_t>(nseg, SSD_MAX_CHAINED_SEG);
@@ -403,7 +418,7 @@ CpWorkspace cp_workspace(const ssd::Dims& d) {
         const int64_t ntiles = (d.T + 127) / 128;
         w.kh = ssd::pick_kheads(d.H / d.G);
         const int64_t units_per_seg = std::max<int64_t>(1, d.b * (d.H / w.kh));
-        int64_t nseg = std::max<int64_t>(1, std::min<int64_t>(ntiles, (kTargetUnits + units_per_seg - 1) / units_per_seg));
+        int64_t nseg = std::max<int64_t>(1, std::min<int64_t>(ntiles, (kCpTargetUnits + units_per_seg - 1) / units_per_seg));
         int64_t K = std::min<int64_t>((ntiles + nseg - 1) / nseg, ssd::segment_max_tiles());
         w.seg_tiles = (int)K;
         w.nseg = (int)((ntiles + K - 1) / K);

@@ -420,7 +420,7 @@ done:
 // segments 0 .. nseg_out - 1 there: the decay over all of them. The walk over the
 // segments is a dependent chain of FMAs; the loads of the next kScanAhead slots are
 // in flight while it runs. With store = 0 the slots are only read.
-constexpr int kScanAhead = 4;
+constexpr int kScanAhead = 8;
 __global__ void segment_scan_kernel(const float* __restrict__ init, float* __restrict__ segbuf,
                                     const float* __restrict__ decay, int64_t nvec, int64_t H,
                                     int64_t PN4, int nseg, int nslot, int nseg_out, float* __restrict__ final_out,

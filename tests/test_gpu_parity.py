@@ -291,7 +291,7 @@ def test_zero_decay_is_causal_linear_attention(ssd, path_env, path):
 
 
 def test_segmented_several_tiles_per_segment(ssd, path_env):
-    # 200 tiles per sequence and 4 chains: segments of 3 tiles, 67 segments per
+    # 200 tiles per sequence and 8 chains: segments of 6 tiles, 34 segments per
     # chain, the last one short, entering states from the segment scan
     path_env("segmented")
     inp = make_inputs(batch=2, seqlen=128 * 200 - 37, nheads=8, headdim=64, ngroups=2, dstate=128,
