@@ -41,7 +41,7 @@ UNIT = "Mtokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant kernel, from
 # one ncu capture of this workload (profiles/); None until captured for the current kernel
-TRAFFIC = {"fused": 364895488}
+TRAFFIC = {"fused": 359387648}
 KERNEL_NAMES = {"fused": "ssd_fused_kernel",
                 "segmented": "segment_state_kernel + segment_scan_kernel + ssd_fused_kernel",
                 "steps": "chunk_cumsum + chunk_state_tc + state_passing + chunk_scan_tc",
