@@ -297,6 +297,9 @@ DECODE_METRIC = "SSD decode step (recurrent form) Mtokens/s at 2.7B layer shape,
 # dram__bytes_read.sum + dram__bytes_write.sum of one ssd_step_kernel launch on this
 # workload, from one ncu capture (profiles/); None once the kernel changes
 DECODE_TRAFFIC = 614955264
+# ncu DRAM bytes (read + write) of one gate launch, one group of 5120 channels
+# (profiles/gated_rmsnorm_kernel_2.7b_layer.md); the rest of out is still in L2
+GATE_TRAFFIC = 446350848
 
 
 def decode_bytes(w: W.Workload) -> float:
@@ -395,9 +398,9 @@ def measure_gate(ssd, dev, stream, steps, warmup, seed=0):
                        "seqlen": w.seqlen, "channels": w.nheads * w.headdim,
                        "group_size": w.nheads * w.headdim,
                        "l2": "y and z 168 MB each, larger than L2, no flush"},
-            "roofline": {"kernel": "gated_rmsnorm_kernel", "bound": "hbm",
+            "roofline": {"kernel": "gated_rmsnorm_pipelined_kernel", "bound": "hbm",
                          "achieved": by / (ms / 1e3) / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": by / (ms / 1e3) / 1e9 / pk["hbm_gbs"], "traffic": None,
+                         "frac": by / (ms / 1e3) / 1e9 / pk["hbm_gbs"], "traffic": GATE_TRAFFIC,
                          "alg_bytes_per_launch": by,
                          "peak_source": pk_kind + " (burst copy, MEASURED_PEAKS hbm_gbs)"},
             "gpu_launches": steps}
