@@ -15,6 +15,7 @@
 // persistent grid that loads a CTA's next groups while it reduces and writes
 // the current ones; larger groups are re-read (from L2) for the write.
 #include <algorithm>
+#include <type_traits>
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -59,15 +60,22 @@ __device__ __forceinline__ void store_vec(__nv_bfloat16* p, const float (&v)[8])
 __device__ __forceinline__ void store_vec(float* p, const float (&v)[1]) { *p = v[0]; }
 __device__ __forceinline__ void store_vec(__nv_bfloat16* p, const float (&v)[1]) { *p = __float2bfloat16_rn(v[0]); }
 
-// SiLU through the special-function unit (__expf, __fdividef): a few ulp, far
-// inside the fp32 bar at the gate's range, and 0 for very negative z (the
-// divisor overflows to inf). The accurate expf and IEEE division cost about
-// 40 instructions per element and made the pass 0.43 of the copy peak
-// instead of 0.57 (measured).
-template <int VW>
+// SiLU through the special-function unit. fp32 data: __expf and __fdividef, a
+// few ulp, far inside the fp32 bar at the gate's range, and 0 for very negative
+// z (the divisor overflows to inf); the accurate expf and IEEE division cost
+// about 40 instructions per element and made the pass 0.43 of the copy peak
+// instead of 0.57 (measured). bf16 data: z sigmoid(z) = z (1 + tanh(z / 2)) / 2,
+// one tanh.approx (relative error about 2^-11, below bf16's rounding of the
+// output), one special-function operation per element instead of two.
+__device__ __forceinline__ float silu_tanh(float z) {
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * z));
+    return 0.5f * z * (1.f + t);
+}
+template <int VW, bool kTanh>
 __device__ __forceinline__ void gate(const float (&y)[VW], const float (&z)[VW], float (&v)[VW]) {
 #pragma unroll
-    for (int i = 0; i < VW; ++i) v[i] = y[i] * __fdividef(z[i], 1.f + __expf(-z[i]));
+    for (int i = 0; i < VW; ++i) v[i] = kTanh ? y[i] * silu_tanh(z[i]) : y[i] * __fdividef(z[i], 1.f + __expf(-z[i]));
 }
 
 // E: storage type; VW: elements per vector (16 bytes, or 1 when the group size is
@@ -122,6 +130,7 @@ __global__ void __launch_bounds__(kGateThreads, pipe_ctas(TPG)) gated_rmsnorm_pi
     const E* __restrict__ y, const E* __restrict__ z, const float* __restrict__ w, E* __restrict__ out,
     int64_t ngroups_total, int64_t groups_per_row, int64_t gs, float eps) {
     using Raw = typename RawVec<E, VW>::T;
+    constexpr bool kBf16 = std::is_same<E, __nv_bfloat16>::value;
     constexpr int GPB = kGateThreads / TPG;
     constexpr int WPG = TPG / 32 > 0 ? TPG / 32 : 1;
     __shared__ float red[2][kGateThreads / 32];
@@ -155,7 +164,7 @@ __global__ void __launch_bounds__(kGateThreads, pipe_ctas(TPG)) gated_rmsnorm_pi
                 float a[VW], b[VW];
                 unpack(ry[i], a);
                 unpack(rz[i], b);
-                gate<VW>(a, b, v[i]);
+                gate<VW, kBf16>(a, b, v[i]);
 #pragma unroll
                 for (int e = 0; e < VW; ++e) ss = fmaf(v[i][e], v[i][e], ss);
             }
@@ -193,6 +202,7 @@ template <typename E, int VW, int TPG>
 __global__ void __launch_bounds__(kGateThreads, 5) gated_rmsnorm_kernel(
     const E* __restrict__ y, const E* __restrict__ z, const float* __restrict__ w, E* __restrict__ out,
     int64_t ngroups_total, int64_t groups_per_row, int64_t gs, float eps) {
+    constexpr bool kBf16 = std::is_same<E, __nv_bfloat16>::value;
     constexpr int GPB = kGateThreads / TPG;            // groups per CTA
     constexpr int WPG = TPG / 32 > 0 ? TPG / 32 : 1;   // warps per group
     __shared__ float red[kGateThreads / 32];
@@ -213,7 +223,7 @@ __global__ void __launch_bounds__(kGateThreads, 5) gated_rmsnorm_kernel(
             float a[VW], b[VW];
             load_vec(y + base + idx * VW, a);
             load_vec(z + base + idx * VW, b);
-            gate<VW>(a, b, v[i]);
+            gate<VW, kBf16>(a, b, v[i]);
 #pragma unroll
             for (int e = 0; e < VW; ++e) ss = fmaf(v[i][e], v[i][e], ss);
         }
@@ -222,7 +232,7 @@ __global__ void __launch_bounds__(kGateThreads, 5) gated_rmsnorm_kernel(
         float a[VW], b[VW], g[VW];
         load_vec(y + base + idx * VW, a);
         load_vec(z + base + idx * VW, b);
-        gate<VW>(a, b, g);
+        gate<VW, kBf16>(a, b, g);
 #pragma unroll
         for (int e = 0; e < VW; ++e) ss = fmaf(g[e], g[e], ss);
     }
@@ -253,7 +263,7 @@ __global__ void __launch_bounds__(kGateThreads, 5) gated_rmsnorm_kernel(
         float a[VW], b[VW], g[VW], o[VW];
         load_vec(y + base + idx * VW, a);
         load_vec(z + base + idx * VW, b);
-        gate<VW>(a, b, g);
+        gate<VW, kBf16>(a, b, g);
 #pragma unroll
         for (int e = 0; e < VW; ++e) o[e] = g[e] * r * w[wbase + idx * VW + e];
         store_vec(out + base + idx * VW, o);
