@@ -121,7 +121,7 @@ constexpr int64_t kTargetUnits = SSD_TARGET_UNITS;             // units wanted: 
 #define SSD_SEG_TARGET_UNITS (2 * 148)
 #endif
 // Segments whose entering states come from the segment-state pass and scan: fewer,
-// longer ones (about two waves), since every segment adds a state slot to both
+// longer ones (at most two waves), since every segment adds a state slot to both
 // passes and a pipeline fill to each of its units.
 constexpr int64_t kSegTargetUnits = SSD_SEG_TARGET_UNITS;
 #ifndef SSD_CP_TARGET_UNITS
@@ -181,12 +181,10 @@ SegPlan seg_plan(const ssd::Dims& d, Path path) {
     const int64_t chains = std::max<int64_t>(1, d.b * (d.H / sp.kh));
     // Chained segments of one chain run one after another, so with no more
     // chains than SMs splitting them only adds hand-offs to the critical path.
-    const int64_t target = sp.chained ? kTargetUnits : kSegTargetUnits;
-    int64_t nseg = (target + chains - 1) / chains;
+    // chained: at least kTargetUnits units; segmented: at most kSegTargetUnits, so
+    // that the last of the two waves is not a third one of a few units
+    int64_t nseg = sp.chained ? (kTargetUnits + chains - 1) / chains : kSegTargetUnits / chains;
     if (sp.chained && chains <= kSmCount) nseg = 1;
-#ifdef SSD_MAX_CHAINED_SEG
-    if (sp.chained) nseg = std::min<int64_t>(nseg, SSD_MAX_CHAINED_SEG);
-#endif
     if (path == Path::Segmented) nseg = std::max<int64_t>(2, nseg);
     nseg = std::max<int64_t>(1, std::min(nseg, ntiles));
     int64_t K = (ntiles + nseg - 1) / nseg;
