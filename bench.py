@@ -298,9 +298,8 @@ DECODE_METRIC = "SSD decode step (recurrent form) Mtokens/s at 2.7B layer shape,
 # workload, from one ncu capture (profiles/); None once the kernel changes
 DECODE_TRAFFIC = 614955264
 # ncu DRAM bytes (read + write) of one gate launch, one group of 5120 channels
-# (profiles/gated_rmsnorm_kernel_2.7b_layer.md); None while the kernel differs
-# from the one captured
-GATE_TRAFFIC = None
+# (profiles/gated_rmsnorm_kernel_2.7b_layer.md); the rest of out is still in L2
+GATE_TRAFFIC = 446482176
 
 
 def decode_bytes(w: W.Workload) -> float:

@@ -247,7 +247,7 @@ SSD_API ssd_status_t ssd_fwd_varlen_check(const ssd_shape_t* shape, int64_t n_do
  *     y, so y needs neither memory nor a round trip through HBM. The gate's
  *     arithmetic then runs on the kernel's four store warps, which makes the
  *     forward slower than the two separate launches (measured at the 2.7B
- *     layer shape: 0.445 ms against about 0.26 ms); it trades time for the y buffer.
+ *     layer shape: 0.444 ms against 0.258 ms); it trades time for the y buffer.
  *   fuse = 0, or a shape / group size the kernel cannot gate: y is written to
  *     the workspace and the gate kernel follows (two launches more).
  *   z                  [b, T, H, P] in dtype (16-byte aligned), the gate branch.
