@@ -919,7 +919,8 @@ def run_ours(args):
 
 
 def run_decode_only(args):
-    """--workload decode_step / gate_norm: that kernel alone, as the printed line."""
+    """--workload decode_step / gate_norm / long_context: that step alone, as the printed
+    line (long_context: ssd_fwd on the long-context workload, the segmented path)."""
     world, rank, local = dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -929,6 +930,9 @@ def run_decode_only(args):
     stream = torch.cuda.current_stream(dev)
     if args.workload == "gate_norm":
         out = measure_gate(ssd, dev, stream, args.steps, args.warmup, seed=rank)
+    elif args.workload == "long_context":
+        out = measure_workload(ssd, dev, stream, W.LONG_CONTEXT, args.steps, args.warmup, seed=rank)
+        out["metric"] = "SSD fwd Mtokens/s, long context (b1 T65536 H32 P64 N128 G8, state carry)"
     else:
         out = measure_decode(ssd, dev, stream, args.steps, args.warmup, rank,
                              world == 1 and not args.no_cpu_baseline and not args.profile)
@@ -951,16 +955,17 @@ def main():
                     help="untimed load before the timed region, for the clock samples")
     ap.add_argument("--profile", action="store_true",
                     help="warmup and timed steps only (for ncu): no e2e, no CPU baseline")
-    ap.add_argument("--workload", choices=["layer", "decode_step", "gate_norm", "long_context_cp"],
+    ap.add_argument("--workload", choices=["layer", "decode_step", "gate_norm", "long_context", "long_context_cp"],
                     default="layer",
-                    help="decode_step: time only the recurrent decoding step; long_context_cp: "
-                         "the long-context sequence split over the ranks (context parallel)")
+                    help="decode_step: time only the recurrent decoding step; long_context: one ssd_fwd "
+                         "on the long-context workload; long_context_cp: the long-context sequence split "
+                         "over the ranks (context parallel)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
-    if args.workload in ("decode_step", "gate_norm"):
+    if args.workload in ("decode_step", "gate_norm", "long_context"):
         return run_decode_only(args)
     if args.workload == "long_context_cp":
         return run_cp(args)
